@@ -1,0 +1,301 @@
+"""Pins for the fp64 oracle, each against something other than the oracle itself.
+
+* the frame-7 worked example printed on the VDN-H3 article (golden fixture);
+* the partition property of the membership ("the other frames go to the
+  linear memory": every key frame is read through exactly one branch);
+* the softmax branch against dense masked attention evaluated by the library
+  routine torch scaled_dot_product_attention, with a mask built from a token
+  predicate instead of the oracle's frame lists;
+* the one-chunk special case against plain unmasked attention;
+* the linear branch against a state-free per-pair weighted mean;
+* forward/backward states against an independent prefix/suffix chunk scan and
+  against the total-minus-window identity;
+* text counted once, zero linear branch when the window covers everything,
+  text-only closed form, gate saturation limits, the RMS invariant;
+* mutation tests: plausible slips planted in the oracle (on the CPU) make at
+  least one of the pins fail.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import bruteforce as BF
+from oracle import hybrid_attn as O
+from video_diffusion_hybrid_sparse_b200.workloads import Workload, as_float64_numpy, make_inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "frame7_membership.txt")
+
+
+def read_golden():
+    vals = {}
+    with open(GOLDEN) as fh:
+        for line in fh:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *rest = line.split()
+            vals[key] = [int(x) for x in rest]
+    return vals
+
+
+def problem_inputs(F, P, H, d, T, C, B=1, seed=0, dist="normal"):
+    w = Workload("t", B, F, P, H, d, T, C, "fp32", dist, 0)
+    x = as_float64_numpy(make_inputs(w, seed=1000 + seed))
+    prob = O.Problem(B=B, F=F, P=P, H=H, d=d, T=T, C=C)
+    return prob, x
+
+
+SMALL_CASES = [
+    # F, P, H, d, T, C
+    (15, 3, 2, 8, 4, 1),
+    (10, 2, 1, 4, 3, 2),
+    (15, 2, 2, 6, 0, 5),
+    (12, 3, 1, 8, 5, 3),
+    (3, 4, 1, 4, 2, 1),
+    (2, 3, 1, 4, 2, 1),
+    (1, 5, 1, 4, 2, 1),
+    (6, 2, 1, 4, 0, 6),
+]
+
+
+# ---------------------------------------------------------------- membership
+
+
+def test_frame7_membership_matches_page():
+    g = read_golden()
+    F, C, f = g["frames"][0], g["chunk"][0], g["query"][0]
+    assert O.softmax_frames(f, F, C) == g["softmax"]
+    assert O.forward_frames(f, F, C) == g["forward"]
+    assert O.backward_frames(f, F, C) == g["backward"]
+    row = O.membership_table(F, C)[f]
+    assert [i for i in range(F) if row[i] == O.SOFTMAX] == g["softmax"]
+    assert [i for i in range(F) if row[i] == O.FORWARD] == g["forward"]
+    assert [i for i in range(F) if row[i] == O.BACKWARD] == g["backward"]
+
+
+@pytest.mark.parametrize("F,C", [(F, C) for F in range(1, 21) for C in range(1, F + 1) if F % C == 0]
+                         + [(45, 5), (60, 5), (15, 1)])
+def test_membership_partitions_every_row(F, C):
+    t = O.membership_table(F, C)
+    assert t.shape == (F, F)
+    assert np.all(t > 0), "every key frame must be read through exactly one branch"
+    anchors = {0, F - 1}
+    for f in range(F):
+        soft = [g for g in range(F) if t[f, g] == O.SOFTMAX]
+        fwd = [g for g in range(F) if t[f, g] == O.FORWARD]
+        bwd = [g for g in range(F) if t[f, g] == O.BACKWARD]
+        assert anchors <= set(soft)
+        assert f in soft
+        assert all(g < min(set(soft) - anchors) for g in fwd)
+        assert all(g > max(set(soft) - anchors) for g in bwd)
+        # the window is whole chunks: chunk distance <= 1 exactly for softmax non-anchors
+        c = f // C
+        for g in range(F):
+            if g in anchors:
+                continue
+            near = abs(g // C - c) <= 1
+            assert (t[f, g] == O.SOFTMAX) == near
+
+
+# ---------------------------------------------------------------- softmax branch
+
+
+@pytest.mark.parametrize("case", SMALL_CASES)
+def test_softmax_branch_equals_dense_masked_sdpa(case):
+    prob, x = problem_inputs(*case, seed=hash(case) % 1000)
+    got = O.softmax_branch(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], prob)
+    ref = BF.dense_masked_softmax(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], prob)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_one_chunk_is_full_attention():
+    prob, x = problem_inputs(6, 3, 2, 8, 4, 6, seed=3)
+    got = O.softmax_branch(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], prob)
+    for h in range(prob.H):
+        q = torch.from_numpy(x["q"][0, :, h, :])
+        keys = torch.from_numpy(np.concatenate([x["k"][0, :, h, :], x["text_k"][0, :, h, :]]))
+        vals = torch.from_numpy(np.concatenate([x["v"][0, :, h, :], x["text_v"][0, :, h, :]]))
+        p = torch.softmax((q @ keys.T) / np.sqrt(prob.d), dim=-1)
+        np.testing.assert_allclose(got[0, :, h, :], (p @ vals).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_constant_values_give_constant_softmax_output():
+    prob, x = problem_inputs(15, 4, 1, 8, 3, 1, seed=5)
+    ones = np.ones_like(x["v"]) * 2.5
+    got = O.softmax_branch(x["q"], x["k"], ones, x["text_k"], np.ones_like(x["text_v"]) * 2.5, prob)
+    np.testing.assert_allclose(got, 2.5, rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------- linear branch
+
+
+@pytest.mark.parametrize("case", SMALL_CASES)
+def test_linear_branch_equals_pairwise_mean(case):
+    prob, x = problem_inputs(*case, seed=17 + hash(case) % 1000)
+    got, _ = O.linear_branch(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], prob)
+    ref = BF.pairwise_linear(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], prob)
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_phi_is_elu_plus_one():
+    x = np.linspace(-30, 30, 2001)
+    ref = torch.nn.functional.elu(torch.from_numpy(x)).numpy() + 1.0
+    np.testing.assert_allclose(O.phi(x), ref, rtol=1e-15, atol=1e-15)  # elu+1 loses digits near 0
+    assert np.all(O.phi(x) > 0)
+
+
+@pytest.mark.parametrize("F,C", [(15, 1), (45, 5), (12, 3), (60, 5)])
+def test_states_match_independent_chunk_scan(F, C):
+    """Forward state = half text + prefix over chunks <= c-2; backward = half
+    text + suffix over chunks >= c+2, anchors removed, built as a running
+    scan over chunk sums (the oracle itself sums membership sets)."""
+    rng = np.random.default_rng(F * 100 + C)
+    d = 3
+    prob = O.Problem(B=1, F=F, P=1, H=1, d=d, T=2, C=C)
+    S = rng.standard_normal((F, d, d))
+    z = rng.random((F, d))
+    S_t = rng.standard_normal((d, d))
+    z_t = rng.random(d)
+    SF, zF, SB, zB = O.directional_states(S, z, S_t, z_t, prob)
+    nc = F // C
+    chunk_S = np.zeros((nc, d, d))
+    for f in range(1, F - 1):  # anchors 0 and F-1 left out
+        chunk_S[f // C] += S[f]
+    run = np.zeros((d, d))
+    for c in range(nc):
+        if c >= 2:
+            run = run + chunk_S[c - 2]
+        np.testing.assert_allclose(SF[c], 0.5 * S_t + run, rtol=1e-12, atol=1e-12)
+    run = np.zeros((d, d))
+    for c in reversed(range(nc)):
+        if c + 2 < nc:
+            run = run + chunk_S[c + 2]
+        np.testing.assert_allclose(SB[c], 0.5 * S_t + run, rtol=1e-12, atol=1e-12)
+    # total-minus-window identity: S_F + S_B = S_t + sum_{non-anchor} S_f - sum_{window non-anchor} S_f
+    total = S_t + S[1:F - 1].sum(axis=0)
+    for c in range(nc):
+        win = [g for g in O.window_frames(c * C, F, C) if g not in (0, F - 1)]
+        np.testing.assert_allclose(SF[c] + SB[c], total - sum((S[g] for g in win), np.zeros((d, d))),
+                                   rtol=1e-12, atol=1e-12)
+
+
+def test_text_counts_once():
+    prob, x = problem_inputs(15, 3, 1, 6, 5, 1, seed=9)
+    args = (x["q"], x["k"], x["v"], x["text_k"], x["text_v"], prob)
+    half, _ = O.linear_branch(*args, text_weights=(0.5, 0.5))
+    fwd_only, _ = O.linear_branch(*args, text_weights=(1.0, 0.0))
+    both, _ = O.linear_branch(*args, text_weights=(1.0, 1.0))
+    np.testing.assert_allclose(half, fwd_only, rtol=1e-12, atol=1e-13)
+    assert np.max(np.abs(half - both)) > 1e-6
+
+
+@pytest.mark.parametrize("F,C", [(3, 1), (4, 2), (6, 3), (10, 5)])
+def test_linear_branch_empty_without_text(F, C):
+    """Window covers every non-anchor frame (3 frames, or at most two chunks):
+    with no text the linear branch is exactly zero and out = sig(g_s) o_s."""
+    prob, x = problem_inputs(F, 3, 2, 4, 0, C, seed=F + C)
+    res = O.hybrid_attn(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], x["gate_s"], x["gate_l"], prob)
+    assert np.all(res["o_l"] == 0.0)
+    sig = 1.0 / (1.0 + np.exp(-x["gate_s"]))
+    np.testing.assert_allclose(res["out"], sig * res["o_s"], rtol=1e-14, atol=0)
+
+
+def test_linear_branch_text_only_closed_form():
+    prob, x = problem_inputs(3, 4, 1, 5, 6, 1, seed=21)
+    o_l, _ = O.linear_branch(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], prob)
+    fq = torch.nn.functional.elu(torch.from_numpy(x["q"][0, :, 0, :])).numpy() + 1
+    ftk = torch.nn.functional.elu(torch.from_numpy(x["text_k"][0, :, 0, :])).numpy() + 1
+    w = fq @ ftk.T
+    ref = (w @ x["text_v"][0, :, 0, :]) / w.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(o_l[0, :, 0, :], ref, rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- gated fusion
+
+
+def test_gate_saturation_limits():
+    prob, x = problem_inputs(15, 2, 1, 8, 3, 1, seed=31)
+    base = (x["q"], x["k"], x["v"], x["text_k"], x["text_v"])
+    big = np.full_like(x["gate_s"], 40.0)
+    res = O.hybrid_attn(*base, big, -big, prob)
+    np.testing.assert_allclose(res["out"], res["o_s"], rtol=0, atol=1e-15 + 1e-16 * np.abs(res["r"]).max() * 1e3)
+    res = O.hybrid_attn(*base, -big, big, prob)
+    np.testing.assert_allclose(res["out"], res["r"], rtol=0, atol=1e-14)
+
+
+def test_rms_invariant_and_gamma():
+    prob, x = problem_inputs(15, 3, 2, 8, 3, 1, seed=41)
+    res = O.hybrid_attn(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], x["gate_s"], x["gate_l"], prob)
+    ms = np.mean(res["o_l"] ** 2, axis=-1)
+    rms_r = np.sqrt(np.mean(res["r"] ** 2, axis=-1))
+    np.testing.assert_allclose(rms_r, np.sqrt(ms / (ms + prob.eps)), rtol=1e-12)
+    gamma = np.random.default_rng(0).random((prob.H, prob.d)) + 0.5
+    res_g = O.hybrid_attn(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], x["gate_s"], x["gate_l"], prob,
+                          gamma=gamma)
+    np.testing.assert_allclose(res_g["r"], res["r"] * gamma[None, None], rtol=1e-13)
+
+
+def test_row_subset_matches_whole_call():
+    prob, x = problem_inputs(15, 5, 2, 8, 4, 1, seed=51)
+    full = O.hybrid_attn(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], x["gate_s"], x["gate_l"], prob)
+    rows = np.array([0, 4, 5, 33, 37, 74])
+    for h in range(prob.H):
+        sub = O.hybrid_attn_rows(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], x["gate_s"], x["gate_l"],
+                                 prob, 0, h, rows)
+        np.testing.assert_allclose(sub["out"], full["out"][0, rows, h, :], rtol=1e-13, atol=1e-14)
+
+
+def test_softmax_pair_count():
+    prob = O.Problem(B=1, F=15, P=7, H=1, d=4, T=3, C=1)
+    mask = BF.softmax_mask(prob)
+    assert O.softmax_pairs(prob) == int(mask.sum())
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+
+def _pins_hold():
+    """Run the cheap pins; return the list of those that fail."""
+    failed = []
+    g = read_golden()
+    if (O.softmax_frames(7, 15, 1) != g["softmax"] or O.forward_frames(7, 15, 1) != g["forward"]
+            or O.backward_frames(7, 15, 1) != g["backward"]):
+        failed.append("frame7")
+    for case in [(15, 3, 2, 8, 4, 1), (12, 3, 1, 8, 5, 3)]:
+        prob, x = problem_inputs(*case, seed=77)
+        a = (x["q"], x["k"], x["v"], x["text_k"], x["text_v"], prob)
+        if not np.allclose(O.softmax_branch(*a), BF.dense_masked_softmax(*a), rtol=1e-10, atol=1e-10):
+            failed.append("sdpa")
+        if not np.allclose(O.linear_branch(*a)[0], BF.pairwise_linear(*a), rtol=1e-9, atol=1e-10):
+            failed.append("pairwise")
+    return failed
+
+
+MUTATIONS = {
+    "anchor_in_forward": ("forward_frames",
+                          lambda f, F, C: [g for g in range(F) if g // C <= f // C - 2]),
+    "window_not_clipped": ("window_frames",
+                           lambda f, F, C: [g for g in range((f // C - 1) * C, (f // C + 2) * C) if 0 <= g < F][:3 * C]
+                           if 0 < f // C < F // C - 1 else list(range(0, min(F, 3 * C)))),
+    "no_text_halving": ("directional_states",
+                        lambda S, z, S_t, z_t, prob, tw=(0.5, 0.5): O.__dict__["_orig_directional_states"](
+                            S, z, S_t, z_t, prob, (1.0, 1.0))),
+    "transposed_state": ("frame_states",
+                         lambda k, v, prob, b, h: (lambda S, z: (np.transpose(S, (0, 2, 1)), z))(
+                             *O.__dict__["_orig_frame_states"](k, v, prob, b, h))),
+    "phi_plain_exp": ("phi", lambda x: np.exp(np.asarray(x, np.float64))),
+    "softmax_frames_drop_last_anchor": ("softmax_frames",
+                                        lambda f, F, C: sorted(set(O.window_frames(f, F, C)) | {0})),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    fn_name, bad = MUTATIONS[name]
+    monkeypatch.setitem(O.__dict__, "_orig_directional_states", O.directional_states)
+    monkeypatch.setitem(O.__dict__, "_orig_frame_states", O.frame_states)
+    assert _pins_hold() == []
+    monkeypatch.setattr(O, fn_name, bad)
+    assert _pins_hold() != [], f"planted mistake {name} went unnoticed"
