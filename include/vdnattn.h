@@ -1,0 +1,160 @@
+/*
+ * vdnattn.h - C ABI of libvdnattn, the sm_100a (B200) implementation of the
+ * VDN-H3 dual-branch hybrid attention.
+ *
+ * Source of the operation: the VDN-H3 article (tahou.com, article
+ * 216474224916730885), section "技术核心设计 / 双分支混合注意力机制" (the
+ * softmax branch over a chunk window plus boundary anchors plus text; the
+ * bidirectional frame-wise linear memory with half-weight text; the frame-7
+ * example) and section "自适应门控融合双分支输出" (RMSNorm on the linear
+ * branch, one sigmoid gate per branch, sum of the two).
+ *
+ * The call computes, for every video query token i (batch b, head h):
+ *
+ *   o_s[i] = softmax over keys J(i) of (scale * q_i . k_j), applied to v_j,
+ *            J(i) = tokens of the frames in the window of i's chunk (the chunk
+ *            and its two neighbours, clipped at the ends) and of the first and
+ *            last frame, each frame once, plus all text tokens;
+ *   o_l[i] = phi(q_i)^T (S_F + S_B) / (phi(q_i) . (z_F + z_B)), phi = elu + 1,
+ *            S_F/z_F summing phi(k) v^T / phi(k) over the chunks before the
+ *            window, S_B/z_B over the chunks after it, both without the two
+ *            anchor frames, each holding half of the text state; o_l = 0 when
+ *            the states hold no token;
+ *   r[i]   = o_l[i] / sqrt(mean_d(o_l[i]^2) + eps) * gamma[h];
+ *   out[i] = sigmoid(gate_s[i]) * o_s[i] + sigmoid(gate_l[i]) * r[i].
+ *
+ * Layouts (row-major, no padding between rows):
+ *   q, k, v, gate_s, gate_l, out : [batch, frames*tokens_per_frame, heads, head_dim]
+ *   text_k, text_v               : [batch, text_tokens, heads, head_dim]
+ *   token n of a video tensor lies in latent frame n / tokens_per_frame.
+ * All of these are DEVICE pointers in the dtype given by vdn_cfg.dtype, each
+ * 16-byte aligned; the caller owns them.  Accumulation is always fp32; tensor
+ * core operands are bf16 (fp32 inputs are rounded to bf16 before the
+ * contractions, and the intermediate softmax output o_s is kept in bf16).
+ *
+ * Ownership and threading: the library allocates no device memory.  Scratch
+ * space is the caller-owned workspace (vdn_workspace_bytes).  Every device
+ * function enqueues its work on the given stream and returns without host
+ * synchronisation; the caller keeps inputs, outputs and the workspace alive
+ * until that work completes.  Two calls that share a workspace must be
+ * ordered on the GPU.  Functions are thread-safe.
+ *
+ * Errors: every argument check happens before anything is enqueued; on an
+ * error return nothing was launched.  VDN_ERR_CUDA reports a launch error
+ * (cudaGetLastError).  A kernel whose bounded wait runs out (about 2 s)
+ * writes VDN_ERR_TIMEOUT into *status_word (when given) and returns early;
+ * that is read by the caller after synchronising.
+ */
+#ifndef VDNATTN_H
+#define VDNATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define VDN_API __attribute__((visibility("default")))
+#else
+#define VDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VDN_OK = 0,
+  VDN_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, frames % chunk != 0 */
+  VDN_ERR_UNSUPPORTED = 2, /* head_dim not 32/64/128, unknown dtype, too many chunks */
+  VDN_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte aligned */
+  VDN_ERR_WORKSPACE = 4,   /* workspace NULL or smaller than vdn_workspace_bytes */
+  VDN_ERR_CUDA = 5,        /* a CUDA runtime call or launch failed */
+  VDN_ERR_TIMEOUT = 6      /* written to status_word by a kernel whose wait ran out */
+} vdn_status;
+
+typedef enum { VDN_BF16 = 0, VDN_FP32 = 1 } vdn_dtype;
+
+/* debug_flags: what vdn_readout_merge writes into out instead of the merge. */
+enum {
+  VDN_OUT_SOFTMAX_ONLY = 1, /* out = o_s (no gate) */
+  VDN_OUT_LINEAR_ONLY = 2,  /* out = r, the RMS-normalised linear read (no gate) */
+  VDN_OUT_LINEAR_RAW = 4,   /* out = o_l, the linear read before RMSNorm */
+  VDN_EXPORT_STATES = 8     /* vdn_state_scan also writes S_F/z_F and S_B/z_B (fp32) */
+};
+
+typedef struct {
+  int32_t batch;            /* B  >= 1 */
+  int32_t frames;           /* F  >= 1, latent frames; anchors are frames 0 and F-1 */
+  int32_t tokens_per_frame; /* P  >= 1 */
+  int32_t heads;            /* H  >= 1 */
+  int32_t head_dim;         /* d in {32, 64, 128} */
+  int32_t text_tokens;      /* T  >= 0 */
+  int32_t chunk_frames;     /* C  >= 1, F % C == 0 (5 in the article's chunking, 1 in its frame-7 example) */
+  int32_t dtype;            /* vdn_dtype of q, k, v, text, gates and out */
+  float softmax_scale;      /* <= 0 selects 1/sqrt(head_dim) */
+  float rms_eps;            /* < 0 selects 1e-6 */
+  const float* rms_weight;  /* device [heads, head_dim] fp32 gamma, or NULL for ones */
+  int32_t debug_flags;      /* VDN_OUT_* / VDN_EXPORT_STATES, 0 in production */
+  int32_t reserved0;        /* must be 0 */
+  void* workspace;          /* device, 256-byte aligned, >= vdn_workspace_bytes(cfg) bytes */
+  size_t workspace_bytes;
+  int32_t* status_word;     /* optional device int32; set to VDN_ERR_TIMEOUT by a kernel that gave up */
+  float* export_fwd;        /* VDN_EXPORT_STATES: device [B, F/C, H, d+1, d] fp32; row d holds z */
+  float* export_bwd;        /* same layout, backward states */
+} vdn_cfg;
+
+/* Library version, (major << 16) | minor. */
+VDN_API int32_t vdn_version(void);
+
+/* Human-readable name of a status code (static string). */
+VDN_API const char* vdn_status_string(vdn_status s);
+
+/* Host-only argument check of cfg (sizes, dtype, head_dim, chunking).  No CUDA call. */
+VDN_API vdn_status vdn_validate(const vdn_cfg* cfg);
+
+/* Bytes of workspace a call with this cfg needs; 0 if cfg is invalid.  No CUDA call. */
+VDN_API size_t vdn_workspace_bytes(const vdn_cfg* cfg);
+
+/* Host-only membership table of the frame-7 rule: table[f*F + g] = 1 when query
+ * frame f reads key frame g through the softmax branch, 2 through the forward
+ * state, 3 through the backward state.  table is HOST memory of F*F bytes. */
+VDN_API vdn_status vdn_plan_membership(const vdn_cfg* cfg, uint8_t* table);
+
+/* The same table produced on the GPU by the index logic the kernels use
+ * (KV ranges of the softmax kernel, chunk membership of the scan).
+ * table_dev is DEVICE memory of F*F bytes.  stream is a cudaStream_t. */
+VDN_API vdn_status vdn_membership_device(const vdn_cfg* cfg, uint8_t* table_dev, void* stream);
+
+/* Whole call: staging (fp32 or head_dim 32 only), state build, scan, sparse
+ * softmax, readout + merge, all on stream.  out: [B, N, H, d] in dtype. */
+VDN_API vdn_status vdn_hybrid_attn_fwd(const void* q, const void* k, const void* v,
+                               const void* text_k, const void* text_v,
+                               const void* gate_s, const void* gate_l, void* out,
+                               const vdn_cfg* cfg, void* stream);
+
+/* The steps of vdn_hybrid_attn_fwd, for callers that schedule them
+ * separately (e.g. the linear steps on a second stream).  Run in this order:
+ * vdn_stage_inputs (required first when dtype is fp32 or head_dim is 32;
+ * otherwise a no-op), then vdn_state_build -> vdn_state_scan, and
+ * vdn_sparse_softmax, in either order, then vdn_readout_merge.  Each reads
+ * what the earlier steps left in the workspace. */
+VDN_API vdn_status vdn_stage_inputs(const void* q, const void* k, const void* v,
+                            const void* text_k, const void* text_v,
+                            const vdn_cfg* cfg, void* stream);
+/* Per-frame-slice partial states [S | z] = phi(K)^T [V | 1] (tensor cores). */
+VDN_API vdn_status vdn_state_build(const void* k, const void* v, const void* text_k,
+                           const void* text_v, const vdn_cfg* cfg, void* stream);
+/* Forward/backward chunk states and their sum M_c, fp32 scan. */
+VDN_API vdn_status vdn_state_scan(const vdn_cfg* cfg, void* stream);
+/* Block-sparse softmax branch o_s (window + anchors + text) into the workspace. */
+VDN_API vdn_status vdn_sparse_softmax(const void* q, const void* k, const void* v,
+                              const void* text_k, const void* text_v,
+                              const vdn_cfg* cfg, void* stream);
+/* phi(Q) M_c readout, RMSNorm, gates and merge into out. */
+VDN_API vdn_status vdn_readout_merge(const void* q, const void* gate_s, const void* gate_l,
+                             void* out, const vdn_cfg* cfg, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VDNATTN_H */

@@ -1,0 +1,125 @@
+"""Host-only checks of the C ABI (no GPU needed, no kernel launched).
+
+* the shared library loads and exports every function include/vdnattn.h declares;
+* argument validation returns the documented status codes before any CUDA call;
+* the host membership table equals the oracle's, bit for bit, on the workload
+  shapes and on edge cases (one to three frames, one chunk, many chunks).
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import hybrid_attn as O
+from video_diffusion_hybrid_sparse_b200 import binding as vb
+from video_diffusion_hybrid_sparse_b200.workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vdnattn.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"VDN_API\s+[\w\s\*]+?\b(vdn_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    lib = vb.library()
+    names = declared_functions()
+    assert len(names) >= 12
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(vb.EXPORTED)
+
+
+def test_version_and_status_strings():
+    lib = vb.library()
+    assert lib.vdn_version() >> 16 == 1
+    for code, text in vb.STATUS.items():
+        assert lib.vdn_status_string(code).decode() == text
+
+
+def shape(**kw):
+    base = dict(B=1, F=15, P=16, H=2, d=64, T=8, C=1, fp32=False)
+    base.update(kw)
+    return vb.Shape(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(), 0),
+    (dict(F=16, C=5), 1),          # frames not a whole number of chunks
+    (dict(d=48), 2),               # unsupported head_dim
+    (dict(d=256), 2),
+    (dict(T=-1), 1),
+    (dict(B=0), 1),
+    (dict(P=0), 1),
+    (dict(F=200, C=1), 2),         # more chunks than the scan keeps on chip
+    (dict(d=32, fp32=True), 0),
+    (dict(d=128, F=60, C=5, P=4032, H=24, T=512), 0),
+])
+def test_validate_codes(kw, code):
+    assert vb.validate(shape(**kw)) == code
+
+
+def test_validate_rejects_unknown_dtype_and_flags():
+    lib = vb.library()
+    cfg = vb.make_cfg(shape())
+    cfg.dtype = 7
+    assert lib.vdn_validate(ctypes.byref(cfg)) == 2
+    cfg = vb.make_cfg(shape(), debug_flags=64)
+    assert lib.vdn_validate(ctypes.byref(cfg)) == 1
+    cfg = vb.make_cfg(shape())
+    cfg.reserved0 = 3
+    assert lib.vdn_validate(ctypes.byref(cfg)) == 1
+    assert lib.vdn_validate(None) == 1
+
+
+def test_workspace_bytes():
+    for w in WORKLOADS:
+        n = vb.workspace_bytes(vb.Shape(w.B, w.F, w.P, w.H, w.d, w.T, w.C, w.dtype == "fp32"))
+        o_s = w.B * w.N * w.H * max(64, w.d) * 2
+        assert n > o_s
+        assert n % 1024 == 0
+    assert vb.library().vdn_workspace_bytes(ctypes.byref(vb.make_cfg(shape(F=16, C=5)))) == 0
+
+
+def test_call_errors_before_any_launch():
+    """Bad workspace / pointers are reported without touching the GPU."""
+    lib = vb.library()
+    s = shape()
+    cfg = vb.make_cfg(s)  # no workspace
+    p = 1 << 20  # aligned fake device addresses; never dereferenced on these paths
+    args = [p, p, p, p, p, p, p, p]
+    assert lib.vdn_hybrid_attn_fwd(*args, ctypes.byref(cfg), None) == 4
+    cfg.workspace = p
+    cfg.workspace_bytes = 16
+    assert lib.vdn_hybrid_attn_fwd(*args, ctypes.byref(cfg), None) == 4
+    cfg.workspace_bytes = vb.workspace_bytes(s)
+    cfg.workspace = p + 128  # workspace must be 256-byte aligned
+    assert lib.vdn_hybrid_attn_fwd(*args, ctypes.byref(cfg), None) == 3
+    cfg.workspace = p
+    bad = list(args)
+    bad[1] = p + 8  # k misaligned
+    assert lib.vdn_hybrid_attn_fwd(*bad, ctypes.byref(cfg), None) == 3
+    bad = list(args)
+    bad[0] = None  # q missing
+    assert lib.vdn_hybrid_attn_fwd(*bad, ctypes.byref(cfg), None) == 1
+    bad = list(args)
+    bad[3] = None  # text_k missing while T > 0
+    assert lib.vdn_hybrid_attn_fwd(*bad, ctypes.byref(cfg), None) == 1
+    cfg.debug_flags = vb.EXPORT_STATES  # export requested without buffers
+    assert lib.vdn_hybrid_attn_fwd(*args, ctypes.byref(cfg), None) == 1
+    assert lib.vdn_state_scan(ctypes.byref(cfg), None) == 1
+    cfg.debug_flags = 0
+    assert lib.vdn_plan_membership(ctypes.byref(cfg), None) == 1
+
+
+EDGE = [(1, 1), (2, 1), (2, 2), (3, 1), (3, 3), (4, 2), (5, 1), (6, 3), (15, 1), (15, 5), (45, 5), (60, 5),
+        (60, 1), (10, 10), (96, 1)]
+
+
+@pytest.mark.parametrize("F,C", EDGE + [(w.F, w.C) for w in WORKLOADS])
+def test_host_membership_matches_oracle(F, C):
+    np.testing.assert_array_equal(vb.plan_membership(F, C), O.membership_table(F, C))

@@ -1,0 +1,211 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Tolerances (stated for the merged output): max-abs 2e-2 and relative L2
+1e-2; membership tables bit-exact.  Branch outputs read through the debug
+modes use the same relative-L2 bound and a max-abs bound scaled by the
+branch's own magnitude.  Exported forward/backward states: relative L2
+1e-2 (phi(k) is rounded to bf16 for the tensor cores, a relative error of
+2^-9 per term).
+
+Small shapes are checked element by element over the whole output; the
+workload shapes too large for the host oracle are checked on sampled rows
+(chunk edges, ragged tile tails, random rows) of sampled heads, computed by
+the oracle one row set at a time.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import hybrid_attn as O
+from video_diffusion_hybrid_sparse_b200 import binding as vb
+from video_diffusion_hybrid_sparse_b200.workloads import BY_NAME, Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_ABS, TOL_REL = 2e-2, 1e-2
+NAMES = ["q", "k", "v", "text_k", "text_v", "gate_s", "gate_l"]
+
+
+def rel_l2(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def assert_close(got, ref, what, abs_tol=TOL_ABS, rel_tol=TOL_REL):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = np.abs(got - ref)
+    i = np.unravel_index(np.argmax(err), err.shape)
+    assert err[i] <= abs_tol, f"{what}: max-abs {err[i]:.3e} at {i} (got {got[i]}, ref {ref[i]})"
+    r = rel_l2(got, ref)
+    assert r <= rel_tol, f"{what}: rel-L2 {r:.3e}"
+
+
+def to_dev(inputs):
+    return {k: t.cuda() for k, t in inputs.items()}
+
+
+def run(w: Workload, dev, **kw):
+    out = vb.hybrid_attn_fwd(dev["q"], dev["k"], dev["v"], dev["text_k"], dev["text_v"], dev["gate_s"],
+                             dev["gate_l"], frames=w.F, chunk_frames=w.C, **kw)
+    torch.cuda.synchronize()
+    return out
+
+
+def np64(t):
+    return t.to(torch.float64).cpu().numpy()
+
+
+def oracle_full(w: Workload, inputs, gamma=None):
+    x = {k: np64(t) for k, t in inputs.items()}
+    prob = O.Problem(B=w.B, F=w.F, P=w.P, H=w.H, d=w.d, T=w.T, C=w.C)
+    return O.hybrid_attn(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], x["gate_s"], x["gate_l"], prob,
+                         gamma=gamma)
+
+
+# ----------------------------------------------------------------- membership
+
+
+@pytest.mark.parametrize("F,C,P,T", [(15, 1, 16, 8), (45, 5, 4, 3), (60, 5, 3, 0), (1, 1, 5, 2), (2, 1, 5, 2),
+                                     (3, 1, 5, 0), (6, 6, 2, 1), (12, 3, 2, 2), (96, 1, 1, 1)])
+def test_device_membership_matches_oracle(F, C, P, T):
+    np.testing.assert_array_equal(vb.membership_device(F, C, P, T), O.membership_table(F, C))
+
+
+# ----------------------------------------------------------------- whole outputs, small shapes
+
+
+SMALL = [
+    BY_NAME["tiny_fp32"],
+    BY_NAME["small_bf16"],
+    # ragged frames (P not a multiple of 128), two batches, text not a multiple of 128
+    Workload("ragged", 2, 15, 200, 2, 128, 70, 1, "bf16", "normal", 11),
+    Workload("c5_ragged", 1, 10, 130, 2, 128, 40, 5, "bf16", "half", 12),
+    Workload("one_frame", 1, 1, 150, 2, 64, 20, 1, "bf16", "normal", 13),
+    Workload("two_frames", 1, 2, 100, 2, 64, 9, 1, "bf16", "normal", 14),
+    Workload("three_frames_no_text", 1, 3, 90, 2, 128, 0, 1, "bf16", "normal", 15),
+    Workload("one_chunk", 1, 6, 64, 2, 128, 33, 6, "bf16", "normal", 16),
+    Workload("two_chunks_no_text", 1, 4, 64, 1, 64, 0, 2, "bf16", "normal", 17),
+    Workload("d32_bf16", 1, 15, 40, 3, 32, 5, 1, "bf16", "normal", 18),
+    Workload("d64_fp32", 1, 9, 50, 2, 64, 7, 3, "fp32", "normal", 19),
+    Workload("d128_fp32", 1, 5, 300, 1, 128, 130, 1, "fp32", "rms", 20),
+    Workload("tiny_tokens", 1, 7, 1, 2, 64, 1, 1, "bf16", "normal", 21),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
+def test_full_output_matches_oracle(w):
+    inputs = make_inputs(w)
+    dev = to_dev(inputs)
+    ref = oracle_full(w, inputs)
+    out = run(w, dev)
+    assert_close(out.float().cpu().numpy(), ref["out"], f"{w.name} out")
+
+
+@pytest.mark.parametrize("w", SMALL[:4], ids=[w.name for w in SMALL[:4]])
+def test_branches_match_oracle(w):
+    inputs = make_inputs(w)
+    dev = to_dev(inputs)
+    ref = oracle_full(w, inputs)
+    o_s = run(w, dev, debug_flags=vb.OUT_SOFTMAX_ONLY).float().cpu().numpy()
+    assert_close(o_s, ref["o_s"], f"{w.name} o_s")
+    r = run(w, dev, debug_flags=vb.OUT_LINEAR_ONLY).float().cpu().numpy()
+    assert_close(r, ref["r"], f"{w.name} r", abs_tol=3e-2)
+    o_l = run(w, dev, debug_flags=vb.OUT_LINEAR_RAW).float().cpu().numpy()
+    scale = np.abs(ref["o_l"]).max()
+    assert_close(o_l, ref["o_l"], f"{w.name} o_l", abs_tol=TOL_ABS * scale)
+
+
+@pytest.mark.parametrize("w", [SMALL[0], SMALL[2], SMALL[3]], ids=["tiny", "ragged", "c5_ragged"])
+def test_exported_states_match_oracle(w):
+    inputs = make_inputs(w)
+    dev = to_dev(inputs)
+    ref = oracle_full(w, inputs)
+    nc = w.F // w.C
+    fwd = torch.zeros((w.B, nc, w.H, w.d + 1, w.d), dtype=torch.float32, device="cuda")
+    bwd = torch.zeros_like(fwd)
+    run(w, dev, debug_flags=vb.EXPORT_STATES, export=(fwd, bwd))
+    fwd, bwd = fwd.cpu().numpy(), bwd.cpu().numpy()
+    for b in range(w.B):
+        for h in range(w.H):
+            st = ref["states"][(b, h)]
+            # exported layout: row a' < d holds S[:, a'] (value column a'), row d holds z
+            ref_f = np.concatenate([st["SF"].transpose(0, 2, 1), st["zF"][:, None, :]], axis=1)
+            ref_b = np.concatenate([st["SB"].transpose(0, 2, 1), st["zB"][:, None, :]], axis=1)
+            assert rel_l2(fwd[b, :, h], ref_f) <= 1e-2
+            assert rel_l2(bwd[b, :, h], ref_b) <= 1e-2
+            if w.T > 0:  # chunk 0's forward state holds nothing but half of the text state
+                assert rel_l2(fwd[b, 0, h, :w.d, :], 0.5 * st["S_t"].T) <= 1e-2
+
+
+def test_rms_weight_gamma():
+    w = SMALL[2]
+    inputs = make_inputs(w)
+    dev = to_dev(inputs)
+    gamma = torch.rand((w.H, w.d), generator=torch.Generator("cpu").manual_seed(5)) + 0.5
+    ref = oracle_full(w, inputs, gamma=gamma.double().numpy())
+    out = run(w, dev, rms_weight=gamma.cuda())
+    assert_close(out.float().cpu().numpy(), ref["out"], "gamma out")
+
+
+def test_steps_equal_whole_call_and_deterministic():
+    w = BY_NAME["small_bf16"]
+    dev = to_dev(make_inputs(w))
+    a = run(w, dev).clone()
+    b = run(w, dev).clone()
+    assert torch.equal(a, b), "two calls differ"
+    out = torch.empty_like(dev["q"])
+    steps = vb.Steps(dev["q"], dev["k"], dev["v"], dev["text_k"], dev["text_v"], dev["gate_s"], dev["gate_l"], out,
+                     frames=w.F, chunk_frames=w.C)
+    steps.all()
+    torch.cuda.synchronize()
+    assert torch.equal(out, a)
+
+
+def test_status_word_stays_clear():
+    w = SMALL[2]
+    dev = to_dev(make_inputs(w))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    run(w, dev, status=status)
+    assert int(status.item()) == 0
+
+
+# ----------------------------------------------------------------- workload shapes, sampled rows
+
+
+def sample_rows(w: Workload, rng, n_random=24):
+    rpc = w.C * w.P
+    rows = set()
+    for c in range(w.F // w.C):
+        base = c * rpc
+        rows.update({base, base + rpc - 1})
+        last_tile = (rpc - 1) // 128 * 128
+        rows.update({base + last_tile, base + min(rpc - 1, last_tile + 1)})
+    rows.update(rng.integers(0, w.N, n_random).tolist())
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("name,heads", [("chunk5_bf16", [0, 15]), ("768p_bf16", [0, 23]),
+                                        ("768p_long_bf16", [7])])
+def test_workload_sampled_rows(name, heads):
+    w = BY_NAME[name]
+    inputs = make_inputs(w)
+    dev = to_dev(inputs)
+    out = run(w, dev)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out2 = run(w, dev, status=status)
+    assert torch.equal(out, out2)
+    assert int(status.item()) == 0
+    del dev
+    rng = np.random.default_rng(7)
+    rows = sample_rows(w, rng)
+    prob = O.Problem(B=1, F=w.F, P=w.P, H=1, d=w.d, T=w.T, C=w.C)
+    for h in heads:
+        x = {k: np64(t[:, :, h:h + 1, :]) for k, t in inputs.items()}
+        ref = O.hybrid_attn_rows(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], x["gate_s"], x["gate_l"],
+                                 prob, 0, 0, rows)
+        got = out[0, torch.from_numpy(rows).cuda(), h, :].float().cpu().numpy()
+        assert_close(got, ref["out"], f"{name} head {h}")

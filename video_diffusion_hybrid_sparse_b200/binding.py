@@ -1,0 +1,247 @@
+"""ctypes binding of libvdnattn (argument marshalling only).
+
+Every step of the hybrid attention runs in the library's CUDA kernels; this
+module only turns torch tensors into pointers, fills the ``vdn_cfg`` struct,
+passes the current CUDA stream and maps status codes to exceptions.  It
+raises if the library has not been built: there is no other path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvdnattn.so")
+_lib = None
+
+VDN_BF16, VDN_FP32 = 0, 1
+OUT_SOFTMAX_ONLY, OUT_LINEAR_ONLY, OUT_LINEAR_RAW, EXPORT_STATES = 1, 2, 4, 8
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "pointer not aligned",
+          4: "workspace missing or too small", 5: "CUDA error", 6: "device wait timed out"}
+
+EXPORTED = ["vdn_version", "vdn_status_string", "vdn_validate", "vdn_workspace_bytes", "vdn_plan_membership",
+            "vdn_membership_device", "vdn_hybrid_attn_fwd", "vdn_stage_inputs", "vdn_state_build",
+            "vdn_state_scan", "vdn_sparse_softmax", "vdn_readout_merge"]
+
+
+class VdnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, 'unknown')} (status {code})")
+        self.code = code
+
+
+class VdnCfg(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("frames", ctypes.c_int32), ("tokens_per_frame", ctypes.c_int32),
+        ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("text_tokens", ctypes.c_int32),
+        ("chunk_frames", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float), ("rms_eps", ctypes.c_float),
+        ("rms_weight", ctypes.c_void_p),
+        ("debug_flags", ctypes.c_int32), ("reserved0", ctypes.c_int32),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("status_word", ctypes.c_void_p),
+        ("export_fwd", ctypes.c_void_p), ("export_bwd", ctypes.c_void_p),
+    ]
+
+
+def library() -> ctypes.CDLL:
+    """Load libvdnattn.so from the package directory (raises if not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                               "`python -m video_diffusion_hybrid_sparse_b200.build`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        C = ctypes.POINTER(VdnCfg)
+        lib.vdn_version.restype = ctypes.c_int32
+        lib.vdn_status_string.restype = ctypes.c_char_p
+        lib.vdn_status_string.argtypes = [ctypes.c_int]
+        lib.vdn_validate.argtypes = [C]
+        lib.vdn_workspace_bytes.restype = ctypes.c_size_t
+        lib.vdn_workspace_bytes.argtypes = [C]
+        lib.vdn_plan_membership.argtypes = [C, P]
+        lib.vdn_membership_device.argtypes = [C, P, P]
+        lib.vdn_hybrid_attn_fwd.argtypes = [P, P, P, P, P, P, P, P, C, P]
+        lib.vdn_stage_inputs.argtypes = [P, P, P, P, P, C, P]
+        lib.vdn_state_build.argtypes = [P, P, P, P, C, P]
+        lib.vdn_state_scan.argtypes = [C, P]
+        lib.vdn_sparse_softmax.argtypes = [P, P, P, P, P, C, P]
+        lib.vdn_readout_merge.argtypes = [P, P, P, P, C, P]
+        for name in EXPORTED:
+            if name not in ("vdn_version", "vdn_status_string", "vdn_workspace_bytes"):
+                getattr(lib, name).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+@dataclass
+class Shape:
+    """Sizes of one call: batch, latent frames, tokens per frame, heads,
+    head_dim, text tokens, frames per chunk."""
+    B: int
+    F: int
+    P: int
+    H: int
+    d: int
+    T: int
+    C: int
+    fp32: bool = False
+
+    @property
+    def N(self) -> int:
+        return self.F * self.P
+
+
+def make_cfg(s: Shape, *, softmax_scale: float = 0.0, rms_eps: float = -1.0, rms_weight=None,
+             debug_flags: int = 0, workspace=None, status=None, export=None) -> VdnCfg:
+    cfg = VdnCfg()
+    cfg.batch, cfg.frames, cfg.tokens_per_frame = s.B, s.F, s.P
+    cfg.heads, cfg.head_dim, cfg.text_tokens, cfg.chunk_frames = s.H, s.d, s.T, s.C
+    cfg.dtype = VDN_FP32 if s.fp32 else VDN_BF16
+    cfg.softmax_scale = softmax_scale
+    cfg.rms_eps = rms_eps
+    cfg.rms_weight = _ptr(rms_weight)
+    cfg.debug_flags = debug_flags
+    cfg.reserved0 = 0
+    if workspace is not None:
+        cfg.workspace = workspace.data_ptr()
+        cfg.workspace_bytes = workspace.numel() * workspace.element_size()
+    cfg.status_word = _ptr(status)
+    if export is not None:
+        cfg.export_fwd = export[0].data_ptr()
+        cfg.export_bwd = export[1].data_ptr()
+    return cfg
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise VdnError(code, where)
+
+
+def _stream(stream=None) -> int:
+    return (stream if stream is not None else torch.cuda.current_stream()).cuda_stream
+
+
+def shape_of(q: torch.Tensor, text_k: torch.Tensor, frames: int, chunk_frames: int) -> Shape:
+    B, N, H, d = q.shape
+    if N % frames:
+        raise ValueError("video tokens must be frames * tokens_per_frame")
+    return Shape(B, frames, N // frames, H, d, text_k.shape[1], chunk_frames, q.dtype == torch.float32)
+
+
+def workspace_bytes(s: Shape) -> int:
+    n = library().vdn_workspace_bytes(ctypes.byref(make_cfg(s)))
+    if n == 0:
+        _check(library().vdn_validate(ctypes.byref(make_cfg(s))), "vdn_workspace_bytes")
+    return n
+
+
+_WS: dict = {}
+
+
+def workspace_for(s: Shape, device) -> torch.Tensor:
+    """A cached device workspace large enough for shape s."""
+    n = workspace_bytes(s)
+    dev = torch.device(device)
+    key = (dev.index if dev.index is not None else torch.cuda.current_device())
+    buf = _WS.get(key)
+    if buf is None or buf.numel() < n:
+        buf = torch.empty(n, dtype=torch.uint8, device=dev)
+        _WS[key] = buf
+    return buf
+
+
+def hybrid_attn_fwd(q, k, v, text_k, text_v, gate_s, gate_l, *, frames: int, chunk_frames: int, out=None,
+                    softmax_scale: float = 0.0, rms_eps: float = -1.0, rms_weight=None, debug_flags: int = 0,
+                    workspace=None, status=None, export=None, stream=None) -> torch.Tensor:
+    """The whole hybrid attention call on the current CUDA stream.
+
+    q, k, v, gate_s, gate_l: [B, F*P, H, d]; text_k, text_v: [B, T, H, d];
+    all contiguous CUDA tensors of one dtype (bf16 or fp32)."""
+    s = shape_of(q, text_k, frames, chunk_frames)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = workspace_for(s, q.device)
+    cfg = make_cfg(s, softmax_scale=softmax_scale, rms_eps=rms_eps, rms_weight=rms_weight,
+                   debug_flags=debug_flags, workspace=workspace, status=status, export=export)
+    code = library().vdn_hybrid_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(text_k), _ptr(text_v),
+                                         gate_s.data_ptr(), gate_l.data_ptr(), out.data_ptr(),
+                                         ctypes.byref(cfg), _stream(stream))
+    _check(code, "vdn_hybrid_attn_fwd")
+    return out
+
+
+class Steps:
+    """The separately scheduled steps of one call (same arguments as
+    :func:`hybrid_attn_fwd`), for per-kernel timing and stream overlap."""
+
+    def __init__(self, q, k, v, text_k, text_v, gate_s, gate_l, out, *, frames, chunk_frames, workspace=None,
+                 debug_flags=0, rms_weight=None, export=None, status=None):
+        self.t = (q, k, v, text_k, text_v, gate_s, gate_l, out)
+        self.s = shape_of(q, text_k, frames, chunk_frames)
+        self.ws = workspace if workspace is not None else workspace_for(self.s, q.device)
+        self.cfg = make_cfg(self.s, workspace=self.ws, debug_flags=debug_flags, rms_weight=rms_weight,
+                            export=export, status=status)
+        self.lib = library()
+
+    def stage(self, stream=None):
+        q, k, v, tk, tv = self.t[:5]
+        _check(self.lib.vdn_stage_inputs(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(tk), _ptr(tv),
+                                         ctypes.byref(self.cfg), _stream(stream)), "vdn_stage_inputs")
+
+    def state_build(self, stream=None):
+        _, k, v, tk, tv = self.t[:5]
+        _check(self.lib.vdn_state_build(k.data_ptr(), v.data_ptr(), _ptr(tk), _ptr(tv), ctypes.byref(self.cfg),
+                                        _stream(stream)), "vdn_state_build")
+
+    def state_scan(self, stream=None):
+        _check(self.lib.vdn_state_scan(ctypes.byref(self.cfg), _stream(stream)), "vdn_state_scan")
+
+    def sparse_softmax(self, stream=None):
+        q, k, v, tk, tv = self.t[:5]
+        _check(self.lib.vdn_sparse_softmax(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(tk), _ptr(tv),
+                                           ctypes.byref(self.cfg), _stream(stream)), "vdn_sparse_softmax")
+
+    def readout_merge(self, stream=None):
+        q, gs, gl, out = self.t[0], self.t[5], self.t[6], self.t[7]
+        _check(self.lib.vdn_readout_merge(q.data_ptr(), gs.data_ptr(), gl.data_ptr(), out.data_ptr(),
+                                          ctypes.byref(self.cfg), _stream(stream)), "vdn_readout_merge")
+
+    def all(self, stream=None):
+        self.stage(stream)
+        self.state_build(stream)
+        self.state_scan(stream)
+        self.sparse_softmax(stream)
+        self.readout_merge(stream)
+
+
+def plan_membership(F: int, C: int) -> np.ndarray:
+    """Host membership table from the library (1 softmax, 2 forward, 3 backward)."""
+    s = Shape(1, F, 1, 1, 64, 0, C)
+    table = np.zeros((F, F), dtype=np.uint8)
+    _check(library().vdn_plan_membership(ctypes.byref(make_cfg(s)), table.ctypes.data), "vdn_plan_membership")
+    return table
+
+
+def membership_device(F: int, C: int, P: int = 1, T: int = 0, device="cuda") -> np.ndarray:
+    """The membership table as the kernels' index logic produces it on the GPU."""
+    s = Shape(1, F, P, 1, 64, T, C)
+    table = torch.zeros((F, F), dtype=torch.uint8, device=device)
+    _check(library().vdn_membership_device(ctypes.byref(make_cfg(s)), table.data_ptr(), _stream()),
+           "vdn_membership_device")
+    torch.cuda.synchronize()
+    return table.cpu().numpy()
+
+
+def validate(s: Shape, **kw) -> int:
+    """Status code of the host-side argument check (no CUDA call)."""
+    return library().vdn_validate(ctypes.byref(make_cfg(s, **kw)))

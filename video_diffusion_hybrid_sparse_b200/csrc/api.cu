@@ -1,0 +1,381 @@
+// api.cu - host side of libvdnattn: argument checks, geometry and workspace
+// layout, the host membership table, TMA descriptors and the launch sequence
+// of the hybrid attention (declared in include/vdnattn.h).
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <numeric>
+#include <vector>
+
+#include "kernels.h"
+#include "vdnattn.h"
+
+namespace vdn {
+namespace {
+
+constexpr int kMaxScanChunks = 96;  // chunk sums of the scan live in shared memory
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+vdn_status make_geom(const vdn_cfg* cfg, Geom& g) {
+  if (!cfg) return VDN_ERR_INVALID_ARG;
+  if (cfg->batch < 1 || cfg->frames < 1 || cfg->tokens_per_frame < 1 || cfg->heads < 1 || cfg->text_tokens < 0 ||
+      cfg->chunk_frames < 1 || cfg->reserved0 != 0)
+    return VDN_ERR_INVALID_ARG;
+  if (cfg->frames % cfg->chunk_frames != 0) return VDN_ERR_INVALID_ARG;
+  if (cfg->head_dim != 32 && cfg->head_dim != 64 && cfg->head_dim != 128) return VDN_ERR_UNSUPPORTED;
+  if (cfg->dtype != VDN_BF16 && cfg->dtype != VDN_FP32) return VDN_ERR_UNSUPPORTED;
+  if (cfg->debug_flags & ~(VDN_OUT_SOFTMAX_ONLY | VDN_OUT_LINEAR_ONLY | VDN_OUT_LINEAR_RAW | VDN_EXPORT_STATES))
+    return VDN_ERR_INVALID_ARG;
+  const int Nc = cfg->frames / cfg->chunk_frames;
+  if (Nc > kMaxScanChunks) return VDN_ERR_UNSUPPORTED;
+  const long long N = (long long)cfg->frames * cfg->tokens_per_frame;
+  // TMA row coordinates and tile arithmetic are 32-bit
+  if ((long long)cfg->batch * N >= (1ll << 30) || (long long)cfg->batch * cfg->text_tokens >= (1ll << 30) ||
+      (long long)cfg->chunk_frames * cfg->tokens_per_frame >= (1ll << 28) || cfg->heads > 4096)
+    return VDN_ERR_UNSUPPORTED;
+
+  std::memset(&g, 0, sizeof(g));
+  g.B = cfg->batch;
+  g.F = cfg->frames;
+  g.P = cfg->tokens_per_frame;
+  g.H = cfg->heads;
+  g.d = cfg->head_dim;
+  g.T = cfg->text_tokens;
+  g.C = cfg->chunk_frames;
+  g.Dp = g.d == 128 ? 128 : 64;
+  g.Nc = Nc;
+  g.N = N;
+  g.fp32_io = cfg->dtype == VDN_FP32;
+  g.staged = g.fp32_io || g.d != g.Dp;
+  g.n_slices = (g.P + kSliceTokens - 1) / kSliceTokens;
+  g.n_video_parts = (g.F - n_anchor(g.F)) * g.n_slices;
+  g.n_text_parts = (g.T + kSliceTokens - 1) / kSliceTokens;
+  g.n_parts = g.n_video_parts + g.n_text_parts;
+  g.rows_per_chunk = g.C * g.P;
+  g.n_pairs = (g.rows_per_chunk + 2 * kBlockM - 1) / (2 * kBlockM);
+  g.mt_rows = g.Dp + 16;
+  g.scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.0f / std::sqrt((float)g.d);
+  g.eps = cfg->rms_eps < 0.f ? 1e-6f : cfg->rms_eps;
+
+  const size_t vid = (size_t)g.B * g.N * g.H * g.Dp * 2;
+  const size_t txt = (size_t)g.B * g.T * g.H * g.Dp * 2;
+  size_t off = 0;
+  g.off_status = off; off = align_up(off + 256, 1024);
+  g.off_os = off; off = align_up(off + vid, 1024);
+  if (g.staged) {
+    g.off_q = off; off = align_up(off + vid, 1024);
+    g.off_k = off; off = align_up(off + vid, 1024);
+    g.off_v = off; off = align_up(off + vid, 1024);
+    g.off_tk = off; off = align_up(off + txt, 1024);
+    g.off_tv = off; off = align_up(off + txt, 1024);
+  }
+  g.off_parts = off; off = align_up(off + (size_t)g.n_parts * g.B * g.H * (g.Dp + 1) * g.Dp * 4, 1024);
+  g.off_mt = off; off = align_up(off + (size_t)g.B * g.Nc * g.H * 2 * g.mt_rows * g.Dp * 2, 1024);
+  g.total = off;
+  return VDN_OK;
+}
+
+vdn_status check_ws(const vdn_cfg* cfg, const Geom& g) {
+  if (!cfg->workspace || cfg->workspace_bytes < g.total) return VDN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(cfg->workspace) & 255u) != 0) return VDN_ERR_ALIGNMENT;
+  if (cfg->status_word && (reinterpret_cast<uintptr_t>(cfg->status_word) & 3u) != 0) return VDN_ERR_ALIGNMENT;
+  if (cfg->rms_weight && (reinterpret_cast<uintptr_t>(cfg->rms_weight) & 3u) != 0) return VDN_ERR_ALIGNMENT;
+  return VDN_OK;
+}
+
+vdn_status check_ptrs(std::initializer_list<const void*> required) {
+  for (const void* p : required) {
+    if (!p) return VDN_ERR_INVALID_ARG;
+    if (!aligned16(p)) return VDN_ERR_ALIGNMENT;
+  }
+  return VDN_OK;
+}
+
+uint8_t* ws(const vdn_cfg* cfg, size_t off) { return static_cast<uint8_t*>(cfg->workspace) + off; }
+
+int* status_ptr(const vdn_cfg* cfg, const Geom& g) {
+  return cfg->status_word ? cfg->status_word : reinterpret_cast<int*>(ws(cfg, g.off_status));
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 view [rows, H*Dp] (row pitch H*Dp*2 bytes), box 128 rows x 64
+// columns, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, long long rows, int H, int Dp) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  if (rows < 1) rows = 1;
+  const cuuint64_t dims[2] = {(cuuint64_t)H * Dp, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)H * Dp * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Srcs {
+  const void *q, *k, *v, *tk, *tv;
+};
+
+// Tensors the kernels read: the caller's (bf16, head_dim 64/128) or the staged copies.
+Srcs kernel_srcs(const vdn_cfg* cfg, const Geom& g, const void* q, const void* k, const void* v, const void* tk,
+                 const void* tv) {
+  if (!g.staged) return Srcs{q, k, v, tk, tv};
+  return Srcs{ws(cfg, g.off_q), ws(cfg, g.off_k), ws(cfg, g.off_v), ws(cfg, g.off_tk), ws(cfg, g.off_tv)};
+}
+
+bool make_maps(Maps& m, const Geom& g, const Srcs& s) {
+  const long long vrows = (long long)g.B * g.N;
+  const long long trows = (long long)g.B * g.T;
+  bool ok = make_map(&m.q, s.q, vrows, g.H, g.Dp) && make_map(&m.k, s.k, vrows, g.H, g.Dp) &&
+            make_map(&m.v, s.v, vrows, g.H, g.Dp);
+  if (g.T > 0) {
+    ok = ok && make_map(&m.tk, s.tk, trows, g.H, g.Dp) && make_map(&m.tv, s.tv, trows, g.H, g.Dp);
+  } else {  // never read; any valid descriptor
+    m.tk = m.q;
+    m.tv = m.q;
+  }
+  return ok;
+}
+
+vdn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? VDN_OK : VDN_ERR_CUDA; }
+
+// ---------------------------------------------------------------- steps
+
+vdn_status step_stage(const vdn_cfg* cfg, const Geom& g, const void* q, const void* k, const void* v, const void* tk,
+                      const void* tv, cudaStream_t st) {
+  if (!g.staged) return VDN_OK;
+  const long long vrows = (long long)g.B * g.N, trows = (long long)g.B * g.T;
+  cudaError_t e = launch_stage(q, g.fp32_io, reinterpret_cast<__nv_bfloat16*>(ws(cfg, g.off_q)), vrows, g.H, g.d, g.Dp, st);
+  if (e == cudaSuccess) e = launch_stage(k, g.fp32_io, reinterpret_cast<__nv_bfloat16*>(ws(cfg, g.off_k)), vrows, g.H, g.d, g.Dp, st);
+  if (e == cudaSuccess) e = launch_stage(v, g.fp32_io, reinterpret_cast<__nv_bfloat16*>(ws(cfg, g.off_v)), vrows, g.H, g.d, g.Dp, st);
+  if (e == cudaSuccess && g.T > 0)
+    e = launch_stage(tk, g.fp32_io, reinterpret_cast<__nv_bfloat16*>(ws(cfg, g.off_tk)), trows, g.H, g.d, g.Dp, st);
+  if (e == cudaSuccess && g.T > 0)
+    e = launch_stage(tv, g.fp32_io, reinterpret_cast<__nv_bfloat16*>(ws(cfg, g.off_tv)), trows, g.H, g.d, g.Dp, st);
+  return cuda_status(e);
+}
+
+vdn_status step_state_build(const vdn_cfg* cfg, const Geom& g, const Srcs& s, cudaStream_t st) {
+  if (g.n_parts == 0) return VDN_OK;
+  Maps m;
+  if (!make_maps(m, g, s)) return VDN_ERR_CUDA;
+  K1Params p;
+  p.g = g;
+  p.parts = reinterpret_cast<float*>(ws(cfg, g.off_parts));
+  p.status = status_ptr(cfg, g);
+  return cuda_status(launch_state_build(m, p, st));
+}
+
+vdn_status step_state_scan(const vdn_cfg* cfg, const Geom& g, cudaStream_t st) {
+  K2Params p;
+  p.g = g;
+  p.parts = reinterpret_cast<const float*>(ws(cfg, g.off_parts));
+  p.mt = ws(cfg, g.off_mt);
+  const bool exp = (cfg->debug_flags & VDN_EXPORT_STATES) != 0;
+  p.export_fwd = exp ? cfg->export_fwd : nullptr;
+  p.export_bwd = exp ? cfg->export_bwd : nullptr;
+  return cuda_status(launch_state_scan(p, st));
+}
+
+vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s, cudaStream_t st) {
+  Maps m;
+  if (!make_maps(m, g, s)) return VDN_ERR_CUDA;
+  K3Params p;
+  std::memset(&p, 0, sizeof(p));
+  p.g = g;
+  p.scale_log2 = g.scale * 1.4426950408889634f;
+  p.o_s = reinterpret_cast<__nv_bfloat16*>(ws(cfg, g.off_os));
+  p.status = status_ptr(cfg, g);
+  p.items_per_chunk = g.B * g.H * g.n_pairs;
+  p.n_items = g.Nc * p.items_per_chunk;
+  // longest chunks first (static longest-processing-time order)
+  std::vector<int> order(g.Nc);
+  std::iota(order.begin(), order.end(), 0);
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return kv_tiles(a, g) > kv_tiles(b, g); });
+  for (int i = 0; i < g.Nc; ++i) p.chunk_order[i] = order[i];
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = std::min(p.n_items, sms);
+  return cuda_status(launch_sparse_softmax(m, p, grid, st));
+}
+
+vdn_status step_readout_merge(const vdn_cfg* cfg, const Geom& g, const Srcs& s, const void* gs, const void* gl,
+                              void* out, cudaStream_t st) {
+  Maps m;
+  if (!make_maps(m, g, s)) return VDN_ERR_CUDA;
+  K4Params p;
+  p.g = g;
+  p.o_s = reinterpret_cast<const __nv_bfloat16*>(ws(cfg, g.off_os));
+  p.mt = ws(cfg, g.off_mt);
+  p.gamma = cfg->rms_weight;
+  p.gate_s = gs;
+  p.gate_l = gl;
+  p.out = out;
+  p.flags = cfg->debug_flags & (VDN_OUT_SOFTMAX_ONLY | VDN_OUT_LINEAR_ONLY | VDN_OUT_LINEAR_RAW);
+  p.status = status_ptr(cfg, g);
+  return cuda_status(launch_readout_merge(m, p, st));
+}
+
+vdn_status check_inputs(const vdn_cfg* cfg, const Geom& g, std::initializer_list<const void*> video,
+                        std::initializer_list<const void*> text) {
+  vdn_status s = check_ws(cfg, g);
+  if (s != VDN_OK) return s;
+  s = check_ptrs(video);
+  if (s != VDN_OK) return s;
+  if (g.T > 0) s = check_ptrs(text);
+  return s;
+}
+
+}  // namespace
+}  // namespace vdn
+
+using namespace vdn;
+
+extern "C" {
+
+int32_t vdn_version(void) { return (1 << 16) | 0; }
+
+const char* vdn_status_string(vdn_status s) {
+  switch (s) {
+    case VDN_OK: return "ok";
+    case VDN_ERR_INVALID_ARG: return "invalid argument";
+    case VDN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case VDN_ERR_ALIGNMENT: return "pointer not aligned";
+    case VDN_ERR_WORKSPACE: return "workspace missing or too small";
+    case VDN_ERR_CUDA: return "CUDA error";
+    case VDN_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+vdn_status vdn_validate(const vdn_cfg* cfg) {
+  Geom g;
+  return make_geom(cfg, g);
+}
+
+size_t vdn_workspace_bytes(const vdn_cfg* cfg) {
+  Geom g;
+  return make_geom(cfg, g) == VDN_OK ? g.total : 0;
+}
+
+vdn_status vdn_plan_membership(const vdn_cfg* cfg, uint8_t* table) {
+  Geom g;
+  vdn_status s = make_geom(cfg, g);
+  if (s != VDN_OK) return s;
+  if (!table) return VDN_ERR_INVALID_ARG;
+  for (int f = 0; f < g.F; ++f) {
+    const int c = f / g.C;
+    const int wlo = std::max(0, c - 1), whi = std::min(g.Nc - 1, c + 1);
+    for (int x = 0; x < g.F; ++x) {
+      const int cx = x / g.C;
+      uint8_t code;
+      if ((cx >= wlo && cx <= whi) || is_anchor(x, g.F)) code = 1;
+      else if (cx <= fwd_last_chunk(c)) code = 2;
+      else code = 3;
+      table[f * g.F + x] = code;
+    }
+  }
+  return VDN_OK;
+}
+
+vdn_status vdn_membership_device(const vdn_cfg* cfg, uint8_t* table_dev, void* stream) {
+  Geom g;
+  vdn_status s = make_geom(cfg, g);
+  if (s != VDN_OK) return s;
+  if (!table_dev) return VDN_ERR_INVALID_ARG;
+  return cuda_status(launch_membership(g, table_dev, static_cast<cudaStream_t>(stream)));
+}
+
+vdn_status vdn_stage_inputs(const void* q, const void* k, const void* v, const void* text_k, const void* text_v,
+                            const vdn_cfg* cfg, void* stream) {
+  Geom g;
+  vdn_status s = make_geom(cfg, g);
+  if (s != VDN_OK) return s;
+  s = check_inputs(cfg, g, {q, k, v}, {text_k, text_v});
+  if (s != VDN_OK) return s;
+  return step_stage(cfg, g, q, k, v, text_k, text_v, static_cast<cudaStream_t>(stream));
+}
+
+vdn_status vdn_state_build(const void* k, const void* v, const void* text_k, const void* text_v, const vdn_cfg* cfg,
+                           void* stream) {
+  Geom g;
+  vdn_status s = make_geom(cfg, g);
+  if (s != VDN_OK) return s;
+  s = check_inputs(cfg, g, {k, v}, {text_k, text_v});
+  if (s != VDN_OK) return s;
+  return step_state_build(cfg, g, kernel_srcs(cfg, g, k, k, v, text_k, text_v), static_cast<cudaStream_t>(stream));
+}
+
+vdn_status vdn_state_scan(const vdn_cfg* cfg, void* stream) {
+  Geom g;
+  vdn_status s = make_geom(cfg, g);
+  if (s != VDN_OK) return s;
+  s = check_ws(cfg, g);
+  if (s != VDN_OK) return s;
+  if ((cfg->debug_flags & VDN_EXPORT_STATES) && (!cfg->export_fwd || !cfg->export_bwd)) return VDN_ERR_INVALID_ARG;
+  return step_state_scan(cfg, g, static_cast<cudaStream_t>(stream));
+}
+
+vdn_status vdn_sparse_softmax(const void* q, const void* k, const void* v, const void* text_k, const void* text_v,
+                              const vdn_cfg* cfg, void* stream) {
+  Geom g;
+  vdn_status s = make_geom(cfg, g);
+  if (s != VDN_OK) return s;
+  s = check_inputs(cfg, g, {q, k, v}, {text_k, text_v});
+  if (s != VDN_OK) return s;
+  return step_sparse_softmax(cfg, g, kernel_srcs(cfg, g, q, k, v, text_k, text_v), static_cast<cudaStream_t>(stream));
+}
+
+vdn_status vdn_readout_merge(const void* q, const void* gate_s, const void* gate_l, void* out, const vdn_cfg* cfg,
+                             void* stream) {
+  Geom g;
+  vdn_status s = make_geom(cfg, g);
+  if (s != VDN_OK) return s;
+  s = check_inputs(cfg, g, {q, gate_s, gate_l, out}, {});
+  if (s != VDN_OK) return s;
+  return step_readout_merge(cfg, g, kernel_srcs(cfg, g, q, q, q, q, q), gate_s, gate_l, out,
+                            static_cast<cudaStream_t>(stream));
+}
+
+vdn_status vdn_hybrid_attn_fwd(const void* q, const void* k, const void* v, const void* text_k, const void* text_v,
+                               const void* gate_s, const void* gate_l, void* out, const vdn_cfg* cfg, void* stream) {
+  Geom g;
+  vdn_status s = make_geom(cfg, g);
+  if (s != VDN_OK) return s;
+  s = check_inputs(cfg, g, {q, k, v, gate_s, gate_l, out}, {text_k, text_v});
+  if (s != VDN_OK) return s;
+  if ((cfg->debug_flags & VDN_EXPORT_STATES) && (!cfg->export_fwd || !cfg->export_bwd)) return VDN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Srcs src = kernel_srcs(cfg, g, q, k, v, text_k, text_v);
+  if ((s = step_stage(cfg, g, q, k, v, text_k, text_v, st)) != VDN_OK) return s;
+  if ((s = step_state_build(cfg, g, src, st)) != VDN_OK) return s;
+  if ((s = step_state_scan(cfg, g, st)) != VDN_OK) return s;
+  if ((s = step_sparse_softmax(cfg, g, src, st)) != VDN_OK) return s;
+  return step_readout_merge(cfg, g, src, gate_s, gate_l, out, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,383 @@
+// k3_sparse_softmax.cu - softmax branch of the VDN-H3 hybrid attention
+// (article section 双分支混合注意力机制): exact attention of every video query
+// over the keys of its chunk window (chunk c-1..c+1, clipped), the two anchor
+// frames and all text tokens.
+//
+// Design (sm_100a):
+//  * persistent CTAs, one per SM; a work item is two 128-row query tiles of
+//    one (batch, head, chunk); items are handed out statically in an order
+//    sorted by KV tile count (longest first);
+//  * only the KV tiles of the item's chunk are enumerated: at most three
+//    merged video token ranges plus the text range, 128 keys per tile; the
+//    last tile of a range is masked past the range end;
+//  * warp 0 issues TMA loads (Q once per item, K and V per tile, two stages);
+//    warp 1 issues tcgen05 MMAs from one thread: S_t = Q_t K^T (both operands
+//    K-major in shared memory, fp32 accumulator in TMEM) and O_t += P_t V
+//    (P_t read from TMEM, V MN-major in shared memory);
+//  * warps 4-7 and 8-11 are the softmax warpgroups of query tile 0 and 1;
+//    each thread owns one query row (TMEM lane), so row max and row sum are
+//    in-thread; P is written back as bf16 over the first half of S's columns;
+//  * online softmax with a lazy rescale: the running max only moves (and O is
+//    rescaled in TMEM) when a tile's max exceeds it by more than 8 in log2
+//    units; the final 1/l is applied in the epilogue;
+//  * TMEM: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
+//
+// The MMA issue order per KV tile j is PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), so
+// the tensor core works on one tile while the other tile's softmax runs.  A
+// commit after S_t(j+1) also covers PV_t(j), so when the softmax of tile t sees
+// S_t(j+1) its O_t is quiescent and may be rescaled.
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace vdn {
+
+namespace {
+
+template <int D>
+struct K3Layout {
+  static constexpr int kTile = kBlockM * D * 2;  // bytes of one 128-row bf16 tile
+  static constexpr int kStages = 2;
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + 2 * kTile;
+  static constexpr int kV = kK + kStages * kTile;
+  static constexpr int kBar = kV + kStages * kTile;
+  static constexpr int kBytes = kBar + 256 + 1024;  // + barriers + alignment slack
+};
+
+struct Item {
+  int b, h, c, pair, ntiles, row0;  // row0: first query row of the item within the batch
+};
+
+__device__ __forceinline__ Item decode_item(int item, const K3Params& p) {
+  const Geom& g = p.g;
+  Item it;
+  const int pos = item / p.items_per_chunk;
+  int rem = item - pos * p.items_per_chunk;
+  it.c = p.chunk_order[pos];
+  const int per_b = g.H * g.n_pairs;
+  it.b = rem / per_b;
+  rem -= it.b * per_b;
+  it.h = rem / g.n_pairs;
+  it.pair = rem - it.h * g.n_pairs;
+  it.row0 = it.c * g.rows_per_chunk + it.pair * 2 * kBlockM;
+  it.ntiles = (it.pair * 2 * kBlockM + kBlockM < g.rows_per_chunk) ? 2 : 1;
+  return it;
+}
+
+// Barrier slots.
+enum {
+  kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = 4, kVFull = 6, kVEmpty = 8,
+  kSFull = 10, kPFull = 12, kOFull = 14, kDone = 16, kNumBars = 17
+};
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+    k3_sparse_softmax(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_tk,
+                      const __grid_constant__ CUtensorMap tm_tv, const __grid_constant__ K3Params p) {
+  using L = K3Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + kNumBars * 8);
+  int* abort_flag = reinterpret_cast<int*>(smem + L::kBar + kNumBars * 8 + 4);
+
+  const Geom& g = p.g;
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[kQFull], 1);
+    mbar_init(&bars[kQEmpty], 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(&bars[kKFull + s], 1);
+      mbar_init(&bars[kKEmpty + s], 1);
+      mbar_init(&bars[kVFull + s], 1);
+      mbar_init(&bars[kVEmpty + s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars[kSFull + t], 1);
+      mbar_init(&bars[kPFull + t], kBlockM);
+      mbar_init(&bars[kOFull + t], 1);
+    }
+    mbar_init(&bars[kDone], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const CtaAbort ab{abort_flag, p.status};
+
+  uint8_t* sQ = smem + L::kQ;
+  uint8_t* sK = smem + L::kK;
+  uint8_t* sV = smem + L::kV;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t kv_cnt = 0, item_cnt = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++item_cnt) {
+        const Item it = decode_item(item, p);
+        if (item_cnt > 0 && !mbar_wait(&bars[kQEmpty], (item_cnt - 1) & 1, ab)) { ok = false; break; }
+        mbar_expect_tx(&bars[kQFull], it.ntiles * L::kTile);
+        for (int t = 0; t < it.ntiles; ++t)
+          for (int bx = 0; bx < D / 64; ++bx)
+            tma_load_2d(sQ + t * L::kTile + bx * 16384, &tm_q, &bars[kQFull], it.h * D + bx * 64,
+                        it.b * (int)g.N + it.row0 + t * kBlockM);
+        KvRanges kr;
+        kv_ranges(it.c, g, kr);
+        for (int ri = 0; ri <= kr.n && ok; ++ri) {
+          const bool text = (ri == kr.n);
+          const int len = text ? g.T : (int)kr.len[ri];
+          const int base = text ? it.b * g.T : it.b * (int)g.N + (int)kr.start[ri];
+          const CUtensorMap* mk = text ? &tm_tk : &tm_k;
+          const CUtensorMap* mv = text ? &tm_tv : &tm_v;
+          for (int off = 0; off < len; off += kBlockN, ++kv_cnt) {
+            const int st = kv_cnt % L::kStages;
+            const uint32_t ph = (kv_cnt / L::kStages) & 1;
+            if (!mbar_wait(&bars[kKEmpty + st], ph ^ 1, ab)) { ok = false; break; }
+            mbar_expect_tx(&bars[kKFull + st], L::kTile);
+            for (int bx = 0; bx < D / 64; ++bx)
+              tma_load_2d(sK + st * L::kTile + bx * 16384, mk, &bars[kKFull + st], it.h * D + bx * 64, base + off);
+            if (!mbar_wait(&bars[kVEmpty + st], ph ^ 1, ab)) { ok = false; ++kv_cnt; break; }
+            mbar_expect_tx(&bars[kVFull + st], L::kTile);
+            for (int bx = 0; bx < D / 64; ++bx)
+              tma_load_2d(sV + st * L::kTile + bx * 16384, mv, &bars[kVFull + st], it.h * D + bx * 64, base + off);
+          }
+        }
+      }
+      if (!ok) {
+        // Let loads already in flight land before the CTA's shared memory goes away.
+        for (uint32_t i = (kv_cnt > (uint32_t)L::kStages ? kv_cnt - L::kStages : 0); i < kv_cnt; ++i) {
+          mbar_drain(&bars[kKFull + i % L::kStages], (i / L::kStages) & 1);
+          mbar_drain(&bars[kVFull + i % L::kStages], (i / L::kStages) & 1);
+        }
+        if (item_cnt > 0) mbar_drain(&bars[kQFull], (item_cnt - 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kBlockN, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      uint32_t kv_cnt = 0, item_cnt = 0, p_cnt[2] = {0, 0};
+      bool ok = true;
+
+      auto issue_qk = [&](int t, int st) {
+        const uint32_t d_tmem = tmem + t * 128;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint64_t a = smem_desc(q_addr + t * L::kTile + off, 16, 1024, kLayoutSw128);
+          const uint64_t b = smem_desc(k_addr + st * L::kTile + off, 16, 1024, kLayoutSw128);
+          mma_ss(d_tmem, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int st, bool acc) {
+        const uint32_t d_tmem = tmem + 256 + t * D;
+#pragma unroll
+        for (int kk = 0; kk < kBlockN / 16; ++kk) {
+          const uint64_t b = smem_desc(v_addr + st * L::kTile + kk * 2048, 16384, 1024, kLayoutSw128);
+          mma_ts(d_tmem, tmem + t * 128 + kk * 8, b, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++item_cnt) {
+        const Item it = decode_item(item, p);
+        const int nkv = kv_tiles(it.c, g);
+        if (!mbar_wait(&bars[kQFull], item_cnt & 1, ab)) { ok = false; break; }
+        {
+          const int st = kv_cnt % L::kStages;
+          if (!mbar_wait(&bars[kKFull + st], (kv_cnt / L::kStages) & 1, ab)) { ok = false; break; }
+          tc_fence_after();
+          for (int t = 0; t < it.ntiles; ++t) {
+            issue_qk(t, st);
+            mma_commit(&bars[kSFull + t]);
+          }
+          mma_commit(&bars[kKEmpty + st]);
+        }
+        for (int j = 0; j < nkv; ++j, ++kv_cnt) {
+          const int st = kv_cnt % L::kStages;
+          const int nst = (kv_cnt + 1) % L::kStages;
+          const bool has_next = j + 1 < nkv;
+          if (!mbar_wait(&bars[kVFull + st], (kv_cnt / L::kStages) & 1, ab)) { ok = false; break; }
+          for (int t = 0; t < it.ntiles; ++t) {
+            if (!mbar_wait(&bars[kPFull + t], p_cnt[t] & 1, ab)) { ok = false; break; }
+            ++p_cnt[t];
+            tc_fence_after();
+            issue_pv(t, st, j > 0);
+            if (!has_next) mma_commit(&bars[kOFull + t]);
+            if (has_next) {
+              if (t == 0 && !mbar_wait(&bars[kKFull + nst], ((kv_cnt + 1) / L::kStages) & 1, ab)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              issue_qk(t, nst);
+              mma_commit(&bars[kSFull + t]);
+            }
+          }
+          if (!ok) break;
+          mma_commit(&bars[kVEmpty + st]);
+          if (has_next) mma_commit(&bars[kKEmpty + nst]);
+        }
+        if (!ok) break;
+        mma_commit(&bars[kQEmpty]);
+      }
+      // All MMAs issued by this thread complete before TMEM is released.
+      mma_commit(&bars[kDone]);
+      mbar_drain(&bars[kDone], 0);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int t = (warp - 4) >> 2;
+    const uint32_t quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // query row of the tile == TMEM lane
+    const uint32_t lane_base = quarter * 32;
+    const float sl2 = p.scale_log2;
+    uint32_t s_cnt = 0, o_cnt = 0;
+
+    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+      const Item it = decode_item(item, p);
+      if (t >= it.ntiles) continue;
+      const int tile_row0 = it.pair * 2 * kBlockM + t * kBlockM;  // within the chunk
+      const int nrows = min(kBlockM, g.rows_per_chunk - tile_row0);
+      float m_run = 0.f, l_run = 0.f;
+      KvRanges kr;
+      kv_ranges(it.c, g, kr);
+      bool ok = true;
+      int j = 0;
+      for (int ri = 0; ri <= kr.n && ok; ++ri) {
+        const int len = (ri == kr.n) ? g.T : (int)kr.len[ri];
+        for (int off = 0; off < len; off += kBlockN, ++j) {
+          const int n_valid = min(kBlockN, len - off);
+          const bool got = mbar_wait(&bars[kSFull + t], s_cnt & 1, ab);
+          if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
+          ++s_cnt;
+          tc_fence_after();
+          uint32_t s[128];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t (&chunk)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32 * i]);
+            tmem_ld32(tmem_addr(tmem, lane_base, t * 128 + 32 * i), chunk);
+          }
+          tmem_wait_ld();
+          if (n_valid < kBlockN) {
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+              if (i >= n_valid) s[i] = __float_as_uint(-INFINITY);
+          }
+          float mx = __uint_as_float(s[0]);
+#pragma unroll
+          for (int i = 1; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(s[i]));
+          const float mxs = mx * sl2;
+          // lazy rescale: move the running max only when this tile's max is
+          // more than 2^8 above it (O is rescaled below, once P is stored)
+          float alpha = 1.0f;
+          bool rescale = false;
+          if (j == 0) {
+            m_run = mxs;
+          } else {
+            const bool need = mxs > m_run + 8.0f;
+            rescale = __any_sync(0xffffffffu, need);
+            if (need) {
+              alpha = ex2_approx(m_run - mxs);
+              m_run = mxs;
+            }
+          }
+          l_run *= alpha;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float p0 = ex2_approx(fmaf(__uint_as_float(s[32 * i + 2 * e]), sl2, -m_run));
+              const float p1 = ex2_approx(fmaf(__uint_as_float(s[32 * i + 2 * e + 1]), sl2, -m_run));
+              l_run += p0 + p1;
+              pk[e] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(tmem_addr(tmem, lane_base, t * 128 + 16 * i), pk);
+          }
+          if (rescale) {
+            // O_t is quiescent here: S_t(j) completing implies PV_t(j-1) completed
+#pragma unroll 1
+            for (int i = 0; i < D / 32; ++i) {
+              uint32_t o[32];
+              const uint32_t ta = tmem_addr(tmem, lane_base, 256 + t * D + 32 * i);
+              tmem_ld32(ta, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(ta, o);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&bars[kPFull + t]);
+        }
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue: o_s = O / l
+      const bool got = mbar_wait(&bars[kOFull + t], o_cnt & 1, ab);
+      if (__any_sync(0xffffffffu, !got)) break;
+      ++o_cnt;
+      tc_fence_after();
+      const float inv_l = 1.0f / l_run;
+      __nv_bfloat16* dst = p.o_s + (((size_t)it.b * g.N + (size_t)(it.c * g.rows_per_chunk + tile_row0 + row)) * g.H + it.h) * D;
+#pragma unroll
+      for (int i = 0; i < D / 32; ++i) {
+        uint32_t o[32];
+        tmem_ld32(tmem_addr(tmem, lane_base, 256 + t * D + 32 * i), o);
+        tmem_wait_ld();
+        if (row < nrows) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * i);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(o[8 * v4 + 0]) * inv_l, __uint_as_float(o[8 * v4 + 1]) * inv_l);
+            w.y = pack_bf16x2(__uint_as_float(o[8 * v4 + 2]) * inv_l, __uint_as_float(o[8 * v4 + 3]) * inv_l);
+            w.z = pack_bf16x2(__uint_as_float(o[8 * v4 + 4]) * inv_l, __uint_as_float(o[8 * v4 + 5]) * inv_l);
+            w.w = pack_bf16x2(__uint_as_float(o[8 * v4 + 6]) * inv_l, __uint_as_float(o[8 * v4 + 7]) * inv_l);
+            d4[v4] = w;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem, 512);
+}
+
+size_t k3_smem_bytes(int Dp) {
+  // At least ~116 KB so that a second CTA never shares the SM (each claims all 512 TMEM columns).
+  const size_t need = Dp == 128 ? (size_t)K3Layout<128>::kBytes : (size_t)K3Layout<64>::kBytes;
+  return need < 118 * 1024 ? 118 * 1024 : need;
+}
+
+template <int D>
+static cudaError_t launch_k3(const Maps& m, const K3Params& p, int grid, cudaStream_t st) {
+  const size_t smem = k3_smem_bytes(D);
+  cudaError_t e = cudaFuncSetAttribute(k3_sparse_softmax<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k3_sparse_softmax<D><<<grid, 384, smem, st>>>(m.q, m.k, m.v, m.tk, m.tv, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sparse_softmax(const Maps& m, const K3Params& p, int grid, cudaStream_t st) {
+  return p.g.Dp == 128 ? launch_k3<128>(m, p, grid, st) : launch_k3<64>(m, p, grid, st);
+}
+
+}  // namespace vdn

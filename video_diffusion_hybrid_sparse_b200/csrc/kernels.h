@@ -1,0 +1,64 @@
+// kernels.h - parameter blocks and host launchers of the CUDA kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "plan.h"
+
+namespace vdn {
+
+struct K3Params {
+  Geom g;
+  float scale_log2;        // softmax scale * log2(e)
+  __nv_bfloat16* o_s;      // [B, N, H, Dp] bf16
+  int* status;
+  int n_items;             // Nc * B * H * n_pairs
+  int items_per_chunk;     // B * H * n_pairs
+  int chunk_order[kMaxChunks];  // chunks by decreasing KV tile count
+};
+
+struct K1Params {
+  Geom g;
+  float* parts;            // [n_parts, B, H, Dp+1, Dp] fp32; row Dp holds z
+  int* status;
+};
+
+struct K2Params {
+  Geom g;
+  const float* parts;
+  uint8_t* mt;             // readout B-tiles (hi, lo) per (b, chunk, head)
+  float* export_fwd;       // optional [B, Nc, H, d+1, d]
+  float* export_bwd;
+};
+
+struct K4Params {
+  Geom g;
+  const __nv_bfloat16* o_s;
+  const uint8_t* mt;
+  const float* gamma;      // [H, d] or null
+  const void* gate_s;
+  const void* gate_l;
+  void* out;
+  int flags;
+  int* status;
+};
+
+// Tensor maps: 2-D bf16 views [rows, H*Dp] with a 128-row x 64-column box and
+// 128-byte swizzle.
+struct Maps {
+  CUtensorMap q, k, v, tk, tv;
+};
+
+cudaError_t launch_stage(const void* src, int fp32_in, __nv_bfloat16* dst, long long rows, int H, int d, int Dp,
+                         cudaStream_t st);
+cudaError_t launch_state_build(const Maps& m, const K1Params& p, cudaStream_t st);
+cudaError_t launch_state_scan(const K2Params& p, cudaStream_t st);
+cudaError_t launch_sparse_softmax(const Maps& m, const K3Params& p, int grid, cudaStream_t st);
+cudaError_t launch_readout_merge(const Maps& m, const K4Params& p, cudaStream_t st);
+cudaError_t launch_membership(const Geom& g, uint8_t* table, cudaStream_t st);
+
+size_t k3_smem_bytes(int Dp);
+
+}  // namespace vdn

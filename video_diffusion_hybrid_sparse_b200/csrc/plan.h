@@ -1,0 +1,118 @@
+// plan.h - problem geometry, workspace layout and the index rules of the
+// hybrid attention, shared by the host (validation, membership table, launch
+// set-up) and the kernels (KV tile enumeration, state membership).
+//
+// Index rules (VDN-H3 article, section 双分支混合注意力机制):
+//   * latent frames are grouped into chunks of C consecutive frames;
+//   * the softmax branch of chunk c reads the window chunks
+//     max(0, c-1) .. min(Nc-1, c+1) plus the anchor frames 0 and F-1 plus the
+//     text; an anchor already inside the window is read once;
+//   * the forward state of chunk c holds chunks 0 .. c-2, the backward state
+//     chunks c+2 .. Nc-1, both without the anchor frames;
+//   * each state also holds half of the text state.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#ifdef __CUDACC__
+#define VDN_HD __host__ __device__ __forceinline__
+#else
+#define VDN_HD inline
+#endif
+
+namespace vdn {
+
+constexpr int kMaxChunks = 256;     // chunk-order table carried in kernel parameters
+constexpr int kSliceTokens = 1024;  // tokens per state-build work item
+constexpr int kBlockM = 128;        // query rows per tile
+constexpr int kBlockN = 128;        // keys per tile
+
+struct Geom {
+  int B, F, P, H, d, T, C;  // batch, frames, tokens/frame, heads, head_dim, text tokens, chunk frames
+  int Dp;                   // head_dim as stored for the tensor cores (64 or 128)
+  int Nc;                   // chunks
+  long long N;              // F * P video tokens per batch
+  int staged;               // inputs are converted/padded into the workspace first
+  int fp32_io;              // q/k/v/text/gates/out are fp32
+  int n_slices;             // state-build slices per non-anchor frame
+  int n_video_parts;        // (F - |anchors|) * n_slices
+  int n_text_parts;         // ceil(T / kSliceTokens)
+  int n_parts;
+  int rows_per_chunk;       // C * P query rows
+  int n_pairs;              // work items of two 128-row query tiles per chunk
+  int mt_rows;              // rows of one readout B-tile: Dp + 16 (values, z, zero padding)
+  float scale;              // softmax scale
+  float eps;                // RMSNorm epsilon
+  // workspace layout (byte offsets; each 1024-aligned)
+  size_t off_status, off_os, off_q, off_k, off_v, off_tk, off_tv, off_parts, off_mt, total;
+};
+
+VDN_HD int is_anchor(int f, int F) { return f == 0 || f == F - 1; }
+VDN_HD int n_anchor(int F) { return F == 1 ? 1 : 2; }
+
+// Number of non-anchor frames in chunks [c0, c1] (empty if c1 < c0).
+VDN_HD int nonanchor_frames_in_chunks(int c0, int c1, int C, int F) {
+  if (c1 < c0) return 0;
+  int f0 = c0 * C, f1 = (c1 + 1) * C - 1;  // inclusive frame range
+  int n = f1 - f0 + 1;
+  if (f0 <= 0 && 0 <= f1) n--;
+  if (F - 1 != 0 && f0 <= F - 1 && F - 1 <= f1) n--;
+  return n;
+}
+
+// Tokens held by the two states of chunk c (text counted once); 0 means an empty read.
+VDN_HD long long state_tokens(int c, const Geom& g) {
+  int nf = nonanchor_frames_in_chunks(0, c - 2, g.C, g.F) + nonanchor_frames_in_chunks(c + 2, g.Nc - 1, g.C, g.F);
+  return (long long)g.T + (long long)g.P * nf;
+}
+
+// Video key token ranges [start, start+len) read by the softmax branch of
+// chunk c: window plus anchors, adjacent ranges merged, at most three.
+struct KvRanges {
+  long long start[3];
+  long long len[3];
+  int n;
+};
+
+VDN_HD void kv_ranges(int c, const Geom& g, KvRanges& r) {
+  const int wlo = (c - 1 > 0 ? c - 1 : 0) * g.C;                        // first window frame
+  const int whi = ((c + 1 < g.Nc - 1 ? c + 1 : g.Nc - 1) + 1) * g.C;    // one past last window frame
+  long long s[3], e[3];
+  int n = 0;
+  if (wlo > 0) { s[n] = 0; e[n] = g.P; n++; }                            // anchor 0 before the window
+  s[n] = (long long)wlo * g.P; e[n] = (long long)whi * g.P; n++;          // window
+  if (whi < g.F) { s[n] = (long long)(g.F - 1) * g.P; e[n] = (long long)g.F * g.P; n++; }  // last anchor after it
+  // merge touching ranges
+  r.n = 0;
+  for (int i = 0; i < n; ++i) {
+    if (r.n > 0 && r.start[r.n - 1] + r.len[r.n - 1] == s[i]) {
+      r.len[r.n - 1] += e[i] - s[i];
+    } else {
+      r.start[r.n] = s[i];
+      r.len[r.n] = e[i] - s[i];
+      r.n++;
+    }
+  }
+}
+
+VDN_HD int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// KV tiles of 128 keys enumerated by the softmax kernel for chunk c.
+VDN_HD int kv_tiles(int c, const Geom& g) {
+  KvRanges r;
+  kv_ranges(c, g, r);
+  int n = 0;
+  for (int i = 0; i < r.n; ++i) n += ceil_div(r.len[i], kBlockN);
+  return n + ceil_div(g.T, kBlockN);
+}
+
+// Last chunk summed by the forward state of chunk c, first chunk summed by
+// its backward state (the window is c-1 .. c+1).
+VDN_HD int fwd_last_chunk(int c) { return c - 2; }
+VDN_HD int bwd_first_chunk(int c) { return c + 2; }
+
+// Frame of video state part p (parts ordered by non-anchor frame, then slice).
+VDN_HD int part_frame(int p, const Geom& g) { return 1 + p / g.n_slices; }
+
+}  // namespace vdn
