@@ -1,0 +1,414 @@
+"""Benchmark of the VDN-H3 hybrid attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 768p_bf16] [--impl ours|reference]
+
+A step is one whole hybrid-attention call (staging when needed, state build,
+state scan, sparse softmax, readout + merge) on one batch of seeded synthetic
+inputs already resident in HBM.  Each step's kernels are launched through the
+library's per-step C-ABI entry points with a CUDA event after each one, on the
+launching stream, so the dominant kernel's time is measured live.  The inputs
+of one call (1.9 GB at 768p) are larger than L2, so no flush is needed.
+
+Multi-GPU: the path runs on one GPU; under torchrun every rank runs an
+independent replica of the same workload (no data-path collective) and the
+timing is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle (the method's definition) on
+the host cores, on a bounded sample of the same workload, scaled to the
+metric's unit.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from video_diffusion_hybrid_sparse_b200.workloads import BY_NAME, make_inputs  # noqa: E402
+
+METRIC = "hybrid-attn ms/call & TFLOP/s at 768p-shaped latent, 1×B200, % of roofline"
+SPEC_TFLOPS, SPEC_GBS = 2250.0, 8000.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS = ["stage", "state_build", "state_scan", "sparse_softmax", "readout_merge"]
+
+
+# ---------------------------------------------------------------- algorithmic work
+
+
+def softmax_key_frames(c, F, C):
+    n_chunks = F // C
+    win = set(range(max(0, c - 1) * C, (min(n_chunks - 1, c + 1) + 1) * C))
+    return win | {0, F - 1}
+
+
+def work(w):
+    """Algorithmic FLOPs and bytes per call (counts only what the method must do)."""
+    e = 2 if w.dtype == "bf16" else 4
+    n_chunks, anchors = w.F // w.C, len({0, w.F - 1})
+    pairs = sum(w.C * w.P * (w.P * len(softmax_key_frames(c, w.F, w.C)) + w.T) for c in range(n_chunks))
+    softmax_flops = 4.0 * w.d * w.H * w.B * pairs
+    linear_flops = 2.0 * w.d * (w.d + 1) * w.H * w.B * (w.P * (w.F - anchors) + w.T + w.N)
+    state = w.B * w.H * w.d * (w.d + 1) * 4
+    k1 = 2 * (w.P * (w.F - anchors) + w.T) * w.B * w.H * w.d * e + (w.F - anchors + 1) * state
+    k2 = (w.F - anchors + 1) * state + n_chunks * state
+    k4 = 5 * w.B * w.N * w.H * w.d * e + n_chunks * state
+    k3_bytes = (3 * w.B * w.N + 2 * w.B * w.T) * w.H * w.d * e + w.B * w.N * w.H * w.d * 2
+    return dict(softmax_flops=softmax_flops, linear_flops=linear_flops, k1_bytes=k1, k2_bytes=k2, k4_bytes=k4,
+                k3_bytes=k3_bytes, linear_bytes=k1 + k2 + k4)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return p, "measured"
+    return FALLBACK, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sms, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sms.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+def gpu_id_for(local_rank: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ---------------------------------------------------------------- ncu traffic record
+
+
+def kernel_source_hash(name: str) -> str:
+    files = {"sparse_softmax": "k3_sparse_softmax.cu"}
+    path = os.path.join(ROOT, "video_diffusion_hybrid_sparse_b200", "csrc", files[name])
+    with open(path, "rb") as fh:
+        return hashlib.sha1(fh.read()).hexdigest()[:12]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel (lines: kernel workload bytes source_hash)."""
+    path = os.path.join(ROOT, "profiles", "ncu_dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    cur = kernel_source_hash(kernel)
+    with open(path) as fh:
+        for ln in fh:
+            f = ln.split()
+            if len(f) >= 4 and not ln.startswith("#") and f[0] == kernel and f[1] == workload and f[3] == cur:
+                return float(f[2])
+    return None
+
+
+# ---------------------------------------------------------------- CPU baseline (oracle)
+
+
+class CpuBaseline:
+    """The fp64 oracle timed on a bounded sample of the workload, scaled to one
+    whole call.  Per head the call costs the frame states plus, per query
+    frame, the softmax rows, readout, RMSNorm and merge; a query frame's cost
+    is taken proportional to the number of keys it scores (window + anchors +
+    text), from the frames actually timed.  The sample is head 0: its frame
+    states and the given query frames."""
+
+    def __init__(self, w, inputs):
+        from oracle import hybrid_attn as O  # only this leg imports the oracle
+
+        self.O, self.w = O, w
+        self.cores = len(os.sched_getaffinity(0))
+        self.x = {k: t[:, :, 0:1, :].to(torch.float64).numpy() for k, t in inputs.items()}
+        self.prob = O.Problem(B=1, F=w.F, P=w.P, H=1, d=w.d, T=w.T, C=w.C)
+        t0 = time.perf_counter()
+        self.cache = {(0, 0): O.frame_states(self.x["k"], self.x["v"], self.prob, 0, 0)}
+        self.t_states = time.perf_counter() - t0
+        self.keys = [w.P * len(softmax_key_frames(f // w.C, w.F, w.C)) + w.T for f in range(w.F)]
+
+    def interior_frame(self):
+        return (self.w.F // self.w.C // 2) * self.w.C
+
+    def time_frames(self, frames):
+        """Seconds per key-weighted frame from timing the given query frames."""
+        x, O = self.x, self.O
+        spent, keys = 0.0, 0
+        for f in frames:
+            rows = np.arange(f * self.w.P, (f + 1) * self.w.P)
+            t0 = time.perf_counter()
+            O.hybrid_attn_rows(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], x["gate_s"], x["gate_l"],
+                               self.prob, 0, 0, rows, frame_state_cache=self.cache)
+            spent += time.perf_counter() - t0
+            keys += self.keys[f]
+        per_head = self.t_states + spent / keys * sum(self.keys)
+        return per_head * self.w.H * self.w.B, spent
+
+
+# ---------------------------------------------------------------- main
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank time over all ranks (NCCL on GPU, gloo on CPU)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return
+    wk = work(w)
+    flops = (wk["softmax_flops"] + wk["linear_flops"]) * world
+    cb = CpuBaseline(w, make_inputs(w))
+    frame = cb.interior_frame()
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        est_s, _ = cb.time_frames([frame])
+        if i >= args.warmup:
+            per_step.append(est_s)
+    est = statistics.median(per_step)
+    value = flops / est / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, world),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cb.cores, "kind": "oracle",
+                         "sample": "fp64 oracle; each step times head 0's query frame %d (softmax rows, readout, "
+                                   "RMSNorm, merge); with head 0's frame states it is scaled by key count to all "
+                                   "frames and heads of one call" % frame},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, world):
+    return {"workload": w.name, "B": w.B, "F": w.F, "P": w.P, "H": w.H, "d": w.d, "T": w.T, "C": w.C,
+            "dtype": w.dtype, "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"}
+
+
+def run_ours(args, w, world, rank, local):
+    from video_diffusion_hybrid_sparse_b200 import binding as vb
+
+    dev_t = make_inputs(w)
+    dev = {k: t.cuda() for k, t in dev_t.items()}
+    out = torch.empty_like(dev["q"])
+    steps = vb.Steps(dev["q"], dev["k"], dev["v"], dev["text_k"], dev["text_v"], dev["gate_s"], dev["gate_l"], out,
+                     frames=w.F, chunk_frames=w.C)
+    stream = torch.cuda.current_stream()
+    wk = work(w)
+    staged = w.dtype == "fp32" or w.d == 32
+    launches_per_step = 4 + (5 if staged else 0)
+
+    for _ in range(args.warmup):
+        steps.all()
+    torch.cuda.synchronize()
+
+    # ------------------------------------------------ device-resident timing
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(KERNELS) + 1)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_id_for(local)) as clk:
+        for s in range(args.steps):
+            ev[s][0].record(stream)
+            for i, name in enumerate(KERNELS):
+                getattr(steps, name)()
+                ev[s][i + 1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    per_kernel = {n: 0.0 for n in KERNELS}
+    total_ms = 0.0
+    for s in range(args.steps):
+        total_ms += ev[s][0].elapsed_time(ev[s][-1])
+        for i, n in enumerate(KERNELS):
+            per_kernel[n] += ev[s][i].elapsed_time(ev[s][i + 1]) / args.steps
+    total_ms = max_over_ranks(total_ms, world)
+    ms = total_ms / args.steps
+
+    # ------------------------------------------------ end to end from pinned host memory
+    host = {k: t.pin_memory() for k, t in dev_t.items()}
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = host_out.numel() * host_out.element_size()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, args.steps // 4)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n_e2e):
+        for k in host:
+            dev[k].copy_(host[k], non_blocking=True)
+        vb.hybrid_attn_fwd(dev["q"], dev["k"], dev["v"], dev["text_k"], dev["text_v"], dev["gate_s"], dev["gate_l"],
+                           frames=w.F, chunk_frames=w.C, out=out, workspace=steps.ws)
+        host_out.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / n_e2e
+
+    flops_call = wk["softmax_flops"] + wk["linear_flops"]
+    value = flops_call * world / (ms * 1e-3) / 1e12
+    pk, src = peaks()
+    tc_peak, hbm = pk["bf16_tflops"], pk["hbm_gbs"]
+    k3_ms = per_kernel["sparse_softmax"]
+    achieved = wk["softmax_flops"] / (k3_ms * 1e-3) / 1e12
+    traffic = recorded_traffic("sparse_softmax", w.name)
+    kern = {}
+    for n, amount, bound in (("state_build", wk["k1_bytes"], "hbm"), ("state_scan", wk["k2_bytes"], "hbm"),
+                             ("readout_merge", wk["k4_bytes"], "hbm"), ("sparse_softmax", wk["softmax_flops"], "tensor")):
+        t = per_kernel[n] * 1e-3
+        if bound == "hbm":
+            a = amount / t / 1e9 if t > 0 else None
+            kern[n] = {"ms": per_kernel[n], "bound": "hbm", "achieved_gbs": a, "frac": a / hbm if a else None}
+        else:
+            a = amount / t / 1e12
+            kern[n] = {"ms": per_kernel[n], "bound": "tensor", "achieved_tflops": a, "frac": a / tc_peak}
+    kern["stage"] = {"ms": per_kernel["stage"]}
+    roof_s = wk["softmax_flops"] / (tc_peak * 1e12) + wk["linear_bytes"] / (hbm * 1e9)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(w, world),
+        "roofline": {"bound": "tensor", "kernel": "sparse_softmax", "achieved": achieved, "peak": tc_peak,
+                     "unit": "TFLOP/s", "frac": achieved / tc_peak, "traffic": traffic,
+                     "peak_source": f"{src} bf16 burst (MEASURED_PEAKS.json)" if src == "measured" else "fallback",
+                     "frac_of_sustained": achieved / pk.get("bf16_tflops_sustained", tc_peak),
+                     "frac_of_spec": achieved / SPEC_TFLOPS},
+        "call_roofline": {"roofline_ms": roof_s * 1e3, "frac": roof_s * 1e3 / ms},
+        "kernels": kern,
+        "e2e": {"value": flops_call * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = CpuBaseline(w, dev_t)
+        frames = sorted({0, cb.interior_frame(), w.F - 1})
+        est_s, spent = cb.time_frames(frames)
+        line["cpu_baseline"] = {"value": flops_call / est_s / 1e12, "unit": "TFLOP/s", "cores": cb.cores,
+                                "kind": "oracle", "ms_per_call_est": est_s * 1e3, "sampled_s": spent + cb.t_states,
+                                "sample": "fp64 oracle: head 0's frame states and query frames %s (softmax rows, "
+                                          "readout, RMSNorm, merge), scaled by key count to all frames and heads "
+                                          "of one call" % frames}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="768p_bf16", choices=sorted(BY_NAME))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = BY_NAME[args.workload]
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, w, world, rank)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, w, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -62,6 +62,8 @@ WORKLOADS = [
     Workload("chunk5_bf16", 1, 45, 1024, 16, 128, 256, 5, "bf16", "normal", 2),
     Workload("768p_bf16", 1, 15, 4032, 24, 128, 512, 1, "bf16", "rms", 3),
     Workload("768p_long_bf16", 1, 60, 4032, 24, 128, 512, 5, "bf16", "rms", 4),
+    # profiling shape: the 768p latent with 4 of its 24 heads (inputs still larger than L2)
+    Workload("768p_h4_bf16", 1, 15, 4032, 4, 128, 512, 1, "bf16", "rms", 5),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
 
