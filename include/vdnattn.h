@@ -153,6 +153,30 @@ VDN_API vdn_status vdn_sparse_softmax(const void* q, const void* k, const void* 
 VDN_API vdn_status vdn_readout_merge(const void* q, const void* gate_s, const void* gate_l,
                              void* out, const vdn_cfg* cfg, void* stream);
 
+/* For callers that cannot allocate device memory (code running inside another
+ * runtime's plugin/operator interface that hands over tensors but no
+ * allocator, or latency-critical loops where cudaMalloc is not acceptable).
+ * There is no counterpart on the article's pages: this is an interface
+ * addition, not part of the method.
+ *
+ * Same operation, arguments and layouts as vdn_hybrid_attn_fwd, but
+ * cfg->workspace / workspace_bytes are ignored: the scratch is a static device
+ * array of vdn_static_scratch_bytes() (32 MiB) inside the library, which every
+ * GPU that loads the library holds until the process exits.  The first call on
+ * a device (with that device current) looks up the array's device address
+ * with cudaGetSymbolAddress; make that first call before any stream capture.
+ * Nothing is allocated.  Returns VDN_ERR_WORKSPACE, before any CUDA call, when
+ * vdn_workspace_bytes(cfg) exceeds the static size (it fits, e.g., 15 frames
+ * x 256 tokens x 8 heads x head_dim 64).  All calls on a device share the one
+ * array: calls whose GPU work overlaps race and must be ordered by the caller.
+ * The status slot of the array is cleared on every call. */
+VDN_API vdn_status vdn_hybrid_attn_fwd_static(const void* q, const void* k, const void* v,
+                                              const void* text_k, const void* text_v,
+                                              const void* gate_s, const void* gate_l, void* out,
+                                              const vdn_cfg* cfg, void* stream);
+/* Size in bytes of the static scratch used by vdn_hybrid_attn_fwd_static. */
+VDN_API size_t vdn_static_scratch_bytes(void);
+
 #ifdef __cplusplus
 }
 #endif

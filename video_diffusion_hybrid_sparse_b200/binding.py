@@ -24,7 +24,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "po
 
 EXPORTED = ["vdn_version", "vdn_status_string", "vdn_validate", "vdn_workspace_bytes", "vdn_plan_membership",
             "vdn_membership_device", "vdn_hybrid_attn_fwd", "vdn_stage_inputs", "vdn_state_build",
-            "vdn_state_scan", "vdn_sparse_softmax", "vdn_readout_merge"]
+            "vdn_state_scan", "vdn_sparse_softmax", "vdn_readout_merge", "vdn_hybrid_attn_fwd_static",
+            "vdn_static_scratch_bytes"]
 
 
 class VdnError(RuntimeError):
@@ -71,8 +72,10 @@ def library() -> ctypes.CDLL:
         lib.vdn_state_scan.argtypes = [C, P]
         lib.vdn_sparse_softmax.argtypes = [P, P, P, P, P, C, P]
         lib.vdn_readout_merge.argtypes = [P, P, P, P, C, P]
+        lib.vdn_hybrid_attn_fwd_static.argtypes = [P, P, P, P, P, P, P, P, C, P]
+        lib.vdn_static_scratch_bytes.restype = ctypes.c_size_t
         for name in EXPORTED:
-            if name not in ("vdn_version", "vdn_status_string", "vdn_workspace_bytes"):
+            if name not in ("vdn_version", "vdn_status_string", "vdn_workspace_bytes", "vdn_static_scratch_bytes"):
                 getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
