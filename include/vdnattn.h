@@ -92,7 +92,7 @@ typedef struct {
   int32_t dtype;            /* vdn_dtype of q, k, v, text, gates and out */
   float softmax_scale;      /* <= 0 selects 1/sqrt(head_dim) */
   float rms_eps;            /* < 0 selects 1e-6 */
-  const float* rms_weight;  /* device [heads, head_dim] fp32 gamma, or NULL for ones */
+  const float* rms_weight;  /* device [heads, head_dim] fp32 gamma (16-byte aligned), or NULL for ones */
   int32_t debug_flags;      /* VDN_OUT_* / VDN_EXPORT_STATES, 0 in production */
   int32_t reserved0;        /* must be 0 */
   void* workspace;          /* device, 256-byte aligned, >= vdn_workspace_bytes(cfg) bytes */

@@ -83,7 +83,7 @@ vdn_status check_ws(const vdn_cfg* cfg, const Geom& g) {
   if (!cfg->workspace || cfg->workspace_bytes < g.total) return VDN_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(cfg->workspace) & 255u) != 0) return VDN_ERR_ALIGNMENT;
   if (cfg->status_word && (reinterpret_cast<uintptr_t>(cfg->status_word) & 3u) != 0) return VDN_ERR_ALIGNMENT;
-  if (cfg->rms_weight && (reinterpret_cast<uintptr_t>(cfg->rms_weight) & 3u) != 0) return VDN_ERR_ALIGNMENT;
+  if (cfg->rms_weight && (reinterpret_cast<uintptr_t>(cfg->rms_weight) & 15u) != 0) return VDN_ERR_ALIGNMENT;
   return VDN_OK;
 }
 

@@ -1,7 +1,7 @@
 // k1_state_build.cu - per-slice linear-attention states of the VDN-H3 linear
 // branch (article section 双分支混合注意力机制: the frame-wise linear memory).
 //
-// For one slice of up to 1024 key tokens of one non-anchor frame (or of the
+// For one slice of up to 2048 key tokens of one non-anchor frame (or of the
 // text), one batch and one head, it computes on the tensor cores
 //
 //     [S | z] = phi(K)^T [V | 1],   S: d x d,  z: d,   phi = elu + 1,
@@ -12,7 +12,7 @@
 // readout consumes.
 //
 // Per 128-token tile: TMA brings the K tile and the V tile (128-byte swizzle);
-// four warps apply phi in place on the K tile (zeroing rows past the slice and
+// eight warps apply phi in place on the K tile (zeroing rows past the slice and
 // padded head_dim columns) and fence it to the async proxy; one thread issues
 //   D[:, 0:Dp]    += phi(K)^T V      (A and B both MN-major, M = 128 = head_dim slots)
 //   D[:, Dp:Dp+16] += phi(K)^T 1     (B = a block of ones)
@@ -38,11 +38,13 @@ struct K1Layout {
 };
 
 enum { kFull = 0, kPhi = 3, kEmpty = 6, kAcc = 9, kNumBars1 = 10 };
+constexpr int kPhiThreads = 256;  // warps 2..9
+constexpr int kK1Threads = 64 + kPhiThreads;
 
 }  // namespace
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kK1Threads, 1)
     k1_state_build(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const __grid_constant__ CUtensorMap tm_tk, const __grid_constant__ CUtensorMap tm_tv,
                    const __grid_constant__ K1Params p) {
@@ -81,7 +83,7 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&bars[kFull + s], 1);
-      mbar_init(&bars[kPhi + s], 128);
+      mbar_init(&bars[kPhi + s], kPhiThreads);
       mbar_init(&bars[kEmpty + s], 1);
     }
     mbar_init(&bars[kAcc], 1);
@@ -152,18 +154,18 @@ __global__ void __launch_bounds__(192, 1)
       mma_commit(&bars[kAcc]);
     }
   } else {
-    // warps 2..5: phi workers, then the epilogue
+    // warps 2..9: phi workers; warps 2..5 then read the accumulator out
     const int tid = threadIdx.x - 64;
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
       const int st = i % L::kStages;
       const bool got = mbar_wait(&bars[kFull + st], (i / L::kStages) & 1, ab);
       if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
-      phi_tile_inplace(smem + st * L::kStage, D / 64, ntok - i * 128, g.d, tid);
+      phi_tile_inplace(smem + st * L::kStage, D / 64, ntok - i * 128, g.d, tid, kPhiThreads);
       fence_proxy_async_smem();
       mbar_arrive(&bars[kPhi + st]);
     }
-    if (ok) {
+    if (ok && warp < 6) {
       const bool got = mbar_wait(&bars[kAcc], 0, ab);
       if (!__any_sync(0xffffffffu, !got)) {
         tc_fence_after();
@@ -204,12 +206,12 @@ cudaError_t launch_state_build(const Maps& m, const K1Params& p, cudaStream_t st
     const int smem = K1Layout<128>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(k1_state_build<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    k1_state_build<128><<<grid, 192, smem, st>>>(m.k, m.v, m.tk, m.tv, p);
+    k1_state_build<128><<<grid, kK1Threads, smem, st>>>(m.k, m.v, m.tk, m.tv, p);
   } else {
     const int smem = K1Layout<64>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(k1_state_build<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    k1_state_build<64><<<grid, 192, smem, st>>>(m.k, m.v, m.tk, m.tv, p);
+    k1_state_build<64><<<grid, kK1Threads, smem, st>>>(m.k, m.v, m.tk, m.tv, p);
   }
   return cudaGetLastError();
 }

@@ -3,21 +3,21 @@
 // the local window, a backward state the context after it, both without the
 // window and the anchor frames; the text is written at half weight into each).
 //
-// Per element e of [S | z] (batch, head, row n in [0, Dp], 8 consecutive
+// Per element group of [S | z] (batch, head, row n in [0, Dp], 4 consecutive
 // columns a) one thread:
-//   1. sums the slice partials of every non-anchor frame into its chunk:
-//      cs[c] = sum_{f in chunk c, f not an anchor} [S|z]_f      (fp32)
-//      and the text partials into t;
-//   2. forms, exactly by running sums in both directions,
-//      F_c = t/2 + sum_{c' <= c-2} cs[c'],   B_c = t/2 + sum_{c' >= c+2} cs[c'],
-//      M_c = F_c + B_c;
+//   1. sums the slice partials of every non-anchor frame into its chunk,
+//      cs[c] = sum_{f in chunk c, f not an anchor} [S|z]_f  (fp32; partials
+//      are read in batches of four for memory-level parallelism), and the text
+//      partials into t;
+//   2. turns cs into running prefix sums P[c] = sum_{c' <= c} cs[c'] and forms
+//      F_c = t/2 + P[c-2],  B_c = t/2 + (P[Nc-1] - P[c+1]),  M_c = F_c + B_c
+//      (B_c is exactly t/2 for the last two chunks);
 //   3. writes M_c as a bf16 hi/lo pair (hi = bf16(M), lo = bf16(M - hi)) into
 //      the readout's B-operand image: rows n (value column; row Dp = z, rows
 //      Dp+1..Dp+15 zero), K = a, K-major with the 128-byte swizzle, so the
 //      readout copies it to shared memory with one bulk copy;
 //   4. optionally exports F_c and B_c in fp32.
-// The chunk sums and backward sums of a thread live in shared memory
-// (2 x n_chunks x 8 floats each).
+// The chunk sums live in shared memory, thread-fastest ([Nc][4][threads]).
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -25,7 +25,7 @@ namespace vdn {
 
 namespace {
 
-__device__ __forceinline__ uint32_t mt_offset(int n, int a, int Dp, int rows) {
+__device__ __forceinline__ uint32_t mt_offset(int n, int a, int rows) {
   // byte offset of element (row n, column a) in one K-major SW128 B-tile image
   const int ac = a >> 6;
   const int chunk = ((a & 63) >> 3) ^ (n & 7);
@@ -35,105 +35,93 @@ __device__ __forceinline__ uint32_t mt_offset(int n, int a, int Dp, int rows) {
 }  // namespace
 
 __global__ void k2_state_scan(const __grid_constant__ K2Params p, int n_threads_total) {
-  extern __shared__ float scan_smem[];  // [2][Nc][8][blockDim.x]: thread-fastest, no bank conflicts
+  extern __shared__ float scan_smem[];
   const Geom& g = p.g;
   const int Dp = g.Dp;
   const int Nc = g.Nc;
-  const int gid = blockIdx.x * blockDim.x + threadIdx.x;
   const int T_ = blockDim.x;
-  float* cs = scan_smem + threadIdx.x;  // cs[(c * 8 + e) * T_]
+  float* cs = scan_smem + threadIdx.x;  // cs[(c * 4 + e) * T_]
+  const int gid = blockIdx.x * blockDim.x + threadIdx.x;
   if (gid >= n_threads_total) return;
 
-  const int a8s = Dp / 8;
+  const int a4s = Dp / 4;
   int rem = gid;
-  const int a8 = rem % a8s; rem /= a8s;
+  const int a4 = rem % a4s; rem /= a4s;
   const int n = rem % (Dp + 1); rem /= (Dp + 1);
   const int h = rem % g.H;
   const int b = rem / g.H;
   const size_t part_stride = (size_t)g.B * g.H * (Dp + 1) * Dp;
-  const size_t elem = (((size_t)b * g.H + h) * (Dp + 1) + n) * Dp + a8 * 8;
+  const float* src0 = p.parts + (((size_t)b * g.H + h) * (Dp + 1) + n) * Dp + a4 * 4;
 
   for (int c = 0; c < Nc; ++c)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) cs[(c * 8 + e) * T_] = 0.f;
-  float t[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) t[e] = 0.f;
+    for (int e = 0; e < 4; ++e) cs[(c * 4 + e) * T_] = 0.f;
+  float t[4] = {0.f, 0.f, 0.f, 0.f};
 
-  for (int pp = 0; pp < g.n_parts; ++pp) {
-    const float4* src = reinterpret_cast<const float4*>(p.parts + pp * part_stride + elem);
-    const float4 x0 = src[0], x1 = src[1];
-    const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-    if (pp < g.n_video_parts) {
-      float* dst = cs + (part_frame(pp, g) / g.C) * 8 * T_;
+  for (int p0 = 0; p0 < g.n_parts; p0 += 4) {
+    float4 x[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) dst[e * T_] += x[e];
-    } else {
+    for (int u = 0; u < 4; ++u)
+      x[u] = (p0 + u < g.n_parts) ? __ldg(reinterpret_cast<const float4*>(src0 + (size_t)(p0 + u) * part_stride))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) t[e] += x[e];
+    for (int u = 0; u < 4; ++u) {
+      const int pp = p0 + u;
+      if (pp >= g.n_parts) break;
+      if (pp < g.n_video_parts) {
+        float* dst = cs + (part_frame(pp, g) / g.C) * 4 * T_;
+        dst[0] += x[u].x; dst[T_] += x[u].y; dst[2 * T_] += x[u].z; dst[3 * T_] += x[u].w;
+      } else {
+        t[0] += x[u].x; t[1] += x[u].y; t[2] += x[u].z; t[3] += x[u].w;
+      }
     }
   }
 
-  // bw[c] = sum of cs[c'] for c' >= bwd_first_chunk(c), by a backward running sum
-  float* bw = cs + (size_t)T_ * Nc * 8;  // second array, same layout
-  {
-    float run[8];
+  // running prefix sums in place
+  for (int c = 1; c < Nc; ++c)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) run[e] = 0.f;
-    int next = Nc - 1;  // highest chunk not yet added to run
-    for (int c = Nc - 1; c >= 0; --c) {
-      for (; next >= 0 && next >= bwd_first_chunk(c); --next)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) run[e] += cs[(next * 8 + e) * T_];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) bw[(c * 8 + e) * T_] = run[e];
-    }
-  }
+    for (int e = 0; e < 4; ++e) cs[(c * 4 + e) * T_] += cs[((c - 1) * 4 + e) * T_];
 
   const int rows = Dp + 16;
   const size_t tile_bytes = (size_t)rows * Dp * 2;
   const int d = g.d;
   const bool exp_row = (n < d) || (n == Dp);
   const int exp_n = (n == Dp) ? d : n;
-  float fw[8];  // sum of cs[c'] for c' <= fwd_last_chunk(c), forward running sum
-#pragma unroll
-  for (int e = 0; e < 8; ++e) fw[e] = 0.f;
-  int next_f = 0;  // lowest chunk not yet added to fw
+  const uint32_t off = mt_offset(n, a4 * 4, rows);
   for (int c = 0; c < Nc; ++c) {
-    for (; next_f < Nc && next_f <= fwd_last_chunk(c); ++next_f)
+    const int fl = fwd_last_chunk(c), bf = bwd_first_chunk(c);
+    float Fv[4], Bv[4], M[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) fw[e] += cs[(next_f * 8 + e) * T_];
-    float Fv[8], Bv[8], M[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      Fv[e] = 0.5f * t[e] + fw[e];
-      Bv[e] = 0.5f * t[e] + bw[(c * 8 + e) * T_];
+    for (int e = 0; e < 4; ++e) {
+      const float pre = fl >= 0 ? cs[(fl * 4 + e) * T_] : 0.f;
+      const float suf = bf <= Nc - 1 ? cs[((Nc - 1) * 4 + e) * T_] - cs[((bf - 1) * 4 + e) * T_] : 0.f;
+      Fv[e] = 0.5f * t[e] + pre;
+      Bv[e] = 0.5f * t[e] + suf;
       M[e] = Fv[e] + Bv[e];
     }
     uint8_t* tile = p.mt + (((size_t)b * Nc + c) * g.H + h) * 2 * tile_bytes;
-    uint32_t hi[4], lo[4];
+    uint32_t hi[2], lo[2];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
+    for (int e = 0; e < 2; ++e) {
       const __nv_bfloat16 h0 = __float2bfloat16_rn(M[2 * e]), h1 = __float2bfloat16_rn(M[2 * e + 1]);
       const float r0 = M[2 * e] - __bfloat162float(h0), r1 = M[2 * e + 1] - __bfloat162float(h1);
       hi[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
       lo[e] = pack_bf16x2(r0, r1);
     }
-    const uint32_t off = mt_offset(n, a8 * 8, Dp, rows);
-    *reinterpret_cast<uint4*>(tile + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    *reinterpret_cast<uint4*>(tile + tile_bytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    *reinterpret_cast<uint2*>(tile + off) = make_uint2(hi[0], hi[1]);
+    *reinterpret_cast<uint2*>(tile + tile_bytes + off) = make_uint2(lo[0], lo[1]);
     if (n == Dp) {
       for (int z = Dp + 1; z < rows; ++z) {  // zero padding rows
-        const uint32_t oz = mt_offset(z, a8 * 8, Dp, rows);
-        *reinterpret_cast<uint4*>(tile + oz) = make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(tile + tile_bytes + oz) = make_uint4(0, 0, 0, 0);
+        const uint32_t oz = mt_offset(z, a4 * 4, rows);
+        *reinterpret_cast<uint2*>(tile + oz) = make_uint2(0, 0);
+        *reinterpret_cast<uint2*>(tile + tile_bytes + oz) = make_uint2(0, 0);
       }
     }
     if (p.export_fwd && exp_row) {
       const size_t base = ((((size_t)b * Nc + c) * g.H + h) * (d + 1) + exp_n) * d;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int a = a8 * 8 + e;
+      for (int e = 0; e < 4; ++e) {
+        const int a = a4 * 4 + e;
         if (a < d) {
           p.export_fwd[base + a] = Fv[e];
           p.export_bwd[base + a] = Bv[e];
@@ -144,19 +132,19 @@ __global__ void k2_state_scan(const __grid_constant__ K2Params p, int n_threads_
 }
 
 int k2_threads_per_block(int Nc) {
-  // chunk sums + backward sums in shared memory: Nc * 64 bytes per thread, at most ~200 KB per block
-  int tpb = (200 * 1024) / (Nc * 64);
+  // chunk sums in shared memory: Nc * 16 bytes per thread, at most ~96 KB per block
+  int tpb = (96 * 1024) / (Nc * 16);
   tpb = (tpb / 32) * 32;
-  if (tpb > 128) tpb = 128;
+  if (tpb > 256) tpb = 256;
   return tpb;
 }
 
 cudaError_t launch_state_scan(const K2Params& p, cudaStream_t st) {
   const Geom& g = p.g;
-  const int total = g.B * g.H * (g.Dp + 1) * (g.Dp / 8);
+  const int total = g.B * g.H * (g.Dp + 1) * (g.Dp / 4);
   const int tpb = k2_threads_per_block(g.Nc);
   if (tpb < 32) return cudaErrorInvalidValue;
-  const int smem = tpb * g.Nc * 64;
+  const int smem = tpb * g.Nc * 16;
   cudaError_t e = cudaFuncSetAttribute(k2_state_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   k2_state_scan<<<(total + tpb - 1) / tpb, tpb, smem, st>>>(p, total);

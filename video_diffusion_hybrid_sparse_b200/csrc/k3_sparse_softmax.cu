@@ -44,6 +44,12 @@ struct K3Layout {
   static constexpr int kBytes = kBar + 256 + 1024;  // + barriers + alignment slack
 };
 
+// One column pair in kPolyEvery takes the FMA-pipe exponential.
+#ifndef VDN_POLY_EVERY
+#define VDN_POLY_EVERY 8
+#endif
+constexpr int kPolyEvery = VDN_POLY_EVERY;
+
 struct Item {
   int b, h, c, pair, ntiles, row0;  // row0: first query row of the item within the batch
 };
@@ -277,9 +283,16 @@ __global__ void __launch_bounds__(384, 1)
             for (int i = 0; i < 128; ++i)
               if (i >= n_valid) s[i] = __float_as_uint(-INFINITY);
           }
-          float mx = __uint_as_float(s[0]);
+          // row max: four independent fmax3 chains
+          float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-          for (int i = 1; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(s[i]));
+          for (int i = 0; i < 128; i += 8) {
+            a0 = fmax3(a0, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
+            a1 = fmax3(a1, __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
+            a2 = fmax3(a2, __uint_as_float(s[i + 4]), __uint_as_float(s[i + 5]));
+            a3 = fmax3(a3, __uint_as_float(s[i + 6]), __uint_as_float(s[i + 7]));
+          }
+          const float mx = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
           const float mxs = mx * sl2;
           // lazy rescale: move the running max only when this tile's max is
           // more than 2^8 above it (O is rescaled below, once P is stored)
@@ -296,17 +309,39 @@ __global__ void __launch_bounds__(384, 1)
             }
           }
           l_run *= alpha;
+          // p = 2^(s * scale * log2(e) - m): the exponent argument and the
+          // row sum in packed f32x2; every kPolyEvery-th column pair is
+          // exponentiated on the FMA pipe, the rest on the special-function unit.
+          const uint64_t sl2x2 = f32x2_pack(sl2, sl2);
+          const uint64_t negm = f32x2_pack(-m_run, -m_run);
+          uint64_t lsum0 = f32x2_pack(0.f, 0.f), lsum1 = lsum0;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint32_t pk[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const float p0 = ex2_approx(fmaf(__uint_as_float(s[32 * i + 2 * e]), sl2, -m_run));
-              const float p1 = ex2_approx(fmaf(__uint_as_float(s[32 * i + 2 * e + 1]), sl2, -m_run));
-              l_run += p0 + p1;
+              const uint64_t sx = f32x2_pack(__uint_as_float(s[32 * i + 2 * e]), __uint_as_float(s[32 * i + 2 * e + 1]));
+              float x0, x1;
+              f32x2_unpack(f32x2_fma(sx, sl2x2, negm), x0, x1);
+              float p0, p1;
+              if ((e % kPolyEvery) == kPolyEvery - 1) {
+                p0 = exp2_fma(x0);
+                p1 = exp2_fma(x1);
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              if (e & 1) lsum1 = f32x2_add(lsum1, f32x2_pack(p0, p1));
+              else lsum0 = f32x2_add(lsum0, f32x2_pack(p0, p1));
               pk[e] = pack_bf16x2(p0, p1);
             }
             tmem_st16(tmem_addr(tmem, lane_base, t * 128 + 16 * i), pk);
+          }
+          {
+            float l0, l1, l2, l3;
+            f32x2_unpack(lsum0, l0, l1);
+            f32x2_unpack(lsum1, l2, l3);
+            l_run += (l0 + l1) + (l2 + l3);
           }
           if (rescale) {
             // O_t is quiescent here: S_t(j) completing implies PV_t(j-1) completed

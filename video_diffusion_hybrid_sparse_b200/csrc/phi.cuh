@@ -11,11 +11,13 @@ __device__ __forceinline__ float phi_f(float x) { return x > 0.f ? x + 1.f : __e
 // Tile: 128 rows x (nbox * 64) bf16 columns as loaded by TMA with 128-byte
 // swizzle (box b at byte offset b * 16384, row r at r * 128 inside a box, the
 // 16-byte chunk index XOR-ed with r % 8).  Rows >= n_valid and columns >=
-// d_real become 0; every other element x becomes bf16(phi(x)).  Called by 128
-// threads with tid in [0, 128).
-__device__ __forceinline__ void phi_tile_inplace(uint8_t* tile, int nbox, int n_valid, int d_real, int tid) {
+// d_real become 0; every other element x becomes bf16(phi(x)).  Called by
+// nthreads threads with tid in [0, nthreads).
+__device__ __forceinline__ void phi_tile_inplace(uint8_t* tile, int nbox, int n_valid, int d_real, int tid,
+                                                 int nthreads) {
   const int nchunks = nbox * 1024;
-  for (int q = tid; q < nchunks; q += 128) {
+#pragma unroll 4
+  for (int q = tid; q < nchunks; q += nthreads) {
     const int bx = q >> 10, w = q & 1023;
     const int row = w >> 3, c16 = w & 7;
     const int a0 = bx * 64 + ((c16 ^ (row & 7)) << 3);

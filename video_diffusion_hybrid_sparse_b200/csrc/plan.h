@@ -24,7 +24,7 @@
 namespace vdn {
 
 constexpr int kMaxChunks = 256;     // chunk-order table carried in kernel parameters
-constexpr int kSliceTokens = 1024;  // tokens per state-build work item
+constexpr int kSliceTokens = 2048;  // tokens per state-build work item
 constexpr int kBlockM = 128;        // query rows per tile
 constexpr int kBlockN = 128;        // keys per tile
 

@@ -48,6 +48,51 @@ __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// ------------------------------------------------------------------ packed fp32 math
+
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f32x2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+// (a * b + c) on two fp32 lanes in one instruction
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x on the FMA/ALU pipes (no special-function unit), for x <= 64.
+// Cody-Waite style reduction x = n + f, n = round(x) by the 1.5 * 2^23
+// magic-number addition, f in [-1/2, 1/2]; 2^f by a degree-3 polynomial
+// fitted for minimax relative error (Lawson's algorithm; coefficients from
+// csrc/exp2_poly.py, max relative error 7.5e-5 in float32); 2^n applied by
+// adding n to the exponent field.  x is clamped at -126 so the result stays a
+// (tiny) non-negative float; masked -inf scores give 2^-126-ish, not 0.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = __fadd_rn(x, 12582912.0f);  // 1.5 * 2^23: n in the low mantissa bits
+  const float n = __fadd_rn(t, -12582912.0f);
+  const float f = __fadd_rn(x, -n);
+  float p = fmaf(0.05517149344086647f, f, 0.24261093139648438f);
+  p = fmaf(p, f, 0.6932609677314758f);
+  p = fmaf(p, f, 0.9999280571937561f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 // ------------------------------------------------------------------ abort / status
 
 // Status shared by the warps of one CTA.  A wait that runs out sets `abort`
