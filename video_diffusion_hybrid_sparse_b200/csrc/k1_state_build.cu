@@ -12,7 +12,7 @@
 // readout consumes.
 //
 // Per 128-token tile: TMA brings the K tile and the V tile (128-byte swizzle);
-// eight warps apply phi in place on the K tile (zeroing rows past the slice and
+// sixteen warps apply phi in place on the K tile (zeroing rows past the slice and
 // padded head_dim columns) and fence it to the async proxy; one thread issues
 //   D[:, 0:Dp]    += phi(K)^T V      (A and B both MN-major, M = 128 = head_dim slots)
 //   D[:, Dp:Dp+16] += phi(K)^T 1     (B = a block of ones)
@@ -38,7 +38,7 @@ struct K1Layout {
 };
 
 enum { kFull = 0, kPhi = 3, kEmpty = 6, kAcc = 9, kNumBars1 = 10 };
-constexpr int kPhiThreads = 256;  // warps 2..9
+constexpr int kPhiThreads = 512;  // warps 2..17
 constexpr int kK1Threads = 64 + kPhiThreads;
 
 }  // namespace
@@ -58,8 +58,10 @@ __global__ void __launch_bounds__(kK1Threads, 1)
   int* abort_flag = reinterpret_cast<int*>(smem + L::kBar + kNumBars1 * 8 + 4);
 
   const Geom& g = p.g;
-  const int part = blockIdx.x;
-  const int bh = blockIdx.y;
+  // (batch, head) is the fastest grid index: CTAs that run together read
+  // whole [H, d] token rows of k and v rather than scattered 256-byte pieces
+  const int bh = blockIdx.x;
+  const int part = blockIdx.y;
   const int b = bh / g.H, h = bh % g.H;
   const uint32_t warp = warp_id(), lane = lane_id();
 
@@ -154,7 +156,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
       mma_commit(&bars[kAcc]);
     }
   } else {
-    // warps 2..9: phi workers; warps 2..5 then read the accumulator out
+    // warps 2..17: phi workers; warps 2..5 then read the accumulator out
     const int tid = threadIdx.x - 64;
     bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
@@ -200,7 +202,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
 }
 
 cudaError_t launch_state_build(const Maps& m, const K1Params& p, cudaStream_t st) {
-  dim3 grid(p.g.n_parts, p.g.B * p.g.H);
+  dim3 grid(p.g.B * p.g.H, p.g.n_parts);
   if (p.g.n_parts == 0) return cudaSuccess;
   if (p.g.Dp == 128) {
     const int smem = K1Layout<128>::kBytes;

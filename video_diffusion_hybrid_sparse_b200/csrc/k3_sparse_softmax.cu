@@ -175,27 +175,30 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kBlockN, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      // descriptors of tile 0 / stage 0; tiles, stages and K steps add byte offsets >> 4
+      const uint64_t q_desc0 = smem_desc(smem_u32(sQ), 16, 1024, kLayoutSw128);
+      const uint64_t k_desc0 = smem_desc(smem_u32(sK), 16, 1024, kLayoutSw128);
+      const uint64_t v_desc0 = smem_desc(smem_u32(sV), 16384, 1024, kLayoutSw128);
       uint32_t kv_cnt = 0, item_cnt = 0, p_cnt[2] = {0, 0};
       bool ok = true;
 
       auto issue_qk = [&](int t, int st) {
         const uint32_t d_tmem = tmem + t * 128;
+        const uint64_t qd = q_desc0 + (uint64_t)((t * L::kTile) >> 4);
+        const uint64_t kd = k_desc0 + (uint64_t)((st * L::kTile) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint64_t a = smem_desc(q_addr + t * L::kTile + off, 16, 1024, kLayoutSw128);
-          const uint64_t b = smem_desc(k_addr + st * L::kTile + off, 16, 1024, kLayoutSw128);
-          mma_ss(d_tmem, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+          mma_ss(d_tmem, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int st, bool acc) {
         const uint32_t d_tmem = tmem + 256 + t * D;
+        const uint64_t vd = v_desc0 + (uint64_t)((st * L::kTile) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk) {
-          const uint64_t b = smem_desc(v_addr + st * L::kTile + kk * 2048, 16384, 1024, kLayoutSw128);
-          mma_ts(d_tmem, tmem + t * 128 + kk * 8, b, idesc_pv, (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < kBlockN / 16; ++kk)
+          mma_ts(d_tmem, tmem + t * 128 + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
+                 (acc || kk > 0) ? 1u : 0u);
       };
 
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++item_cnt) {

@@ -2,22 +2,29 @@
 // hybrid attention (article sections 双分支混合注意力机制 and
 // 自适应门控融合双分支输出).
 //
-// One CTA (256 threads) handles 128 query rows of one (batch, chunk, head):
-//   1. TMA loads the q tile (128-byte swizzle) and one bulk copy brings the
-//      chunk's readout operand M_c = F_c + B_c as a bf16 hi/lo pair
-//      (rows: value column b, row Dp = z; K = head_dim slot a);
-//   2. phi is applied to the q tile in place;
-//   3. one thread issues D = phi(Q) M_hi^T + phi(Q) M_lo^T on the tensor cores
-//      (M = 128, N = Dp + 16, fp32 in TMEM): columns [0, Dp) are the
-//      numerators phi(q)^T M, column Dp is the denominator phi(q) . z;
-//   4. two warps share each TMEM row (one per half of the columns):
-//      o_l = num / den (0 when the states of the chunk hold no token), the
-//      row's sum of squares is combined through shared memory, and
-//      r = o_l / sqrt(mean(o_l^2) + eps) is staged in shared memory (fp32,
-//      16-byte chunks XOR-swizzled by row, over the no longer needed operand
-//      buffers);
-//   5. a coalesced pass, 16 bytes per thread per item, reads o_s and both
-//      gates, applies gamma, and writes out = sigmoid(g_s) o_s + sigmoid(g_l) r.
+// Work item: 128 query rows (a tile) of one (batch, chunk, head).  Persistent
+// CTAs: with S = max(1, SMs / H) streams, CTA k keeps head k % H and walks the
+// tile positions (batch, chunk, tile) s, s + S, s + 2S, ... of stream
+// s = k / H.  At any moment the CTAs therefore cover every head of a few
+// neighbouring tiles, so together they read whole [H, d] token rows from HBM
+// rather than scattered 256-byte pieces, and consecutive items of a CTA mostly
+// share the chunk's readout operand M_c.  Warp roles:
+//   * warp 0 (one thread): bulk-copies M_c = F_c + B_c as a bf16 hi/lo pair
+//     (rows: value column b, row Dp = z; K = head_dim slot a; already in the
+//     K-major 128-byte-swizzled operand image) whenever (batch, chunk, head)
+//     changes, and TMA-loads each q tile into one of two buffers;
+//   * warp 1 (one thread): D = phi(Q) M_hi^T + phi(Q) M_lo^T on the tensor
+//     cores (M = 128, N = Dp + 16, fp32) into one of two TMEM accumulators:
+//     columns [0, Dp) are the numerators phi(q)^T M, column Dp the
+//     denominator phi(q) . z;
+//   * warps 2-9 (256 threads): apply phi to q tile i in place, then finish
+//     tile i-1 while the MMA of tile i runs: two warps per TMEM row compute
+//     o_l = num / den (0 when the chunk's states hold no token) and the
+//     row's RMS, stage r = o_l / sqrt(mean(o_l^2) + eps) in shared memory, and
+//     a coalesced pass reads o_s and both gates (prefetched into L2 one tile
+//     ahead), applies gamma and writes out = sigmoid(g_s) o_s + sigmoid(g_l) r.
+// Every wait is bounded; the worker warps agree on giving up through a
+// barrier with an OR reduction, so none is left waiting for another.
 #include "kernels.h"
 #include "phi.cuh"
 #include "sm100.cuh"
@@ -29,32 +36,27 @@ namespace {
 template <int D>
 struct K4Layout {
   static constexpr int kRows = D + 16;
-  static constexpr int kA = 0;
   static constexpr int kATile = 128 * D * 2;
   static constexpr int kBTile = kRows * D * 2;
-  static constexpr int kB = kA + kATile;
-  static constexpr int kR = 0;                 // r staging [128][D] fp32, reuses A and B
-  static constexpr int kRBytes = 128 * D * 4;
-  static constexpr int kOperandEnd = kB + 2 * kBTile;
-  static_assert(kRBytes <= kOperandEnd, "r staging must fit in the operand buffers");
-  static constexpr int kSs = kOperandEnd;      // [2][128] partial sums of squares
+  static constexpr int kA = 0;                       // two q tiles
+  static constexpr int kB = kA + 2 * kATile;         // M_c hi, lo
+  static constexpr int kR = kB + 2 * kBTile;         // r staging [128][D] fp32
+  static constexpr int kSs = kR + 128 * D * 4;       // [2][128] partial sums of squares
   static constexpr int kBar = kSs + 2 * 128 * 4;
-  static constexpr int kBytes = kBar + 64 + 1024;
+  static constexpr int kBytes = kBar + 128 + 1024;
+  static constexpr int kAccCols = D + 16 <= 128 ? 128 : 256;  // one accumulator
 };
 
-__device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + __expf(-x)); }
+enum { kAFull = 0, kAReady = 2, kAEmpty = 4, kAccFull = 6, kAccEmpty = 8, kBFull = 10, kBEmpty = 11, kDone4 = 12,
+       kNumBars4 = 13 };
+constexpr int kWorkers = 256;
+constexpr int kK4Threads = 64 + kWorkers;
 
-template <bool FP32>
-__device__ __forceinline__ void load8(const void* base, size_t idx, float (&x)[8]) {
-  if constexpr (FP32) {
-    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx);
-    const float4 a = __ldg(p), b = __ldg(p + 1);
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-  } else {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + idx));
-    x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x); x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
-    x[4] = bf16_lo(u.z); x[5] = bf16_hi(u.z); x[6] = bf16_lo(u.w); x[7] = bf16_hi(u.w);
-  }
+// sigmoid(x) = (1 + tanh(x / 2)) / 2 with the hardware tanh (one special-function op)
+__device__ __forceinline__ float sigmoid_f(float x) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+  return fmaf(0.5f, t, 0.5f);
 }
 
 template <bool FP32>
@@ -78,37 +80,76 @@ __device__ __forceinline__ float4* r_chunk(uint8_t* base, int row, int j) {
   return reinterpret_cast<float4*>(base + (size_t)row * D * 4 + ((j ^ (row & (kChunks - 1))) << 4));
 }
 
+// Barrier among the 256 worker threads (id 1) that also ORs a predicate:
+// every worker leaves with the same answer.
+__device__ __forceinline__ bool workers_any(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
+}
+
+struct Item4 {
+  int b, h, c, tile, key;
+};
+
+// The i-th item of the CTA (head h, stream s of n_streams).
+__device__ __forceinline__ Item4 decode4(int i, int h, int s, int n_streams, const Geom& g, int tiles) {
+  Item4 it;
+  const int pos = s + i * n_streams;  // (batch, chunk, tile) position
+  it.tile = pos % tiles;
+  const int rem = pos / tiles;
+  it.c = rem % g.Nc;
+  it.b = rem / g.Nc;
+  it.h = h;
+  it.key = rem;  // (batch, chunk) of this head identifies the readout operand
+  return it;
+}
+
 }  // namespace
 
 template <int D, bool FP32>
-__global__ void __launch_bounds__(256)
-    k4_readout_merge(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ K4Params p) {
+__global__ void __launch_bounds__(kK4Threads, 1)
+    k4_readout_merge(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ K4Params p, int n_streams) {
   using L = K4Layout<D>;
   constexpr int kCols = D + 16;
-  constexpr int kAlloc = kCols <= 128 ? 128 : 256;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);  // [0] loads, [1] mma
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + 16);
-  int* abort_flag = reinterpret_cast<int*>(smem + L::kBar + 20);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + kNumBars4 * 8);
+  int* abort_flag = reinterpret_cast<int*>(smem + L::kBar + kNumBars4 * 8 + 4);
   float* ss_part = reinterpret_cast<float*>(smem + L::kSs);
 
   const Geom& g = p.g;
-  const int r0 = blockIdx.x * 128;  // first row of the tile within the chunk
-  const int c = blockIdx.y;
-  const int b = blockIdx.z / g.H, h = blockIdx.z % g.H;
-  const int nrows = min(128, g.rows_per_chunk - r0);
-  const int tid = threadIdx.x;
+  const int tiles = (g.rows_per_chunk + 127) / 128;
+  const int head = blockIdx.x % g.H, stream = blockIdx.x / g.H;
+  const int positions = g.B * g.Nc * tiles;
+  const int n_mine = stream < positions ? (positions - stream + n_streams - 1) / n_streams : 0;
+  const int first = 0, last = n_mine;  // item index i in [first, last)
   const uint32_t warp = warp_id(), lane = lane_id();
 
-  if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars[kAFull + s], 1);
+      mbar_init(&bars[kAReady + s], kWorkers);
+      mbar_init(&bars[kAEmpty + s], 1);
+      mbar_init(&bars[kAccFull + s], 1);
+      mbar_init(&bars[kAccEmpty + s], kWorkers);
+    }
+    mbar_init(&bars[kBFull], 1);
+    mbar_init(&bars[kBEmpty], 1);
+    mbar_init(&bars[kDone4], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, kAlloc);
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 2 * L::kAccCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -117,60 +158,105 @@ __global__ void __launch_bounds__(256)
   const uint32_t tmem = *tmem_slot;
   const CtaAbort ab{abort_flag, p.status};
 
-  if (tid == 0) {
-    mbar_expect_tx(&bars[0], (uint32_t)(L::kATile + 2 * L::kBTile));
-    for (int bx = 0; bx < D / 64; ++bx)
-      tma_load_2d(smem + L::kA + bx * 16384, &tm_q, &bars[0], h * D + bx * 64,
-                  b * (int)g.N + c * g.rows_per_chunk + r0);
-    const uint8_t* src = p.mt + (((size_t)b * g.Nc + c) * g.H + h) * 2 * (size_t)L::kBTile;
-    bulk_load(smem + L::kB, src, (uint32_t)(2 * L::kBTile), &bars[0]);
-  }
-  bool issued = false;
-  bool ok = mbar_wait(&bars[0], 0, ab);
-  if (__syncthreads_or(!ok)) {
-    if (tid == 0) mbar_drain(&bars[0], 0);
-  } else {
-    phi_tile_inplace(smem + L::kA, D / 64, 128, g.d, tid, 256);
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t idesc = idesc_bf16_f32(128, kCols, 0, 0);
-      const uint32_t a_addr = smem_u32(smem + L::kA);
-      const uint32_t b_addr = smem_u32(smem + L::kB);
-#pragma unroll
-      for (int hl = 0; hl < 2; ++hl)
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = smem_desc(a_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kLayoutSw128);
-          const uint64_t bd = smem_desc(b_addr + hl * L::kBTile + (kk >> 2) * (L::kRows * 128) + (kk & 3) * 32, 16,
-                                        1024, kLayoutSw128);
-          mma_ss(tmem, a, bd, idesc, (hl | kk) ? 1u : 0u);
+  if (warp == 0) {
+    // ------------------------------------------------------------ loads
+    if (lane == 0) {
+      int prev_key = -1, b_loads = 0, a_issued = 0;
+      bool ok = true;
+      for (int item = first; item < last && ok; ++item) {
+        const Item4 it = decode4(item, head, stream, n_streams, g, tiles);
+        const int i = item - first, s = i & 1;
+        if (it.key != prev_key) {
+          if (b_loads > 0 && !mbar_wait(&bars[kBEmpty], (b_loads - 1) & 1, ab)) { ok = false; break; }
+          mbar_expect_tx(&bars[kBFull], (uint32_t)(2 * L::kBTile));
+          bulk_load(smem + L::kB, p.mt + (((size_t)it.b * g.Nc + it.c) * g.H + it.h) * 2 * (size_t)L::kBTile,
+                    (uint32_t)(2 * L::kBTile), &bars[kBFull]);
+          ++b_loads;
+          prev_key = it.key;
         }
-      mma_commit(&bars[1]);
-      issued = true;
+        if (!mbar_wait(&bars[kAEmpty + s], ((i >> 1) & 1) ^ 1, ab)) { ok = false; break; }
+        mbar_expect_tx(&bars[kAFull + s], (uint32_t)L::kATile);
+        for (int bx = 0; bx < D / 64; ++bx)
+          tma_load_2d(smem + L::kA + s * L::kATile + bx * 16384, &tm_q, &bars[kAFull + s], it.h * D + bx * 64,
+                      it.b * (int)g.N + it.c * g.rows_per_chunk + it.tile * 128);
+        ++a_issued;
+      }
+      if (!ok) {
+        for (int k = (a_issued > 2 ? a_issued - 2 : 0); k < a_issued; ++k)
+          mbar_drain(&bars[kAFull + (k & 1)], (k >> 1) & 1);
+        if (b_loads > 0) mbar_drain(&bars[kBFull], (b_loads - 1) & 1);
+      }
     }
-    ok = mbar_wait(&bars[1], 0, ab);
-    if (!__syncthreads_or(!ok)) {
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, kCols, 0, 0);
+      int prev_key = -1, b_loads = 0;
+      for (int item = first; item < last; ++item) {
+        const Item4 it = decode4(item, head, stream, n_streams, g, tiles);
+        const int i = item - first, s = i & 1;
+        const uint32_t ph = (i >> 1) & 1;
+        if (it.key != prev_key) {
+          ++b_loads;
+          prev_key = it.key;
+          if (!mbar_wait(&bars[kBFull], (b_loads - 1) & 1, ab)) break;
+        }
+        if (!mbar_wait(&bars[kAReady + s], ph, ab)) break;
+        if (!mbar_wait(&bars[kAccEmpty + s], ph ^ 1, ab)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + L::kA + s * L::kATile);
+        const uint32_t b_addr = smem_u32(smem + L::kB);
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t a = smem_desc(a_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kLayoutSw128);
+            const uint64_t bd = smem_desc(b_addr + hl * L::kBTile + (kk >> 2) * (L::kRows * 128) + (kk & 3) * 32,
+                                          16, 1024, kLayoutSw128);
+            mma_ss(tmem + s * L::kAccCols, a, bd, idesc, (hl | kk) ? 1u : 0u);
+          }
+        mma_commit(&bars[kAccFull + s]);
+        mma_commit(&bars[kAEmpty + s]);
+        const bool key_ends = item + 1 >= last || decode4(item + 1, head, stream, n_streams, g, tiles).key != it.key;
+        if (key_ends) mma_commit(&bars[kBEmpty]);
+      }
+      mma_commit(&bars[kDone4]);
+      mbar_drain(&bars[kDone4], 0);
+    }
+  } else {
+    // ------------------------------------------------------------ workers
+    const int tid = threadIdx.x - 64;
+    const uint32_t quarter = warp & 3, half = (warp - 2) >> 2;
+    const int row = quarter * 32 + lane;
+    const int col0 = half * (D / 2);
+    const int d = g.d;
+    const int c8s = d / 8;
+    // output: 0 merged, 1 softmax branch only, 2 linear read (normalised or raw)
+    const int mode = (p.flags & 1) ? 1 : ((p.flags & 6) ? 2 : 0);
+    const bool use_gamma = p.gamma != nullptr && !(p.flags & 4);
+
+    // Finish tile `item` (slot s): TMEM -> r -> coalesced merge.  Returns false on a timeout.
+    auto finish = [&](int item, int s) -> bool {
+      const Item4 it = decode4(item, head, stream, n_streams, g, tiles);
+      const int i = item - first;
+      const bool got = mbar_wait(&bars[kAccFull + s], (i >> 1) & 1, ab);
+      if (workers_any(!got)) return false;
       tc_fence_after();
-      // ---------------------------------------------------------- TMEM -> r (two warps per row)
-      const uint32_t quarter = warp & 3, half = warp >> 2;
-      const int row = quarter * 32 + lane;
-      const int col0 = half * (D / 2);
-      const int d = g.d;
       float num[D / 2];
 #pragma unroll
-      for (int i = 0; i < D / 64; ++i) {
+      for (int k = 0; k < D / 64; ++k) {
         uint32_t r[32];
-        tmem_ld32(tmem_addr(tmem, quarter * 32, col0 + 32 * i), r);
+        tmem_ld32(tmem_addr(tmem + s * L::kAccCols, quarter * 32, col0 + 32 * k), r);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) num[32 * i + e] = __uint_as_float(r[e]);
+        for (int e = 0; e < 32; ++e) num[32 * k + e] = __uint_as_float(r[e]);
       }
       uint32_t dr;
-      tmem_ld1(tmem_addr(tmem, quarter * 32, D), dr);
+      tmem_ld1(tmem_addr(tmem + s * L::kAccCols, quarter * 32, D), dr);
       tmem_wait_ld();
-      const bool empty = state_tokens(c, g) == 0;
+      tc_fence_before();
+      mbar_arrive(&bars[kAccEmpty + s]);  // the accumulator may be overwritten now
+      const bool empty = state_tokens(it.c, g) == 0;
       const float inv_den = empty ? 0.f : 1.0f / __uint_as_float(dr);
       float ss = 0.f;
 #pragma unroll
@@ -179,7 +265,7 @@ __global__ void __launch_bounds__(256)
         if (col0 + a < d) ss = fmaf(num[a], num[a], ss);
       }
       ss_part[half * 128 + row] = ss;
-      __syncthreads();
+      workers_any(false);
       const float inv_rms = (p.flags & 4) ? 1.0f : rsqrtf((ss_part[row] + ss_part[128 + row]) / (float)d + g.eps);
 #pragma unroll
       for (int j = 0; j < D / 8; ++j) {
@@ -187,47 +273,122 @@ __global__ void __launch_bounds__(256)
                                      num[4 * j + 3] * inv_rms);
         *r_chunk<D>(smem + L::kR, row, col0 / 4 + j) = v;
       }
-      __syncthreads();
-      // ---------------------------------------------------------- coalesced merge
-      const int c8s = d / 8;
+      workers_any(false);
+      // coalesced merge: each thread issues the raw 16-byte loads of a whole
+      // batch of items (eight for bf16 gates, two for fp32) before using any
+      constexpr int kBatch = FP32 ? 2 : 4;
+      constexpr int kGv = FP32 ? 2 : 1;  // 16-byte vectors per 8 gate values
+      const int nrows = min(128, g.rows_per_chunk - it.tile * 128);
       const int items = 128 * c8s;
-      const size_t tok0 = (size_t)b * g.N + (size_t)(c * g.rows_per_chunk + r0);
-#pragma unroll 4
-      for (int it = tid; it < items; it += 256) {
-        const int rr = it / c8s, c8 = it - rr * c8s;
-        if (rr >= nrows) continue;
-        const size_t tok = tok0 + rr;
-        float os[8], gs[8], gl[8], o[8];
-        load8<false>(p.o_s, (tok * g.H + h) * D + c8 * 8, os);
-        load8<FP32>(p.gate_s, (tok * g.H + h) * d + c8 * 8, gs);
-        load8<FP32>(p.gate_l, (tok * g.H + h) * d + c8 * 8, gl);
-        const float4 ra = *r_chunk<D>(smem + L::kR, rr, 2 * c8);
-        const float4 rb = *r_chunk<D>(smem + L::kR, rr, 2 * c8 + 1);
-        float r[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
-        if (p.gamma && !(p.flags & 4)) {
-          const float4 ga = __ldg(reinterpret_cast<const float4*>(p.gamma + h * d + c8 * 8));
-          const float4 gb = __ldg(reinterpret_cast<const float4*>(p.gamma + h * d + c8 * 8) + 1);
-          r[0] *= ga.x; r[1] *= ga.y; r[2] *= ga.z; r[3] *= ga.w;
-          r[4] *= gb.x; r[5] *= gb.y; r[6] *= gb.z; r[7] *= gb.w;
+      const size_t tok0 = (size_t)it.b * g.N + (size_t)(it.c * g.rows_per_chunk + it.tile * 128);
+      for (int e0 = tid; e0 < items; e0 += kBatch * kWorkers) {
+        uint4 vos[kBatch], vgs[kBatch][kGv], vgl[kBatch][kGv];
+        size_t tok[kBatch];
+        int rrs[kBatch], c8v[kBatch];
+        bool valid[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          const int e = e0 + u * kWorkers;
+          const int rr = e / c8s, c8 = e - rr * c8s;
+          valid[u] = e < items && rr < nrows;
+          rrs[u] = valid[u] ? rr : 0;
+          c8v[u] = valid[u] ? c8 : 0;
+          tok[u] = tok0 + rrs[u];
+          const size_t row_h = tok[u] * g.H + it.h;
+          vos[u] = __ldg(reinterpret_cast<const uint4*>(p.o_s + row_h * D + c8v[u] * 8));
+          const uint4* gsp = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.gate_s) +
+                                                            (row_h * d + c8v[u] * 8) * (FP32 ? 4 : 2));
+          const uint4* glp = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.gate_l) +
+                                                            (row_h * d + c8v[u] * 8) * (FP32 ? 4 : 2));
+#pragma unroll
+          for (int k = 0; k < kGv; ++k) {
+            vgs[u][k] = __ldg(gsp + k);
+            vgl[u][k] = __ldg(glp + k);
+          }
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float v;
-          if (p.flags & 1) v = os[e];        // softmax branch only
-          else if (p.flags & 6) v = r[e];    // linear read: normalised (2) or raw (4)
-          else v = sigmoid_f(gs[e]) * os[e] + sigmoid_f(gl[e]) * r[e];
-          o[e] = v;
+        for (int u = 0; u < kBatch; ++u) {
+          const float4 ra = *r_chunk<D>(smem + L::kR, rrs[u], 2 * c8v[u]);
+          const float4 rb = *r_chunk<D>(smem + L::kR, rrs[u], 2 * c8v[u] + 1);
+          float r[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+          if (use_gamma) {
+            const float4 ga = __ldg(reinterpret_cast<const float4*>(p.gamma + it.h * d + c8v[u] * 8));
+            const float4 gb = __ldg(reinterpret_cast<const float4*>(p.gamma + it.h * d + c8v[u] * 8) + 1);
+            r[0] *= ga.x; r[1] *= ga.y; r[2] *= ga.z; r[3] *= ga.w;
+            r[4] *= gb.x; r[5] *= gb.y; r[6] *= gb.z; r[7] *= gb.w;
+          }
+          const uint32_t ow[4] = {vos[u].x, vos[u].y, vos[u].z, vos[u].w};
+          float os[8], gs[8], gl[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            os[2 * k] = bf16_lo(ow[k]);
+            os[2 * k + 1] = bf16_hi(ow[k]);
+          }
+          if constexpr (FP32) {
+            const float* fs = reinterpret_cast<const float*>(&vgs[u][0]);
+            const float* fl = reinterpret_cast<const float*>(&vgl[u][0]);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) { gs[k] = fs[k]; gl[k] = fl[k]; }
+          } else {
+            const uint32_t sw[4] = {vgs[u][0].x, vgs[u][0].y, vgs[u][0].z, vgs[u][0].w};
+            const uint32_t lw[4] = {vgl[u][0].x, vgl[u][0].y, vgl[u][0].z, vgl[u][0].w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              gs[2 * k] = bf16_lo(sw[k]); gs[2 * k + 1] = bf16_hi(sw[k]);
+              gl[2 * k] = bf16_lo(lw[k]); gl[2 * k + 1] = bf16_hi(lw[k]);
+            }
+          }
+          float o[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float merged = sigmoid_f(gs[k]) * os[k] + sigmoid_f(gl[k]) * r[k];
+            o[k] = mode == 0 ? merged : (mode == 1 ? os[k] : r[k]);
+          }
+          if (valid[u]) store8<FP32>(p.out, (tok[u] * g.H + it.h) * d + c8v[u] * 8, o);
         }
-        store8<FP32>(p.out, (tok * g.H + h) * d + c8 * 8, o);
       }
+      workers_any(false);  // r staging is rewritten by the next tile
+      return true;
+    };
+
+    bool ok = true;
+    for (int item = first; item < last && ok; ++item) {
+      const Item4 it = decode4(item, head, stream, n_streams, g, tiles);
+      const int i = item - first, s = i & 1;
+      // bring this tile's o_s and gate rows into L2 for its merge (one tile later):
+      // thread t covers row t % 128 of o_s (t < 128) or of both gates (t >= 128)
+      {
+        const int rr = tid & 127;
+        if (rr < min(128, g.rows_per_chunk - it.tile * 128)) {
+          const size_t row_h = ((size_t)it.b * g.N + (size_t)(it.c * g.rows_per_chunk + it.tile * 128 + rr)) * g.H + it.h;
+          if (tid < 128) {
+            const uint8_t* o = reinterpret_cast<const uint8_t*>(p.o_s + row_h * D);
+#pragma unroll
+            for (int l = 0; l < D * 2 / 128; ++l) prefetch_l2(o + l * 128);
+          } else {
+            const size_t rb = row_h * (size_t)d * (FP32 ? 4 : 2);
+            for (int l = 0; l < d * (FP32 ? 4 : 2); l += 128) {
+              prefetch_l2(static_cast<const uint8_t*>(p.gate_s) + rb + l);
+              prefetch_l2(static_cast<const uint8_t*>(p.gate_l) + rb + l);
+            }
+          }
+        }
+      }
+      const bool got = mbar_wait(&bars[kAFull + s], (i >> 1) & 1, ab);
+      if (workers_any(!got)) { ok = false; break; }
+      phi_tile_inplace(smem + L::kA + s * L::kATile, D / 64, 128, d, tid, kWorkers);
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[kAReady + s]);
+      if (item > first) ok = finish(item - 1, (i - 1) & 1);
     }
+    if (ok && last > first) finish(last - 1, (last - 1 - first) & 1);
   }
-  if (issued) mbar_drain(&bars[1], 0);  // the MMA finished before TMEM is released
+
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kAlloc);
+    tmem_dealloc(tmem, 2 * L::kAccCols);
   }
 }
 
@@ -236,8 +397,15 @@ static cudaError_t launch_k4(const Maps& m, const K4Params& p, cudaStream_t st) 
   const int smem = K4Layout<D>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(k4_readout_merge<D, FP32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((p.g.rows_per_chunk + 127) / 128, p.g.Nc, p.g.B * p.g.H);
-  k4_readout_merge<D, FP32><<<grid, 256, smem, st>>>(m.q, p);
+  const int tiles = (p.g.rows_per_chunk + 127) / 128;
+  const int positions = tiles * p.g.Nc * p.g.B;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int n_streams = sms / p.g.H;
+  if (n_streams < 1) n_streams = 1;
+  if (n_streams > positions) n_streams = positions;
+  k4_readout_merge<D, FP32><<<n_streams * p.g.H, kK4Threads, smem, st>>>(m.q, p, n_streams);
   return cudaGetLastError();
 }
 
