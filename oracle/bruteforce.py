@@ -11,10 +11,12 @@ operand) makes the two disagree:
   routine ``torch.nn.functional.scaled_dot_product_attention`` in float64.
   Mask predicate (VDN-H3 article, section 双分支混合注意力机制): query token i
   may read key token j when their chunks differ by at most one, or when j lies
-  in the first or last latent frame; every text key is readable.
+  in the first or last latent frame; every text key is readable.  Under the
+  GLOBAL anchor reading a query in the first or last frame reads every key.
 * :func:`pairwise_linear` - the linear branch without any state: for each
   query, a weighted mean over every key outside the window and outside the
-  anchors plus every text key taken once, with weights phi(q_i) . phi(k_j).
+  anchors plus every text key taken once, with weights phi(q_i) . phi(k_j)
+  (nothing for a GLOBAL anchor query).
 """
 from __future__ import annotations
 
@@ -28,12 +30,17 @@ def _token_frame_chunk(prob):
     return frame, frame // prob.C
 
 
+def _global_anchor_query(prob, frame) -> np.ndarray:
+    mode = getattr(prob, "anchor_query_mode", "local")
+    return ((frame == 0) | (frame == prob.F - 1)) & (mode == "global")
+
+
 def softmax_mask(prob) -> np.ndarray:
     """bool [N, N + T]: True where query i reads key j in the softmax branch."""
     frame, chunk = _token_frame_chunk(prob)
     near = np.abs(chunk[:, None] - chunk[None, :]) <= 1
     anchor_key = (frame == 0) | (frame == prob.F - 1)
-    video = near | anchor_key[None, :]
+    video = near | anchor_key[None, :] | _global_anchor_query(prob, frame)[:, None]
     text = np.ones((prob.N, prob.T), dtype=bool)
     return np.concatenate([video, text], axis=1)
 
@@ -43,7 +50,7 @@ def linear_mask(prob) -> np.ndarray:
     frame, chunk = _token_frame_chunk(prob)
     far = np.abs(chunk[:, None] - chunk[None, :]) >= 2
     anchor_key = (frame == 0) | (frame == prob.F - 1)
-    return far & ~anchor_key[None, :]
+    return far & ~anchor_key[None, :] & ~_global_anchor_query(prob, frame)[:, None]
 
 
 def dense_masked_softmax(q, k, v, tk, tv, prob) -> np.ndarray:
@@ -84,10 +91,11 @@ def pairwise_linear(q, k, v, tk, tv, prob) -> np.ndarray:
             den = w.sum(axis=1)
             if prob.T:
                 ftk = _elu_plus_one(tk[b, :, h, :])
-                wt = fq @ ftk.T
+                wt = (fq @ ftk.T) * (~_global_anchor_query(prob, np.arange(prob.N) // prob.P))[:, None]
                 num = num + wt @ np.asarray(tv[b, :, h, :], np.float64)
                 den = den + wt.sum(axis=1)
-            has = (lm.sum(axis=1) > 0) | (prob.T > 0)
+            frame = np.arange(prob.N) // prob.P
+            has = ((lm.sum(axis=1) > 0) | (prob.T > 0)) & ~_global_anchor_query(prob, frame)
             o = np.zeros_like(num)
             o[has] = num[has] / den[has, None]
             out[b, :, h, :] = o

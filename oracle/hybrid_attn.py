@@ -29,14 +29,21 @@ Source of every step: the VDN-H3 article "VDN-Minimax-H3 ... 11.23 秒生成
 Readings of points the page leaves open (each also listed in the design doc):
 chunk size C is a parameter (5 in the chunking sentence, 1 in the frame-7
 example); the window is clipped at the sequence ends; anchor frames as queries
-follow the same rule as every other frame; the feature map is
+follow the same rule as every other frame (LOCAL, the default) -- the other
+reading of "the first and last frames also interact with the other frames",
+GLOBAL, where an anchor query attends through the softmax branch to every
+frame and reads nothing through the states, is available as
+``anchor_query_mode="global"``; the feature map is
 phi(x) = elu(x) + 1; the softmax scale is 1/sqrt(d); the two directional
 states are summed before one normalised read (numerator phi(q)^T (S_F + S_B),
 denominator phi(q) . (z_F + z_B)), which is the reading under which a half
 write into each side counts the text once; an empty state (no text and no
 frames) reads as zero; RMSNorm is over head_dim per (token, head) with
 eps = 1e-6 and an optional per-head weight gamma; gates are element-wise
-logits supplied as inputs; text tokens are keys/values only.
+logits supplied as inputs; text tokens are keys/values only.  The two gated
+branch terms sigmoid(g_s) * o_s and sigmoid(g_l) * r are also returned
+separately (the SPLIT output, for callers that apply a projection per branch
+before summing, as the fusion section's per-branch outputs suggest).
 
 Layout: video tensors are [B, N, H, d] with N = F*P frame-major tokens (token n
 lies in frame n // P); text tensors are [B, T, H, d]; gates [B, N, H, d].
@@ -67,6 +74,7 @@ class Problem:
     C: int  # frames per chunk
     scale: float | None = None  # softmax scale; None -> 1/sqrt(d)
     eps: float = 1e-6  # RMSNorm epsilon
+    anchor_query_mode: str = "local"  # "local" or "global" (see module docstring)
 
     @property
     def N(self) -> int:
@@ -85,6 +93,8 @@ class Problem:
             raise ValueError("sizes must be positive (T >= 0)")
         if self.F % self.C:
             raise ValueError("frames must be a whole number of chunks")
+        if self.anchor_query_mode not in ("local", "global"):
+            raise ValueError("anchor_query_mode is 'local' or 'global'")
 
 
 # --------------------------------------------------------------------------
@@ -112,23 +122,35 @@ def window_frames(f: int, F: int, C: int) -> list[int]:
     return list(range(lo * C, (hi + 1) * C))
 
 
-def softmax_frames(f: int, F: int, C: int) -> list[int]:
+def global_anchor_query(f: int, F: int, mode: str) -> bool:
+    """True when query frame f is an anchor that, under the GLOBAL reading,
+    attends to every frame through the softmax branch."""
+    return mode == "global" and f in anchor_frames(F)
+
+
+def softmax_frames(f: int, F: int, C: int, mode: str = "local") -> list[int]:
     """Frames read exactly by the softmax branch: the window plus the anchors,
-    each frame once."""
+    each frame once (every frame for a GLOBAL anchor query)."""
+    if global_anchor_query(f, F, mode):
+        return list(range(F))
     return sorted(set(window_frames(f, F, C)) | set(anchor_frames(F)))
 
 
-def forward_frames(f: int, F: int, C: int) -> list[int]:
+def forward_frames(f: int, F: int, C: int, mode: str = "local") -> list[int]:
     """Frames summed by the forward state: every chunk before the window,
-    anchors excluded."""
+    anchors excluded (none for a GLOBAL anchor query)."""
+    if global_anchor_query(f, F, mode):
+        return []
     c = chunk_of(f, C)
     anchors = set(anchor_frames(F))
     return [g for g in range(F) if chunk_of(g, C) <= c - 2 and g not in anchors]
 
 
-def backward_frames(f: int, F: int, C: int) -> list[int]:
+def backward_frames(f: int, F: int, C: int, mode: str = "local") -> list[int]:
     """Frames summed by the backward state: every chunk after the window,
-    anchors excluded."""
+    anchors excluded (none for a GLOBAL anchor query)."""
+    if global_anchor_query(f, F, mode):
+        return []
     c = chunk_of(f, C)
     anchors = set(anchor_frames(F))
     return [g for g in range(F) if chunk_of(g, C) >= c + 2 and g not in anchors]
@@ -137,7 +159,7 @@ def backward_frames(f: int, F: int, C: int) -> list[int]:
 SOFTMAX, FORWARD, BACKWARD = 1, 2, 3
 
 
-def membership_table(F: int, C: int) -> np.ndarray:
+def membership_table(F: int, C: int, mode: str = "local") -> np.ndarray:
     """uint8 [F, F]: entry (f, g) says how query frame f reads key frame g:
     1 = softmax branch, 2 = forward state, 3 = backward state.  Every key frame
     is read through exactly one branch ("其余帧则进入线性记忆模块")."""
@@ -145,11 +167,11 @@ def membership_table(F: int, C: int) -> np.ndarray:
         raise ValueError("frames must be a whole number of chunks")
     table = np.zeros((F, F), dtype=np.uint8)
     for f in range(F):
-        for g in softmax_frames(f, F, C):
+        for g in softmax_frames(f, F, C, mode):
             table[f, g] = SOFTMAX
-        for g in forward_frames(f, F, C):
+        for g in forward_frames(f, F, C, mode):
             table[f, g] = FORWARD
-        for g in backward_frames(f, F, C):
+        for g in backward_frames(f, F, C, mode):
             table[f, g] = BACKWARD
     return table
 
@@ -176,7 +198,7 @@ def softmax_branch_rows(q, k, v, tk, tv, prob: Problem, b: int, h: int, rows) ->
     frames_of_rows = rows // prob.P
     for f in np.unique(frames_of_rows):
         sel = np.nonzero(frames_of_rows == f)[0]
-        key_rows = _frame_rows(softmax_frames(int(f), prob.F, prob.C), prob.P)
+        key_rows = _frame_rows(softmax_frames(int(f), prob.F, prob.C, prob.anchor_query_mode), prob.P)
         keys = np.concatenate([k[b, key_rows, h, :], tk[b, :, h, :]], axis=0).astype(np.float64)
         vals = np.concatenate([v[b, key_rows, h, :], tv[b, :, h, :]], axis=0).astype(np.float64)
         qf = q[b, rows[sel], h, :].astype(np.float64)
@@ -265,13 +287,16 @@ def state_token_count(c: int, prob: Problem) -> int:
 def linear_readout_rows(q, SF, zF, SB, zB, prob: Problem, b: int, h: int, rows) -> np.ndarray:
     """o_l for query tokens ``rows``: one normalised read of the summed
     states, phi(q)^T (S_F + S_B) / (phi(q) . (z_F + z_B)); zero when the
-    states hold no token."""
+    states hold no token, and zero for GLOBAL anchor queries (they read
+    nothing through the states)."""
     rows = np.asarray(rows, dtype=np.int64)
     out = np.zeros((rows.size, prob.d))
-    chunks = (rows // prob.P) // prob.C
+    frames = rows // prob.P
+    chunks = frames // prob.C
+    reads = np.array([not global_anchor_query(int(f), prob.F, prob.anchor_query_mode) for f in frames], dtype=bool)
     for c in np.unique(chunks):
-        sel = np.nonzero(chunks == c)[0]
-        if state_token_count(int(c), prob) == 0:
+        sel = np.nonzero((chunks == c) & reads)[0]
+        if sel.size == 0 or state_token_count(int(c), prob) == 0:
             continue
         fq = phi(q[b, rows[sel], h, :])
         num = fq @ (SF[c] + SB[c])
@@ -316,14 +341,21 @@ def sigmoid(x):
         return 1.0 / (1.0 + np.exp(-x))
 
 
+def gated_terms(o_s, r, g_s, g_l):
+    """The two gated branch terms (sigmoid(g_s) * o_s, sigmoid(g_l) * r): the
+    SPLIT output."""
+    return sigmoid(g_s) * o_s, sigmoid(g_l) * r
+
+
 def merge(o_s, r, g_s, g_l):
     """out = sigmoid(g_s) * o_s + sigmoid(g_l) * r, element-wise."""
     return sigmoid(g_s) * o_s + sigmoid(g_l) * r
 
 
 def hybrid_attn(q, k, v, tk, tv, g_s, g_l, prob: Problem, gamma=None, text_weights=(0.5, 0.5)):
-    """Whole call.  Returns a dict with out, o_s, o_l, r (all [B, N, H, d]
-    float64), the per-(b, h) states and the membership table.
+    """Whole call.  Returns a dict with out, o_s, o_l, r, and the SPLIT
+    terms out_s = sigmoid(g_s) * o_s, out_l = sigmoid(g_l) * r (all
+    [B, N, H, d] float64), the per-(b, h) states and the membership table.
 
     ``gamma`` is None (ones) or [H, d]."""
     prob.check()
@@ -332,8 +364,9 @@ def hybrid_attn(q, k, v, tk, tv, g_s, g_l, prob: Problem, gamma=None, text_weigh
     g = None if gamma is None else np.asarray(gamma, dtype=np.float64)[None, None, :, :]
     r = rms_norm(o_l, prob.eps, g)
     out = merge(o_s, r, g_s.astype(np.float64), g_l.astype(np.float64))
-    return dict(out=out, o_s=o_s, o_l=o_l, r=r, states=states,
-                membership=membership_table(prob.F, prob.C))
+    out_s, out_l = gated_terms(o_s, r, g_s.astype(np.float64), g_l.astype(np.float64))
+    return dict(out=out, o_s=o_s, o_l=o_l, r=r, out_s=out_s, out_l=out_l, states=states,
+                membership=membership_table(prob.F, prob.C, prob.anchor_query_mode))
 
 
 def hybrid_attn_rows(q, k, v, tk, tv, g_s, g_l, prob: Problem, b: int, h: int, rows,
@@ -354,8 +387,10 @@ def hybrid_attn_rows(q, k, v, tk, tv, g_s, g_l, prob: Problem, b: int, h: int, r
     o_l = linear_readout_rows(q, SF, zF, SB, zB, prob, b, h, rows)
     g = None if gamma is None else np.asarray(gamma, dtype=np.float64)[h]
     r = rms_norm(o_l, prob.eps, g)
-    out = merge(o_s, r, g_s[b, rows, h, :].astype(np.float64), g_l[b, rows, h, :].astype(np.float64))
-    return dict(out=out, o_s=o_s, o_l=o_l, r=r)
+    gs, gl = g_s[b, rows, h, :].astype(np.float64), g_l[b, rows, h, :].astype(np.float64)
+    out = merge(o_s, r, gs, gl)
+    out_s, out_l = gated_terms(o_s, r, gs, gl)
+    return dict(out=out, o_s=o_s, o_l=o_l, r=r, out_s=out_s, out_l=out_l)
 
 
 # --------------------------------------------------------------------------
@@ -367,5 +402,5 @@ def softmax_pairs(prob: Problem) -> int:
     """Number of (query, key) pairs the softmax branch must score, per (b, h)."""
     total = 0
     for f in range(prob.F):
-        total += prob.P * (prob.P * len(softmax_frames(f, prob.F, prob.C)) + prob.T)
+        total += prob.P * (prob.P * len(softmax_frames(f, prob.F, prob.C, prob.anchor_query_mode)) + prob.T)
     return total

@@ -17,6 +17,8 @@
 """
 import os
 
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -256,6 +258,25 @@ def test_softmax_pair_count():
 # ---------------------------------------------------------------- planted mistakes
 
 
+def table_from_masks(prob):
+    """Frame-level membership codes rebuilt from the token-level predicates of
+    the brute-force module: 1 where the softmax mask reads the key frame, 2 / 3
+    where the linear mask reads it from an earlier / later chunk."""
+    sm = BF.softmax_mask(prob)[:, :prob.N]
+    lm = BF.linear_mask(prob)
+    fr = np.arange(prob.N) // prob.P
+    table = np.zeros((prob.F, prob.F), dtype=np.uint8)
+    for f in range(prob.F):
+        qi = f * prob.P
+        for g in range(prob.F):
+            kj = g * prob.P
+            if sm[qi, kj]:
+                table[f, g] = 1
+            elif lm[qi, kj]:
+                table[f, g] = 2 if fr[kj] // prob.C < f // prob.C else 3
+    return table
+
+
 def _pins_hold():
     """Run the cheap pins; return the list of those that fail."""
     failed = []
@@ -263,19 +284,29 @@ def _pins_hold():
     if (O.softmax_frames(7, 15, 1) != g["softmax"] or O.forward_frames(7, 15, 1) != g["forward"]
             or O.backward_frames(7, 15, 1) != g["backward"]):
         failed.append("frame7")
-    for case in [(15, 3, 2, 8, 4, 1), (12, 3, 1, 8, 5, 3)]:
+    for case, mode in [((15, 3, 2, 8, 4, 1), "local"), ((12, 3, 1, 8, 5, 3), "local"),
+                       ((15, 3, 2, 8, 4, 1), "global"), ((12, 3, 1, 8, 5, 3), "global")]:
         prob, x = problem_inputs(*case, seed=77)
+        prob = dataclasses.replace(prob, anchor_query_mode=mode)
         a = (x["q"], x["k"], x["v"], x["text_k"], x["text_v"], prob)
         if not np.allclose(O.softmax_branch(*a), BF.dense_masked_softmax(*a), rtol=1e-10, atol=1e-10):
-            failed.append("sdpa")
+            failed.append("sdpa " + mode)
         if not np.allclose(O.linear_branch(*a)[0], BF.pairwise_linear(*a), rtol=1e-9, atol=1e-10):
-            failed.append("pairwise")
+            failed.append("pairwise " + mode)
+        if not np.array_equal(O.membership_table(prob.F, prob.C, mode), table_from_masks(prob)):
+            failed.append("membership " + mode)
     return failed
 
 
 MUTATIONS = {
     "anchor_in_forward": ("forward_frames",
-                          lambda f, F, C: [g for g in range(F) if g // C <= f // C - 2]),
+                          lambda f, F, C, mode="local": [g for g in range(F) if g // C <= f // C - 2]),
+    "global_anchor_keeps_window_only": ("softmax_frames",
+                                        lambda f, F, C, mode="local": sorted(set(O.window_frames(f, F, C))
+                                                                             | set(O.anchor_frames(F)))),
+    "global_anchor_reads_states": ("forward_frames",
+                                   lambda f, F, C, mode="local": [g for g in range(F) if g // C <= f // C - 2
+                                                                  and g not in O.anchor_frames(F)]),
     "window_not_clipped": ("window_frames",
                            lambda f, F, C: [g for g in range((f // C - 1) * C, (f // C + 2) * C) if 0 <= g < F][:3 * C]
                            if 0 < f // C < F // C - 1 else list(range(0, min(F, 3 * C)))),
@@ -287,7 +318,7 @@ MUTATIONS = {
                              *O.__dict__["_orig_frame_states"](k, v, prob, b, h))),
     "phi_plain_exp": ("phi", lambda x: np.exp(np.asarray(x, np.float64))),
     "softmax_frames_drop_last_anchor": ("softmax_frames",
-                                        lambda f, F, C: sorted(set(O.window_frames(f, F, C)) | {0})),
+                                        lambda f, F, C, mode="local": sorted(set(O.window_frames(f, F, C)) | {0})),
 }
 
 
@@ -299,3 +330,74 @@ def test_planted_mistake_is_caught(name, monkeypatch):
     assert _pins_hold() == []
     monkeypatch.setattr(O, fn_name, bad)
     assert _pins_hold() != [], f"planted mistake {name} went unnoticed"
+
+
+# ---------------------------------------------------------------- GLOBAL anchor queries, SPLIT output
+
+
+def _global(prob):
+    return dataclasses.replace(prob, anchor_query_mode="global")
+
+
+@pytest.mark.parametrize("case", [(15, 3, 2, 8, 4, 1), (10, 2, 1, 4, 3, 2), (12, 3, 1, 8, 5, 3), (1, 5, 1, 4, 2, 1)])
+def test_global_anchor_rows_are_full_attention_with_no_linear_read(case):
+    """GLOBAL reading: a query in the first or last frame attends (unmasked,
+    plain softmax attention evaluated by torch) to all N + T keys and reads
+    nothing through the states, so its output is sigmoid(g_s) * o_s."""
+    prob, x = problem_inputs(*case, seed=31)
+    gp = _global(prob)
+    res = O.hybrid_attn(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], x["gate_s"], x["gate_l"], gp)
+    anchor_rows = np.concatenate([np.arange(f * prob.P, (f + 1) * prob.P) for f in O.anchor_frames(prob.F)])
+    for h in range(prob.H):
+        q = torch.from_numpy(x["q"][0, anchor_rows, h, :])
+        keys = torch.from_numpy(np.concatenate([x["k"][0, :, h, :], x["text_k"][0, :, h, :]]))
+        vals = torch.from_numpy(np.concatenate([x["v"][0, :, h, :], x["text_v"][0, :, h, :]]))
+        p = torch.softmax((q @ keys.T) / np.sqrt(prob.d), dim=-1)
+        np.testing.assert_allclose(res["o_s"][0, anchor_rows, h, :], (p @ vals).numpy(), rtol=1e-12, atol=1e-12)
+    assert np.all(res["o_l"][:, anchor_rows] == 0) and np.all(res["r"][:, anchor_rows] == 0)
+    gs = 1.0 / (1.0 + np.exp(-x["gate_s"][:, anchor_rows]))
+    np.testing.assert_allclose(res["out"][:, anchor_rows], gs * res["o_s"][:, anchor_rows], rtol=1e-14, atol=1e-15)
+
+
+@pytest.mark.parametrize("case", [(15, 3, 2, 8, 4, 1), (12, 3, 1, 8, 5, 3), (10, 2, 1, 4, 0, 5)])
+def test_global_leaves_other_rows_unchanged(case):
+    prob, x = problem_inputs(*case, seed=37)
+    args = (x["q"], x["k"], x["v"], x["text_k"], x["text_v"], x["gate_s"], x["gate_l"])
+    loc = O.hybrid_attn(*args, prob)
+    glo = O.hybrid_attn(*args, _global(prob))
+    inner = np.arange(prob.P, (prob.F - 1) * prob.P)
+    for key in ("out", "o_s", "o_l", "r"):
+        assert np.array_equal(loc[key][:, inner], glo[key][:, inner]), key
+
+
+def test_global_equals_local_when_window_covers_everything():
+    """F = 3 frames of one-frame chunks and no text: the window already holds
+    every frame and the states are empty, so the two readings coincide."""
+    prob, x = problem_inputs(3, 4, 2, 8, 0, 1, seed=41)
+    args = (x["q"], x["k"], x["v"], x["text_k"], x["text_v"], x["gate_s"], x["gate_l"])
+    loc = O.hybrid_attn(*args, prob)
+    glo = O.hybrid_attn(*args, _global(prob))
+    np.testing.assert_array_equal(loc["out"], glo["out"])
+    np.testing.assert_array_equal(loc["membership"], glo["membership"])
+
+
+@pytest.mark.parametrize("F,C", [(15, 1), (15, 5), (45, 5), (12, 3), (2, 1), (1, 1), (6, 6)])
+def test_global_membership(F, C):
+    t = O.membership_table(F, C, "global")
+    assert np.all(t > 0)
+    for f in O.anchor_frames(F):
+        assert np.all(t[f] == O.SOFTMAX)
+    loc = O.membership_table(F, C)
+    inner = [f for f in range(F) if f not in O.anchor_frames(F)]
+    assert np.array_equal(t[inner], loc[inner])
+
+
+def test_split_terms_sum_to_out_and_saturate():
+    prob, x = problem_inputs(15, 3, 2, 8, 4, 1, seed=43)
+    args = (x["q"], x["k"], x["v"], x["text_k"], x["text_v"])
+    res = O.hybrid_attn(*args, x["gate_s"], x["gate_l"], prob)
+    np.testing.assert_allclose(res["out_s"] + res["out_l"], res["out"], rtol=1e-15, atol=1e-15)
+    big = np.full_like(x["gate_s"], 40.0)
+    sat = O.hybrid_attn(*args, big, -big, prob)
+    np.testing.assert_allclose(sat["out_s"], sat["o_s"], rtol=1e-15, atol=1e-15)
+    assert np.max(np.abs(sat["out_l"])) < 1e-15
