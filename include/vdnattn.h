@@ -23,6 +23,18 @@
  *   r[i]   = o_l[i] / sqrt(mean_d(o_l[i]^2) + eps) * gamma[h];
  *   out[i] = sigmoid(gate_s[i]) * o_s[i] + sigmoid(gate_l[i]) * r[i].
  *
+ * Two readings the article leaves open are selectable (vdn_cfg):
+ *   anchor_query_mode = VDN_ANCHOR_LOCAL (default): the rule above for every
+ *     query frame, the anchors included (the frame-7 example's rule);
+ *     VDN_ANCHOR_GLOBAL: a query in frame 0 or F-1 attends by softmax to
+ *     every video frame (plus text) and reads nothing through the states
+ *     (o_l = 0 there, so out = sigmoid(gate_s) * o_s); other rows unchanged.
+ *   output_mode = VDN_OUTPUT_MERGED (default): out as above;
+ *     VDN_OUTPUT_SPLIT: out = sigmoid(gate_s) * o_s and
+ *     cfg->out_linear = sigmoid(gate_l) * r, the two gated branch terms
+ *     (section 自适应门控融合双分支输出: one output per branch), for callers
+ *     that project each branch before summing.
+ *
  * Layouts (row-major, no padding between rows):
  *   q, k, v, gate_s, gate_l, out : [batch, frames*tokens_per_frame, heads, head_dim]
  *   text_k, text_v               : [batch, text_tokens, heads, head_dim]
@@ -73,6 +85,9 @@ typedef enum {
 
 typedef enum { VDN_BF16 = 0, VDN_FP32 = 1 } vdn_dtype;
 
+typedef enum { VDN_ANCHOR_LOCAL = 0, VDN_ANCHOR_GLOBAL = 1 } vdn_anchor_query_mode;
+typedef enum { VDN_OUTPUT_MERGED = 0, VDN_OUTPUT_SPLIT = 1 } vdn_output_mode;
+
 /* debug_flags: what vdn_readout_merge writes into out instead of the merge. */
 enum {
   VDN_OUT_SOFTMAX_ONLY = 1, /* out = o_s (no gate) */
@@ -94,12 +109,15 @@ typedef struct {
   float rms_eps;            /* < 0 selects 1e-6 */
   const float* rms_weight;  /* device [heads, head_dim] fp32 gamma (16-byte aligned), or NULL for ones */
   int32_t debug_flags;      /* VDN_OUT_* / VDN_EXPORT_STATES, 0 in production */
-  int32_t reserved0;        /* must be 0 */
+  int32_t anchor_query_mode; /* vdn_anchor_query_mode; 0 = LOCAL */
   void* workspace;          /* device, 256-byte aligned, >= vdn_workspace_bytes(cfg) bytes */
   size_t workspace_bytes;
   int32_t* status_word;     /* optional device int32; set to VDN_ERR_TIMEOUT by a kernel that gave up */
   float* export_fwd;        /* VDN_EXPORT_STATES: device [B, F/C, H, d+1, d] fp32; row d holds z */
   float* export_bwd;        /* same layout, backward states */
+  int32_t output_mode;      /* vdn_output_mode; 0 = MERGED.  SPLIT excludes the VDN_OUT_* debug flags */
+  int32_t reserved1;        /* must be 0 */
+  void* out_linear;         /* SPLIT only: device [B, N, H, d] in dtype, 16-byte aligned; else ignored */
 } vdn_cfg;
 
 /* Library version, (major << 16) | minor. */
@@ -116,7 +134,8 @@ VDN_API size_t vdn_workspace_bytes(const vdn_cfg* cfg);
 
 /* Host-only membership table of the frame-7 rule: table[f*F + g] = 1 when query
  * frame f reads key frame g through the softmax branch, 2 through the forward
- * state, 3 through the backward state.  table is HOST memory of F*F bytes. */
+ * state, 3 through the backward state (under VDN_ANCHOR_GLOBAL the rows of
+ * frames 0 and F-1 are all 1).  table is HOST memory of F*F bytes. */
 VDN_API vdn_status vdn_plan_membership(const vdn_cfg* cfg, uint8_t* table);
 
 /* The same table produced on the GPU by the index logic the kernels use
@@ -125,7 +144,8 @@ VDN_API vdn_status vdn_plan_membership(const vdn_cfg* cfg, uint8_t* table);
 VDN_API vdn_status vdn_membership_device(const vdn_cfg* cfg, uint8_t* table_dev, void* stream);
 
 /* Whole call: staging (fp32 or head_dim 32 only), state build, scan, sparse
- * softmax, readout + merge, all on stream.  out: [B, N, H, d] in dtype. */
+ * softmax, readout + merge, all on stream.  out: [B, N, H, d] in dtype (and
+ * cfg->out_linear under VDN_OUTPUT_SPLIT). */
 VDN_API vdn_status vdn_hybrid_attn_fwd(const void* q, const void* k, const void* v,
                                const void* text_k, const void* text_v,
                                const void* gate_s, const void* gate_l, void* out,

@@ -71,9 +71,33 @@ def test_validate_rejects_unknown_dtype_and_flags():
     cfg = vb.make_cfg(shape(), debug_flags=64)
     assert lib.vdn_validate(ctypes.byref(cfg)) == 1
     cfg = vb.make_cfg(shape())
-    cfg.reserved0 = 3
+    cfg.reserved1 = 3
+    assert lib.vdn_validate(ctypes.byref(cfg)) == 1
+    for mode in (2, -1):
+        cfg = vb.make_cfg(shape())
+        cfg.anchor_query_mode = mode
+        assert lib.vdn_validate(ctypes.byref(cfg)) == 1
+        cfg = vb.make_cfg(shape())
+        cfg.output_mode = mode
+        assert lib.vdn_validate(ctypes.byref(cfg)) == 1
+    cfg = vb.make_cfg(shape(), anchor_query_mode=vb.ANCHOR_GLOBAL)
+    assert lib.vdn_validate(ctypes.byref(cfg)) == 0
+    # SPLIT excludes the debug outputs
+    cfg = vb.make_cfg(shape(), debug_flags=vb.OUT_SOFTMAX_ONLY)
+    cfg.output_mode = vb.OUTPUT_SPLIT
     assert lib.vdn_validate(ctypes.byref(cfg)) == 1
     assert lib.vdn_validate(None) == 1
+
+
+def test_cfg_struct_layout_matches_header():
+    """Offsets of the fields that follow the pointers (the ctypes mirror of
+    vdn_cfg must match the C layout on LP64)."""
+    assert vb.VdnCfg.anchor_query_mode.offset == 52
+    assert vb.VdnCfg.workspace.offset == 56
+    assert vb.VdnCfg.export_bwd.offset == 88
+    assert vb.VdnCfg.output_mode.offset == 96
+    assert vb.VdnCfg.out_linear.offset == 104
+    assert ctypes.sizeof(vb.VdnCfg) == 112
 
 
 def test_workspace_bytes():
@@ -114,6 +138,12 @@ def test_call_errors_before_any_launch():
     assert lib.vdn_state_scan(ctypes.byref(cfg), None) == 1
     cfg.debug_flags = 0
     assert lib.vdn_plan_membership(ctypes.byref(cfg), None) == 1
+    cfg.output_mode = vb.OUTPUT_SPLIT  # SPLIT without its second output buffer
+    assert lib.vdn_hybrid_attn_fwd(*args, ctypes.byref(cfg), None) == 1
+    assert lib.vdn_readout_merge(p, p, p, p, ctypes.byref(cfg), None) == 1
+    assert lib.vdn_hybrid_attn_fwd_static(*args, ctypes.byref(cfg), None) == 1
+    cfg.out_linear = p + 4
+    assert lib.vdn_hybrid_attn_fwd(*args, ctypes.byref(cfg), None) == 3
 
 
 EDGE = [(1, 1), (2, 1), (2, 2), (3, 1), (3, 3), (4, 2), (5, 1), (6, 3), (15, 1), (15, 5), (45, 5), (60, 5),
@@ -123,3 +153,4 @@ EDGE = [(1, 1), (2, 1), (2, 2), (3, 1), (3, 3), (4, 2), (5, 1), (6, 3), (15, 1),
 @pytest.mark.parametrize("F,C", EDGE + [(w.F, w.C) for w in WORKLOADS])
 def test_host_membership_matches_oracle(F, C):
     np.testing.assert_array_equal(vb.plan_membership(F, C), O.membership_table(F, C))
+    np.testing.assert_array_equal(vb.plan_membership(F, C, vb.ANCHOR_GLOBAL), O.membership_table(F, C, "global"))

@@ -59,9 +59,9 @@ def np64(t):
     return t.to(torch.float64).cpu().numpy()
 
 
-def oracle_full(w: Workload, inputs, gamma=None):
+def oracle_full(w: Workload, inputs, gamma=None, mode="local"):
     x = {k: np64(t) for k, t in inputs.items()}
-    prob = O.Problem(B=w.B, F=w.F, P=w.P, H=w.H, d=w.d, T=w.T, C=w.C)
+    prob = O.Problem(B=w.B, F=w.F, P=w.P, H=w.H, d=w.d, T=w.T, C=w.C, anchor_query_mode=mode)
     return O.hybrid_attn(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], x["gate_s"], x["gate_l"], prob,
                          gamma=gamma)
 
@@ -117,6 +117,44 @@ def test_branches_match_oracle(w):
     o_l = run(w, dev, debug_flags=vb.OUT_LINEAR_RAW).float().cpu().numpy()
     scale = np.abs(ref["o_l"]).max()
     assert_close(o_l, ref["o_l"], f"{w.name} o_l", abs_tol=TOL_ABS * scale)
+
+
+# ----------------------------------------------------------------- GLOBAL anchor queries, SPLIT output
+
+
+GLOBAL_CASES = [SMALL[i] for i in (0, 2, 3, 4, 5, 7, 10, 12)]
+
+
+@pytest.mark.parametrize("F,C,P,T", [(15, 1, 16, 8), (45, 5, 4, 3), (1, 1, 5, 2), (2, 1, 5, 2), (6, 6, 2, 1),
+                                     (12, 3, 2, 2)])
+def test_device_membership_global_matches_oracle(F, C, P, T):
+    np.testing.assert_array_equal(vb.membership_device(F, C, P, T, anchor_query_mode=vb.ANCHOR_GLOBAL),
+                                  O.membership_table(F, C, "global"))
+
+
+@pytest.mark.parametrize("w", GLOBAL_CASES, ids=[w.name for w in GLOBAL_CASES])
+def test_global_anchor_mode_matches_oracle(w):
+    inputs = make_inputs(w)
+    dev = to_dev(inputs)
+    ref = oracle_full(w, inputs, mode="global")
+    out = run(w, dev, anchor_query_mode=vb.ANCHOR_GLOBAL)
+    assert_close(out.float().cpu().numpy(), ref["out"], f"{w.name} out (GLOBAL)")
+    o_s = run(w, dev, anchor_query_mode=vb.ANCHOR_GLOBAL, debug_flags=vb.OUT_SOFTMAX_ONLY)
+    assert_close(o_s.float().cpu().numpy(), ref["o_s"], f"{w.name} o_s (GLOBAL)")
+
+
+@pytest.mark.parametrize("w", [SMALL[0], SMALL[1], SMALL[3]], ids=["tiny", "small", "c5_ragged"])
+def test_split_output_matches_oracle(w):
+    inputs = make_inputs(w)
+    dev = to_dev(inputs)
+    ref = oracle_full(w, inputs)
+    out_lin = torch.empty_like(dev["q"])
+    out = run(w, dev, out_linear=out_lin)
+    assert_close(out.float().cpu().numpy(), ref["out_s"], f"{w.name} sigmoid(g_s) o_s")
+    assert_close(out_lin.float().cpu().numpy(), ref["out_l"], f"{w.name} sigmoid(g_l) r")
+    merged = run(w, dev).float()
+    # the two stored terms add up to the merged output up to one rounding of each
+    assert_close((out.float() + out_lin.float()).cpu().numpy(), merged.cpu().numpy(), f"{w.name} split sum")
 
 
 @pytest.mark.parametrize("w", [SMALL[0], SMALL[2], SMALL[3]], ids=["tiny", "ragged", "c5_ragged"])
@@ -209,3 +247,25 @@ def test_workload_sampled_rows(name, heads):
                                  prob, 0, 0, rows)
         got = out[0, torch.from_numpy(rows).cuda(), h, :].float().cpu().numpy()
         assert_close(got, ref["out"], f"{name} head {h}")
+
+
+def test_global_anchor_mode_sampled_rows_768p():
+    """GLOBAL at the 768p shape: anchor rows attend to all 60,480 video keys
+    plus text; sampled rows of both anchor frames and of inner frames."""
+    w = BY_NAME["768p_bf16"]
+    inputs = make_inputs(w)
+    dev = to_dev(inputs)
+    out = run(w, dev, anchor_query_mode=vb.ANCHOR_GLOBAL)
+    del dev
+    rng = np.random.default_rng(11)
+    last = (w.F - 1) * w.P
+    rows = np.unique(np.concatenate([[0, 127, 128, 4031, last, last + 127, last + 128, w.N - 1],
+                                     rng.integers(0, w.P, 6), last + rng.integers(0, w.P, 6),
+                                     rng.integers(w.P, last, 6)]))
+    prob = O.Problem(B=1, F=w.F, P=w.P, H=1, d=w.d, T=w.T, C=w.C, anchor_query_mode="global")
+    for h in (0, 17):
+        x = {k: np64(t[:, :, h:h + 1, :]) for k, t in inputs.items()}
+        ref = O.hybrid_attn_rows(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], x["gate_s"], x["gate_l"],
+                                 prob, 0, 0, rows)
+        got = out[0, torch.from_numpy(rows).cuda(), h, :].float().cpu().numpy()
+        assert_close(got, ref["out"], f"768p GLOBAL head {h}")

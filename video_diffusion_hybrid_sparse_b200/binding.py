@@ -41,10 +41,12 @@ class VdnCfg(ctypes.Structure):
         ("chunk_frames", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("softmax_scale", ctypes.c_float), ("rms_eps", ctypes.c_float),
         ("rms_weight", ctypes.c_void_p),
-        ("debug_flags", ctypes.c_int32), ("reserved0", ctypes.c_int32),
+        ("debug_flags", ctypes.c_int32), ("anchor_query_mode", ctypes.c_int32),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("status_word", ctypes.c_void_p),
         ("export_fwd", ctypes.c_void_p), ("export_bwd", ctypes.c_void_p),
+        ("output_mode", ctypes.c_int32), ("reserved1", ctypes.c_int32),
+        ("out_linear", ctypes.c_void_p),
     ]
 
 
@@ -99,8 +101,13 @@ class Shape:
         return self.F * self.P
 
 
+ANCHOR_LOCAL, ANCHOR_GLOBAL = 0, 1
+OUTPUT_MERGED, OUTPUT_SPLIT = 0, 1
+
+
 def make_cfg(s: Shape, *, softmax_scale: float = 0.0, rms_eps: float = -1.0, rms_weight=None,
-             debug_flags: int = 0, workspace=None, status=None, export=None) -> VdnCfg:
+             debug_flags: int = 0, workspace=None, status=None, export=None,
+             anchor_query_mode: int = ANCHOR_LOCAL, out_linear=None) -> VdnCfg:
     cfg = VdnCfg()
     cfg.batch, cfg.frames, cfg.tokens_per_frame = s.B, s.F, s.P
     cfg.heads, cfg.head_dim, cfg.text_tokens, cfg.chunk_frames = s.H, s.d, s.T, s.C
@@ -109,7 +116,9 @@ def make_cfg(s: Shape, *, softmax_scale: float = 0.0, rms_eps: float = -1.0, rms
     cfg.rms_eps = rms_eps
     cfg.rms_weight = _ptr(rms_weight)
     cfg.debug_flags = debug_flags
-    cfg.reserved0 = 0
+    cfg.anchor_query_mode = anchor_query_mode
+    cfg.output_mode = OUTPUT_SPLIT if out_linear is not None else OUTPUT_MERGED
+    cfg.out_linear = _ptr(out_linear)
     if workspace is not None:
         cfg.workspace = workspace.data_ptr()
         cfg.workspace_bytes = workspace.numel() * workspace.element_size()
@@ -164,18 +173,22 @@ def workspace_for(s: Shape, device) -> torch.Tensor:
 
 def hybrid_attn_fwd(q, k, v, text_k, text_v, gate_s, gate_l, *, frames: int, chunk_frames: int, out=None,
                     softmax_scale: float = 0.0, rms_eps: float = -1.0, rms_weight=None, debug_flags: int = 0,
-                    workspace=None, status=None, export=None, stream=None) -> torch.Tensor:
+                    workspace=None, status=None, export=None, stream=None,
+                    anchor_query_mode: int = ANCHOR_LOCAL, out_linear=None) -> torch.Tensor:
     """The whole hybrid attention call on the current CUDA stream.
 
     q, k, v, gate_s, gate_l: [B, F*P, H, d]; text_k, text_v: [B, T, H, d];
-    all contiguous CUDA tensors of one dtype (bf16 or fp32)."""
+    all contiguous CUDA tensors of one dtype (bf16 or fp32).  With
+    ``out_linear`` (a tensor like q) the SPLIT output is written: ``out``
+    gets sigmoid(gate_s) * o_s and ``out_linear`` sigmoid(gate_l) * r."""
     s = shape_of(q, text_k, frames, chunk_frames)
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
         workspace = workspace_for(s, q.device)
     cfg = make_cfg(s, softmax_scale=softmax_scale, rms_eps=rms_eps, rms_weight=rms_weight,
-                   debug_flags=debug_flags, workspace=workspace, status=status, export=export)
+                   debug_flags=debug_flags, workspace=workspace, status=status, export=export,
+                   anchor_query_mode=anchor_query_mode, out_linear=out_linear)
     code = library().vdn_hybrid_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(text_k), _ptr(text_v),
                                          gate_s.data_ptr(), gate_l.data_ptr(), out.data_ptr(),
                                          ctypes.byref(cfg), _stream(stream))
@@ -188,12 +201,14 @@ class Steps:
     :func:`hybrid_attn_fwd`), for per-kernel timing and stream overlap."""
 
     def __init__(self, q, k, v, text_k, text_v, gate_s, gate_l, out, *, frames, chunk_frames, workspace=None,
-                 debug_flags=0, rms_weight=None, export=None, status=None):
+                 debug_flags=0, rms_weight=None, export=None, status=None, anchor_query_mode=ANCHOR_LOCAL,
+                 out_linear=None):
         self.t = (q, k, v, text_k, text_v, gate_s, gate_l, out)
         self.s = shape_of(q, text_k, frames, chunk_frames)
         self.ws = workspace if workspace is not None else workspace_for(self.s, q.device)
         self.cfg = make_cfg(self.s, workspace=self.ws, debug_flags=debug_flags, rms_weight=rms_weight,
-                            export=export, status=status)
+                            export=export, status=status, anchor_query_mode=anchor_query_mode,
+                            out_linear=out_linear)
         self.lib = library()
 
     def stage(self, stream=None):
@@ -227,19 +242,22 @@ class Steps:
         self.readout_merge(stream)
 
 
-def plan_membership(F: int, C: int) -> np.ndarray:
+def plan_membership(F: int, C: int, anchor_query_mode: int = ANCHOR_LOCAL) -> np.ndarray:
     """Host membership table from the library (1 softmax, 2 forward, 3 backward)."""
     s = Shape(1, F, 1, 1, 64, 0, C)
     table = np.zeros((F, F), dtype=np.uint8)
-    _check(library().vdn_plan_membership(ctypes.byref(make_cfg(s)), table.ctypes.data), "vdn_plan_membership")
+    cfg = make_cfg(s, anchor_query_mode=anchor_query_mode)
+    _check(library().vdn_plan_membership(ctypes.byref(cfg), table.ctypes.data), "vdn_plan_membership")
     return table
 
 
-def membership_device(F: int, C: int, P: int = 1, T: int = 0, device="cuda") -> np.ndarray:
+def membership_device(F: int, C: int, P: int = 1, T: int = 0, device="cuda",
+                      anchor_query_mode: int = ANCHOR_LOCAL) -> np.ndarray:
     """The membership table as the kernels' index logic produces it on the GPU."""
     s = Shape(1, F, P, 1, 64, T, C)
     table = torch.zeros((F, F), dtype=torch.uint8, device=device)
-    _check(library().vdn_membership_device(ctypes.byref(make_cfg(s)), table.data_ptr(), _stream()),
+    cfg = make_cfg(s, anchor_query_mode=anchor_query_mode)
+    _check(library().vdn_membership_device(ctypes.byref(cfg), table.data_ptr(), _stream()),
            "vdn_membership_device")
     torch.cuda.synchronize()
     return table.cpu().numpy()

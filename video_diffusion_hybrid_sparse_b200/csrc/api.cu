@@ -23,7 +23,13 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 vdn_status make_geom(const vdn_cfg* cfg, Geom& g) {
   if (!cfg) return VDN_ERR_INVALID_ARG;
   if (cfg->batch < 1 || cfg->frames < 1 || cfg->tokens_per_frame < 1 || cfg->heads < 1 || cfg->text_tokens < 0 ||
-      cfg->chunk_frames < 1 || cfg->reserved0 != 0)
+      cfg->chunk_frames < 1 || cfg->reserved1 != 0)
+    return VDN_ERR_INVALID_ARG;
+  if (cfg->anchor_query_mode != VDN_ANCHOR_LOCAL && cfg->anchor_query_mode != VDN_ANCHOR_GLOBAL)
+    return VDN_ERR_INVALID_ARG;
+  if (cfg->output_mode != VDN_OUTPUT_MERGED && cfg->output_mode != VDN_OUTPUT_SPLIT) return VDN_ERR_INVALID_ARG;
+  if (cfg->output_mode == VDN_OUTPUT_SPLIT &&
+      (cfg->debug_flags & (VDN_OUT_SOFTMAX_ONLY | VDN_OUT_LINEAR_ONLY | VDN_OUT_LINEAR_RAW)))
     return VDN_ERR_INVALID_ARG;
   if (cfg->frames % cfg->chunk_frames != 0) return VDN_ERR_INVALID_ARG;
   if (cfg->head_dim != 32 && cfg->head_dim != 64 && cfg->head_dim != 128) return VDN_ERR_UNSUPPORTED;
@@ -58,6 +64,7 @@ vdn_status make_geom(const vdn_cfg* cfg, Geom& g) {
   g.rows_per_chunk = g.C * g.P;
   g.n_pairs = (g.rows_per_chunk + 2 * kBlockM - 1) / (2 * kBlockM);
   g.mt_rows = g.Dp + 16;
+  g.anchor_global = cfg->anchor_query_mode == VDN_ANCHOR_GLOBAL;
   g.scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.0f / std::sqrt((float)g.d);
   g.eps = cfg->rms_eps < 0.f ? 1e-6f : cfg->rms_eps;
 
@@ -209,13 +216,20 @@ vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s,
   p.scale_log2 = g.scale * 1.4426950408889634f;
   p.o_s = reinterpret_cast<__nv_bfloat16*>(ws(cfg, g.off_os));
   p.status = status_ptr(cfg, g);
-  p.items_per_chunk = g.B * g.H * g.n_pairs;
-  p.n_items = g.Nc * p.items_per_chunk;
-  // longest chunks first (static longest-processing-time order)
-  std::vector<int> order(g.Nc);
-  std::iota(order.begin(), order.end(), 0);
-  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return kv_tiles(a, g) > kv_tiles(b, g); });
-  for (int i = 0; i < g.Nc; ++i) p.chunk_order[i] = order[i];
+  // query segments, longest key set first (static longest-processing-time order)
+  QSeg segs[kMaxSegs];
+  const int n = query_segments(g, segs);
+  std::stable_sort(segs, segs + n, [&](const QSeg& a, const QSeg& b) {
+    return seg_kv_tiles(a.c, g) > seg_kv_tiles(b.c, g);
+  });
+  p.n_segs = n;
+  p.seg_item0[0] = 0;
+  for (int k = 0; k < n; ++k) {
+    p.segs[k] = segs[k];
+    const int pairs = (segs[k].nrows + 2 * kBlockM - 1) / (2 * kBlockM);
+    p.seg_item0[k + 1] = p.seg_item0[k] + g.B * g.H * pairs;
+  }
+  p.n_items = p.seg_item0[n];
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -235,6 +249,7 @@ vdn_status step_readout_merge(const vdn_cfg* cfg, const Geom& g, const Srcs& s, 
   p.gate_s = gs;
   p.gate_l = gl;
   p.out = out;
+  p.out_linear = cfg->output_mode == VDN_OUTPUT_SPLIT ? cfg->out_linear : nullptr;
   p.flags = cfg->debug_flags & (VDN_OUT_SOFTMAX_ONLY | VDN_OUT_LINEAR_ONLY | VDN_OUT_LINEAR_RAW);
   p.status = status_ptr(cfg, g);
   return cuda_status(launch_readout_merge(m, p, st));
@@ -293,7 +308,7 @@ vdn_status vdn_plan_membership(const vdn_cfg* cfg, uint8_t* table) {
     for (int x = 0; x < g.F; ++x) {
       const int cx = x / g.C;
       uint8_t code;
-      if ((cx >= wlo && cx <= whi) || is_anchor(x, g.F)) code = 1;
+      if ((cx >= wlo && cx <= whi) || is_anchor(x, g.F) || no_linear_read(f, g)) code = 1;
       else if (cx <= fwd_last_chunk(c)) code = 2;
       else code = 3;
       table[f * g.F + x] = code;
@@ -357,6 +372,7 @@ vdn_status vdn_readout_merge(const void* q, const void* gate_s, const void* gate
   if (s != VDN_OK) return s;
   s = check_inputs(cfg, g, {q, gate_s, gate_l, out}, {});
   if (s != VDN_OK) return s;
+  if (cfg->output_mode == VDN_OUTPUT_SPLIT && (s = check_ptrs({cfg->out_linear})) != VDN_OK) return s;
   return step_readout_merge(cfg, g, kernel_srcs(cfg, g, q, q, q, q, q), gate_s, gate_l, out,
                             static_cast<cudaStream_t>(stream));
 }
@@ -368,6 +384,7 @@ vdn_status vdn_hybrid_attn_fwd(const void* q, const void* k, const void* v, cons
   if (s != VDN_OK) return s;
   s = check_inputs(cfg, g, {q, k, v, gate_s, gate_l, out}, {text_k, text_v});
   if (s != VDN_OK) return s;
+  if (cfg->output_mode == VDN_OUTPUT_SPLIT && (s = check_ptrs({cfg->out_linear})) != VDN_OK) return s;
   if ((cfg->debug_flags & VDN_EXPORT_STATES) && (!cfg->export_fwd || !cfg->export_bwd)) return VDN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Srcs src = kernel_srcs(cfg, g, q, k, v, text_k, text_v);

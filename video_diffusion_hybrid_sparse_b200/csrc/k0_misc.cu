@@ -41,21 +41,23 @@ cudaError_t launch_stage(const void* src, int fp32_in, __nv_bfloat16* dst, long 
   return cudaGetLastError();
 }
 
-// table[f * F + x]: 1 if the softmax kernel's KV ranges of f's chunk cover key
-// frame x, 2 if the scan puts x in f's forward state, 3 if in the backward
-// state; 255 if not exactly one of them.
+// table[f * F + x]: 1 if the softmax kernel's KV ranges of f's query segment
+// cover key frame x, 2 if the scan puts x in f's forward state, 3 if in the
+// backward state (none for a GLOBAL anchor query, whose readout is zeroed);
+// 255 if not exactly one of them.
 __global__ void k_membership(const __grid_constant__ Geom g, uint8_t* table) {
   const int total = g.F * g.F;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
     const int f = i / g.F, x = i % g.F;
     const int c = f / g.C;
+    const int glob = no_linear_read(f, g);
     KvRanges r;
-    kv_ranges(c, g, r);
+    seg_ranges(glob ? kAllFrames : c, g, r);
     const long long s0 = (long long)x * g.P, e0 = s0 + g.P;
     int soft = 0;
     for (int k = 0; k < r.n; ++k)
       if (r.start[k] <= s0 && e0 <= r.start[k] + r.len[k]) soft = 1;
-    const int has_state = x >= 1 && x <= g.F - 2;  // frames that own state parts
+    const int has_state = !glob && x >= 1 && x <= g.F - 2;  // frames that own state parts
     const int cx = x / g.C;
     const int fwd = has_state && cx <= fwd_last_chunk(c);
     const int bwd = has_state && cx >= bwd_first_chunk(c);

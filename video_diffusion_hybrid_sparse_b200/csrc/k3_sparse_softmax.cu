@@ -5,18 +5,21 @@
 //
 // Design (sm_100a):
 //  * persistent CTAs, one per SM; a work item is two 128-row query tiles of
-//    one (batch, head, chunk); items are handed out statically in an order
-//    sorted by KV tile count (longest first);
-//  * only the KV tiles of the item's chunk are enumerated: at most three
+//    one (batch, head, query segment), a segment being the rows of one chunk
+//    (under the GLOBAL anchor reading the rows of frames 0 and F-1 are
+//    segments of their own whose key set is every frame); items are handed
+//    out statically in an order sorted by KV tile count (longest first);
+//  * only the KV tiles of the item's key set are enumerated: at most three
 //    merged video token ranges plus the text range, 128 keys per tile; the
 //    last tile of a range is masked past the range end;
 //  * warp 0 issues TMA loads (Q once per item, K and V per tile, two stages);
 //    warp 1 issues tcgen05 MMAs from one thread: S_t = Q_t K^T (both operands
 //    K-major in shared memory, fp32 accumulator in TMEM) and O_t += P_t V
 //    (P_t read from TMEM, V MN-major in shared memory);
-//  * warps 4-7 and 8-11 are the softmax warpgroups of query tile 0 and 1;
-//    each thread owns one query row (TMEM lane), so row max and row sum are
-//    in-thread; P is written back as bf16 over the first half of S's columns;
+//  * warps 4-7 and 8-11 are the softmax warpgroups of query tile 0 and 1
+//    (warp w reads TMEM lanes 32*(w%4)..+31); each thread owns one query row
+//    (TMEM lane), so row max and row sum are in-thread; P is written back as
+//    bf16 over the first half of S's columns;
 //  * online softmax with a lazy rescale: the running max only moves (and O is
 //    rescaled in TMEM) when a tile's max exceeds it by more than 8 in log2
 //    units; the final 1/l is applied in the epilogue;
@@ -44,36 +47,64 @@ struct K3Layout {
   static constexpr int kBytes = kBar + 256 + 1024;  // + barriers + alignment slack
 };
 
-// One column pair in kPolyEvery takes the FMA-pipe exponential.
+// With kPolyEvery = n > 0, one column pair in n is exponentiated on the FMA
+// pipe instead of the special-function unit.  Off by default: on B200 the
+// FMA-pipe form costs more cycles per step than it saves on the MUFU (the
+// softmax warps are latency-bound, and the extra instructions lower the
+// clock under the power cap).
 #ifndef VDN_POLY_EVERY
-#define VDN_POLY_EVERY 8
+#define VDN_POLY_EVERY 0
 #endif
 constexpr int kPolyEvery = VDN_POLY_EVERY;
+__host__ __device__ constexpr bool poly_pair(int e) {
+  return kPolyEvery > 0 && (e % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
+}
+
+// P of one tile can be handed to the MMA warp in kPParts column groups, so that
+// the P·V products of the first keys run while the later keys are
+// exponentiated.  One group is fastest on B200 (2 and 4 add MMA-warp waits
+// that cost more than the overlap gains).
+#ifndef VDN_P_PARTS
+#define VDN_P_PARTS 1
+#endif
+constexpr int kPParts = VDN_P_PARTS;
+static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P parts");
 
 struct Item {
-  int b, h, c, pair, ntiles, row0;  // row0: first query row of the item within the batch
+  int b, h, c, pair, ntiles;
+  int row0;   // first query row of the item within the batch
+  int nrows;  // rows of the item's query segment from row0 on (the tiles mask rows past it)
 };
 
 __device__ __forceinline__ Item decode_item(int item, const K3Params& p) {
   const Geom& g = p.g;
+  // segment k with seg_item0[k] <= item < seg_item0[k + 1]
+  int lo = 0, hi = p.n_segs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.seg_item0[mid] <= item) lo = mid;
+    else hi = mid - 1;
+  }
+  const QSeg sg = p.segs[lo];
+  const int n_pairs = (sg.nrows + 2 * kBlockM - 1) / (2 * kBlockM);
   Item it;
-  const int pos = item / p.items_per_chunk;
-  int rem = item - pos * p.items_per_chunk;
-  it.c = p.chunk_order[pos];
-  const int per_b = g.H * g.n_pairs;
+  int rem = item - p.seg_item0[lo];
+  const int per_b = g.H * n_pairs;
   it.b = rem / per_b;
   rem -= it.b * per_b;
-  it.h = rem / g.n_pairs;
-  it.pair = rem - it.h * g.n_pairs;
-  it.row0 = it.c * g.rows_per_chunk + it.pair * 2 * kBlockM;
-  it.ntiles = (it.pair * 2 * kBlockM + kBlockM < g.rows_per_chunk) ? 2 : 1;
+  it.h = rem / n_pairs;
+  it.pair = rem - it.h * n_pairs;
+  it.c = sg.c;
+  it.row0 = sg.row0 + it.pair * 2 * kBlockM;
+  it.nrows = sg.nrows - it.pair * 2 * kBlockM;
+  it.ntiles = it.nrows > kBlockM ? 2 : 1;
   return it;
 }
 
 // Barrier slots.
 enum {
   kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = 4, kVFull = 6, kVEmpty = 8,
-  kSFull = 10, kPFull = 12, kOFull = 14, kDone = 16, kNumBars = 17
+  kSFull = 10, kPFull = 12, kOFull = 12 + 2 * kPParts, kDone = kOFull + 2, kNumBars = kDone + 1
 };
 
 }  // namespace
@@ -105,7 +136,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars[kSFull + t], 1);
-      mbar_init(&bars[kPFull + t], kBlockM);
+      for (int part = 0; part < kPParts; ++part) mbar_init(&bars[kPFull + 2 * part + t], kBlockM);
       mbar_init(&bars[kOFull + t], 1);
     }
     mbar_init(&bars[kDone], 1);
@@ -140,7 +171,7 @@ __global__ void __launch_bounds__(384, 1)
             tma_load_2d(sQ + t * L::kTile + bx * 16384, &tm_q, &bars[kQFull], it.h * D + bx * 64,
                         it.b * (int)g.N + it.row0 + t * kBlockM);
         KvRanges kr;
-        kv_ranges(it.c, g, kr);
+        seg_ranges(it.c, g, kr);
         for (int ri = 0; ri <= kr.n && ok; ++ri) {
           const bool text = (ri == kr.n);
           const int len = text ? g.T : (int)kr.len[ri];
@@ -192,18 +223,22 @@ __global__ void __launch_bounds__(384, 1)
           mma_ss(d_tmem, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, int st, bool acc) {
+      // O_t += P_t·V over the keys of P part `part`
+      auto issue_pv = [&](int t, int st, int part, bool acc) {
         const uint32_t d_tmem = tmem + 256 + t * D;
         const uint64_t vd = v_desc0 + (uint64_t)((st * L::kTile) >> 4);
+        constexpr int kPer = kBlockN / 16 / kPParts;
 #pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk)
+        for (int k = 0; k < kPer; ++k) {
+          const int kk = part * kPer + k;
           mma_ts(d_tmem, tmem + t * 128 + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
                  (acc || kk > 0) ? 1u : 0u);
+        }
       };
 
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++item_cnt) {
         const Item it = decode_item(item, p);
-        const int nkv = kv_tiles(it.c, g);
+        const int nkv = seg_kv_tiles(it.c, g);
         if (!mbar_wait(&bars[kQFull], item_cnt & 1, ab)) { ok = false; break; }
         {
           const int st = kv_cnt % L::kStages;
@@ -221,10 +256,13 @@ __global__ void __launch_bounds__(384, 1)
           const bool has_next = j + 1 < nkv;
           if (!mbar_wait(&bars[kVFull + st], (kv_cnt / L::kStages) & 1, ab)) { ok = false; break; }
           for (int t = 0; t < it.ntiles; ++t) {
-            if (!mbar_wait(&bars[kPFull + t], p_cnt[t] & 1, ab)) { ok = false; break; }
+            for (int part = 0; part < kPParts; ++part) {
+              if (!mbar_wait(&bars[kPFull + 2 * part + t], p_cnt[t] & 1, ab)) { ok = false; break; }
+              tc_fence_after();
+              issue_pv(t, st, part, j > 0);
+            }
+            if (!ok) break;
             ++p_cnt[t];
-            tc_fence_after();
-            issue_pv(t, st, j > 0);
             if (!has_next) mma_commit(&bars[kOFull + t]);
             if (has_next) {
               if (t == 0 && !mbar_wait(&bars[kKFull + nst], ((kv_cnt + 1) / L::kStages) & 1, ab)) {
@@ -257,19 +295,27 @@ __global__ void __launch_bounds__(384, 1)
     uint32_t s_cnt = 0, o_cnt = 0;
 
     for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
-      const Item it = decode_item(item, p);
-      if (t >= it.ntiles) continue;
-      const int tile_row0 = it.pair * 2 * kBlockM + t * kBlockM;  // within the chunk
-      const int nrows = min(kBlockM, g.rows_per_chunk - tile_row0);
+      // only the key set and the tile count live across the KV loop; the
+      // epilogue decodes the item again (fewer registers held in the loop)
+      int seg_c, ntiles;
+      {
+        const Item it = decode_item(item, p);
+        seg_c = it.c;
+        ntiles = it.ntiles;
+      }
+      if (t >= ntiles) continue;
       float m_run = 0.f, l_run = 0.f;
-      KvRanges kr;
-      kv_ranges(it.c, g, kr);
       bool ok = true;
-      int j = 0;
-      for (int ri = 0; ri <= kr.n && ok; ++ri) {
-        const int len = (ri == kr.n) ? g.T : (int)kr.len[ri];
-        for (int off = 0; off < len; off += kBlockN, ++j) {
-          const int n_valid = min(kBlockN, len - off);
+      // keys left in the current key range (video ranges, then text); only
+      // these scalars live across the loop, the ranges are re-derived at
+      // range ends
+      const int nkv = seg_kv_tiles(seg_c, g);
+      int range = 0, left = seg_range_len(seg_c, g, 0);
+      {
+        for (int j = 0; j < nkv; ++j) {
+          while (left == 0) left = seg_range_len(seg_c, g, ++range);
+          const int n_valid = min(kBlockN, left);
+          left -= n_valid;
           const bool got = mbar_wait(&bars[kSFull + t], s_cnt & 1, ab);
           if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
           ++s_cnt;
@@ -313,21 +359,22 @@ __global__ void __launch_bounds__(384, 1)
           }
           l_run *= alpha;
           // p = 2^(s * scale * log2(e) - m): the exponent argument and the
-          // row sum in packed f32x2; every kPolyEvery-th column pair is
-          // exponentiated on the FMA pipe, the rest on the special-function unit.
+          // row sum in packed f32x2; P goes to TMEM 8 columns (16 keys) at a
+          // time, which keeps the live registers under the 168 of a 384-thread
+          // CTA (no spills).
           const uint64_t sl2x2 = f32x2_pack(sl2, sl2);
           const uint64_t negm = f32x2_pack(-m_run, -m_run);
           uint64_t lsum0 = f32x2_pack(0.f, 0.f), lsum1 = lsum0;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t pk[16];
+          for (int i = 0; i < 8; ++i) {
+            uint32_t pk[8];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const uint64_t sx = f32x2_pack(__uint_as_float(s[32 * i + 2 * e]), __uint_as_float(s[32 * i + 2 * e + 1]));
+            for (int e = 0; e < 8; ++e) {
+              const uint64_t sx = f32x2_pack(__uint_as_float(s[16 * i + 2 * e]), __uint_as_float(s[16 * i + 2 * e + 1]));
               float x0, x1;
               f32x2_unpack(f32x2_fma(sx, sl2x2, negm), x0, x1);
               float p0, p1;
-              if ((e % kPolyEvery) == kPolyEvery - 1) {
+              if (poly_pair(e)) {
                 p0 = exp2_fma(x0);
                 p1 = exp2_fma(x1);
               } else {
@@ -338,7 +385,27 @@ __global__ void __launch_bounds__(384, 1)
               else lsum0 = f32x2_add(lsum0, f32x2_pack(p0, p1));
               pk[e] = pack_bf16x2(p0, p1);
             }
-            tmem_st16(tmem_addr(tmem, lane_base, t * 128 + 16 * i), pk);
+            tmem_st8(tmem_addr(tmem, lane_base, t * 128 + 8 * i), pk);
+            if ((i + 1) % (8 / kPParts) == 0) {
+              const int part = (i + 1) / (8 / kPParts) - 1;
+              if (part == 0 && rescale) {
+                // O_t is quiescent here: S_t(j) completing implies PV_t(j-1)
+                // completed, and PV_t(j) starts only after this part arrives.
+#pragma unroll 1
+                for (int c = 0; c < D / 16; ++c) {
+                  uint32_t o[16];
+                  const uint32_t ta = tmem_addr(tmem, lane_base, 256 + t * D + 16 * c);
+                  tmem_ld16(ta, o);
+                  tmem_wait_ld();
+#pragma unroll
+                  for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                  tmem_st16(ta, o);
+                }
+              }
+              tmem_wait_st();
+              tc_fence_before();
+              mbar_arrive(&bars[kPFull + 2 * part + t]);
+            }
           }
           {
             float l0, l1, l2, l3;
@@ -346,22 +413,6 @@ __global__ void __launch_bounds__(384, 1)
             f32x2_unpack(lsum1, l2, l3);
             l_run += (l0 + l1) + (l2 + l3);
           }
-          if (rescale) {
-            // O_t is quiescent here: S_t(j) completing implies PV_t(j-1) completed
-#pragma unroll 1
-            for (int i = 0; i < D / 32; ++i) {
-              uint32_t o[32];
-              const uint32_t ta = tmem_addr(tmem, lane_base, 256 + t * D + 32 * i);
-              tmem_ld32(ta, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32(ta, o);
-            }
-          }
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(&bars[kPFull + t]);
         }
       }
       if (!ok) break;
@@ -371,7 +422,9 @@ __global__ void __launch_bounds__(384, 1)
       ++o_cnt;
       tc_fence_after();
       const float inv_l = 1.0f / l_run;
-      __nv_bfloat16* dst = p.o_s + (((size_t)it.b * g.N + (size_t)(it.c * g.rows_per_chunk + tile_row0 + row)) * g.H + it.h) * D;
+      const Item it = decode_item(item, p);
+      const int nrows = min(kBlockM, it.nrows - t * kBlockM);  // valid rows of this tile
+      __nv_bfloat16* dst = p.o_s + (((size_t)it.b * g.N + (size_t)(it.row0 + t * kBlockM + row)) * g.H + it.h) * D;
 #pragma unroll
       for (int i = 0; i < D / 32; ++i) {
         uint32_t o[32];
@@ -419,3 +472,4 @@ cudaError_t launch_sparse_softmax(const Maps& m, const K3Params& p, int grid, cu
 }
 
 }  // namespace vdn
+

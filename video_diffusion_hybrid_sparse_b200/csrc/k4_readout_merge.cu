@@ -22,7 +22,9 @@
 //     o_l = num / den (0 when the chunk's states hold no token) and the
 //     row's RMS, stage r = o_l / sqrt(mean(o_l^2) + eps) in shared memory, and
 //     a coalesced pass reads o_s and both gates (prefetched into L2 one tile
-//     ahead), applies gamma and writes out = sigmoid(g_s) o_s + sigmoid(g_l) r.
+//     ahead), applies gamma and writes out = sigmoid(g_s) o_s + sigmoid(g_l) r
+//     (SPLIT: the two terms to out and out_linear).  Rows of a GLOBAL anchor
+//     query read nothing through the states (o_l = 0).
 // Every wait is bounded; the worker warps agree on giving up through a
 // barrier with an OR reduction, so none is left waiting for another.
 #include "kernels.h"
@@ -234,6 +236,7 @@ __global__ void __launch_bounds__(kK4Threads, 1)
     // output: 0 merged, 1 softmax branch only, 2 linear read (normalised or raw)
     const int mode = (p.flags & 1) ? 1 : ((p.flags & 6) ? 2 : 0);
     const bool use_gamma = p.gamma != nullptr && !(p.flags & 4);
+    const bool split = p.out_linear != nullptr;  // out gets sigmoid(g_s) o_s, out_linear sigmoid(g_l) r
 
     // Finish tile `item` (slot s): TMEM -> r -> coalesced merge.  Returns false on a timeout.
     auto finish = [&](int item, int s) -> bool {
@@ -256,7 +259,9 @@ __global__ void __launch_bounds__(kK4Threads, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&bars[kAccEmpty + s]);  // the accumulator may be overwritten now
-      const bool empty = state_tokens(it.c, g) == 0;
+      // zero read: the chunk's states hold no token, or the row is a GLOBAL anchor query
+      const int qrow = it.c * g.rows_per_chunk + it.tile * 128 + row;
+      const bool empty = state_tokens(it.c, g) == 0 || no_linear_read(qrow / g.P, g);
       const float inv_den = empty ? 0.f : 1.0f / __uint_as_float(dr);
       float ss = 0.f;
 #pragma unroll
@@ -339,12 +344,23 @@ __global__ void __launch_bounds__(kK4Threads, 1)
             }
           }
           float o[8];
+          const size_t oidx = (tok[u] * g.H + it.h) * d + c8v[u] * 8;
+          if (split) {
+            float ol[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const float merged = sigmoid_f(gs[k]) * os[k] + sigmoid_f(gl[k]) * r[k];
-            o[k] = mode == 0 ? merged : (mode == 1 ? os[k] : r[k]);
+            for (int k = 0; k < 8; ++k) {
+              o[k] = sigmoid_f(gs[k]) * os[k];
+              ol[k] = sigmoid_f(gl[k]) * r[k];
+            }
+            if (valid[u]) store8<FP32>(p.out_linear, oidx, ol);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const float merged = sigmoid_f(gs[k]) * os[k] + sigmoid_f(gl[k]) * r[k];
+              o[k] = mode == 0 ? merged : (mode == 1 ? os[k] : r[k]);
+            }
           }
-          if (valid[u]) store8<FP32>(p.out, (tok[u] * g.H + it.h) * d + c8v[u] * 8, o);
+          if (valid[u]) store8<FP32>(p.out, oidx, o);
         }
       }
       workers_any(false);  // r staging is rewritten by the next tile

@@ -14,9 +14,12 @@ struct K3Params {
   float scale_log2;        // softmax scale * log2(e)
   __nv_bfloat16* o_s;      // [B, N, H, Dp] bf16
   int* status;
-  int n_items;             // Nc * B * H * n_pairs
-  int items_per_chunk;     // B * H * n_pairs
-  int chunk_order[kMaxChunks];  // chunks by decreasing KV tile count
+  int n_items;             // sum over segments of B * H * pairs
+  int n_segs;
+  // query segments by decreasing KV tile count; items of segment k are
+  // [seg_item0[k], seg_item0[k + 1]), ordered (batch, head, pair)
+  QSeg segs[kMaxSegs];
+  int seg_item0[kMaxSegs + 1];
 };
 
 struct K1Params {
@@ -41,6 +44,7 @@ struct K4Params {
   const void* gate_s;
   const void* gate_l;
   void* out;
+  void* out_linear;        // SPLIT output: sigmoid(g_l) * r goes here, out gets sigmoid(g_s) * o_s
   int flags;
   int* status;
 };

@@ -79,6 +79,8 @@ extern "C" VDN_API vdn_status vdn_hybrid_attn_fwd_static(const void* q, const vo
   if (cfg->text_tokens > 0)
     for (const void* p : {text_k, text_v})
       if (bad_ptr(p)) return p ? VDN_ERR_ALIGNMENT : VDN_ERR_INVALID_ARG;
+  if (cfg->output_mode == VDN_OUTPUT_SPLIT && bad_ptr(cfg->out_linear))
+    return cfg->out_linear ? VDN_ERR_ALIGNMENT : VDN_ERR_INVALID_ARG;
   if ((cfg->debug_flags & VDN_EXPORT_STATES) && (!cfg->export_fwd || !cfg->export_bwd)) return VDN_ERR_INVALID_ARG;
   void* scratch = nullptr;
   const vdn_status s = scratch_address(&scratch);

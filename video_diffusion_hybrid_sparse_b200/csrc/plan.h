@@ -9,7 +9,10 @@
 //     text; an anchor already inside the window is read once;
 //   * the forward state of chunk c holds chunks 0 .. c-2, the backward state
 //     chunks c+2 .. Nc-1, both without the anchor frames;
-//   * each state also holds half of the text state.
+//   * each state also holds half of the text state;
+//   * anchor frames as queries follow the same rule (LOCAL), or, under the
+//     GLOBAL reading of "the first and last frames interact with all frames",
+//     attend by softmax to every frame and read nothing through the states.
 #pragma once
 
 #include <cstddef>
@@ -27,6 +30,7 @@ constexpr int kMaxChunks = 256;     // chunk-order table carried in kernel param
 constexpr int kSliceTokens = 2048;  // tokens per state-build work item
 constexpr int kBlockM = 128;        // query rows per tile
 constexpr int kBlockN = 128;        // keys per tile
+constexpr int kMaxSegs = kMaxChunks + 2;  // query segments (chunks, plus the anchor frames under GLOBAL)
 
 struct Geom {
   int B, F, P, H, d, T, C;  // batch, frames, tokens/frame, heads, head_dim, text tokens, chunk frames
@@ -42,6 +46,7 @@ struct Geom {
   int rows_per_chunk;       // C * P query rows
   int n_pairs;              // work items of two 128-row query tiles per chunk
   int mt_rows;              // rows of one readout B-tile: Dp + 16 (values, z, zero padding)
+  int anchor_global;        // 1: anchor query frames attend to every frame, no linear read
   float scale;              // softmax scale
   float eps;                // RMSNorm epsilon
   // workspace layout (byte offsets; each 1024-aligned)
@@ -105,6 +110,64 @@ VDN_HD int kv_tiles(int c, const Geom& g) {
   int n = 0;
   for (int i = 0; i < r.n; ++i) n += ceil_div(r.len[i], kBlockN);
   return n + ceil_div(g.T, kBlockN);
+}
+
+// A query segment: rows [row0, row0 + nrows) of one batch that read the same
+// key set through the softmax branch: the window of chunk c (c >= 0) or every
+// video frame (c = kAllFrames).
+constexpr int kAllFrames = -1;
+struct QSeg {
+  int row0, nrows, c;
+};
+
+// Video key ranges of a segment's key set.
+VDN_HD void seg_ranges(int c, const Geom& g, KvRanges& r) {
+  if (c == kAllFrames) {
+    r.n = 1;
+    r.start[0] = 0;
+    r.len[0] = g.N;
+    return;
+  }
+  kv_ranges(c, g, r);
+}
+
+// Keys in range r of a segment's key set (video ranges in order, then the
+// text as the last range); 0 past the end.
+VDN_HD int seg_range_len(int c, const Geom& g, int r) {
+  KvRanges kr;
+  seg_ranges(c, g, kr);
+  for (int i = 0; i < 3; ++i)
+    if (i < kr.n && i == r) return (int)kr.len[i];
+  return r == kr.n ? g.T : 0;
+}
+
+VDN_HD int seg_kv_tiles(int c, const Geom& g) {
+  KvRanges r;
+  seg_ranges(c, g, r);
+  int n = 0;
+  for (int i = 0; i < r.n; ++i) n += ceil_div(r.len[i], kBlockN);
+  return n + ceil_div(g.T, kBlockN);
+}
+
+// Query frame f reads nothing through the states (GLOBAL anchor).
+VDN_HD int no_linear_read(int f, const Geom& g) { return g.anchor_global && is_anchor(f, g.F); }
+
+// The query segments in row order; returns their number (<= Nc + 2).
+inline int query_segments(const Geom& g, QSeg* out) {
+  int n = 0;
+  for (int c = 0; c < g.Nc; ++c) {
+    int lo = c * g.C, hi = (c + 1) * g.C;  // frames [lo, hi)
+    if (!g.anchor_global) {
+      out[n++] = QSeg{lo * g.P, (hi - lo) * g.P, c};
+      continue;
+    }
+    if (lo == 0) { out[n++] = QSeg{0, g.P, kAllFrames}; lo = 1; }
+    const bool last_here = hi == g.F && g.F - 1 >= lo;
+    if (last_here) hi = g.F - 1;
+    if (hi > lo) out[n++] = QSeg{lo * g.P, (hi - lo) * g.P, c};
+    if (last_here) out[n++] = QSeg{(g.F - 1) * g.P, g.P, kAllFrames};
+  }
+  return n;
 }
 
 // Last chunk summed by the forward state of chunk c, first chunk summed by
