@@ -197,6 +197,29 @@ VDN_API vdn_status vdn_hybrid_attn_fwd_static(const void* q, const void* k, cons
 /* Size in bytes of the static scratch used by vdn_hybrid_attn_fwd_static. */
 VDN_API size_t vdn_static_scratch_bytes(void);
 
+/* The whole call on HOST tensors (same layouts and dtype as vdn_hybrid_attn_fwd;
+ * out, and cfg->out_linear under VDN_OUTPUT_SPLIT, are HOST pointers too).
+ * Not part of the method: an interface for callers whose tensors live in host
+ * memory.  The inputs are copied into `staging`, a caller-owned DEVICE buffer
+ * of at least vdn_host_staging_bytes(cfg) bytes (256-byte aligned), on a
+ * library-owned copy stream in the order the kernels need them (text, k, v,
+ * then q, then the gates), so the state build runs while q is in flight and
+ * the softmax branch while the gates are; the output is copied back on
+ * `stream`.  cfg->workspace is used as in vdn_hybrid_attn_fwd; the export
+ * buffers, if any, are device memory.  Host buffers should be page-locked
+ * (cudaHostAlloc / cudaHostRegister): from pageable memory the copies do
+ * not overlap.  The call returns once everything is enqueued; the caller
+ * synchronises `stream` before reading out and must keep the host and device
+ * buffers alive until then.  Errors: as vdn_hybrid_attn_fwd, plus
+ * VDN_ERR_WORKSPACE for a missing or small staging buffer and
+ * VDN_ERR_ALIGNMENT for a misaligned one. */
+VDN_API size_t vdn_host_staging_bytes(const vdn_cfg* cfg);
+VDN_API vdn_status vdn_hybrid_attn_fwd_host(const void* q, const void* k, const void* v,
+                                            const void* text_k, const void* text_v,
+                                            const void* gate_s, const void* gate_l, void* out,
+                                            void* staging, size_t staging_bytes,
+                                            const vdn_cfg* cfg, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -146,6 +146,35 @@ def test_call_errors_before_any_launch():
     assert lib.vdn_hybrid_attn_fwd(*args, ctypes.byref(cfg), None) == 3
 
 
+def test_host_call_errors_before_any_copy():
+    """vdn_hybrid_attn_fwd_host: argument and staging checks come first."""
+    lib = vb.library()
+    s = shape()
+    cfg = vb.make_cfg(s)
+    n = lib.vdn_host_staging_bytes(ctypes.byref(cfg))
+    e = 2  # bf16
+    vid, txt = s.B * s.N * s.H * s.d * e, s.B * s.T * s.H * s.d * e
+    assert n >= 6 * vid + 2 * txt
+    split = vb.make_cfg(s)
+    split.output_mode = vb.OUTPUT_SPLIT
+    assert lib.vdn_host_staging_bytes(ctypes.byref(split)) >= n + vid
+    assert lib.vdn_host_staging_bytes(ctypes.byref(vb.make_cfg(shape(F=16, C=5)))) == 0
+    p = 1 << 20
+    args = [p] * 8
+    cfg.workspace, cfg.workspace_bytes = p, vb.workspace_bytes(s)
+    assert lib.vdn_hybrid_attn_fwd_host(*args, None, n, ctypes.byref(cfg), None) == 4      # no staging
+    assert lib.vdn_hybrid_attn_fwd_host(*args, p, n - 1, ctypes.byref(cfg), None) == 4     # too small
+    assert lib.vdn_hybrid_attn_fwd_host(*args, p + 16, n, ctypes.byref(cfg), None) == 3    # misaligned
+    bad = list(args)
+    bad[0] = None
+    assert lib.vdn_hybrid_attn_fwd_host(*bad, p, n, ctypes.byref(cfg), None) == 1
+    cfg.output_mode = vb.OUTPUT_SPLIT  # no host out_linear
+    assert lib.vdn_hybrid_attn_fwd_host(*args, p, n, ctypes.byref(cfg), None) == 1
+    cfg.output_mode = 0
+    cfg.workspace = None
+    assert lib.vdn_hybrid_attn_fwd_host(*args, p, n, ctypes.byref(cfg), None) == 4
+
+
 EDGE = [(1, 1), (2, 1), (2, 2), (3, 1), (3, 3), (4, 2), (5, 1), (6, 3), (15, 1), (15, 5), (45, 5), (60, 5),
         (60, 1), (10, 10), (96, 1)]
 

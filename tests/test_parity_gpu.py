@@ -157,6 +157,26 @@ def test_split_output_matches_oracle(w):
     assert_close((out.float() + out_lin.float()).cpu().numpy(), merged.cpu().numpy(), f"{w.name} split sum")
 
 
+@pytest.mark.parametrize("w,mode,split", [(SMALL[0], 0, False), (SMALL[1], 0, False), (SMALL[3], 1, False),
+                                          (SMALL[2], 0, True)], ids=["tiny", "small", "c5_global", "ragged_split"])
+def test_host_tensor_call_equals_device_call(w, mode, split):
+    """vdn_hybrid_attn_fwd_host (pinned host tensors, copies overlapped with
+    the kernels) gives the device call's output bit for bit."""
+    inputs = make_inputs(w)
+    dev = to_dev(inputs)
+    ref_lin = torch.empty_like(dev["q"]) if split else None
+    ref = run(w, dev, anchor_query_mode=mode, out_linear=ref_lin)
+    host = {k: t.pin_memory() for k, t in inputs.items()}
+    out_lin = torch.empty(host["q"].shape, dtype=host["q"].dtype, pin_memory=True) if split else None
+    out = vb.hybrid_attn_fwd_host(host["q"], host["k"], host["v"], host["text_k"], host["text_v"], host["gate_s"],
+                                  host["gate_l"], frames=w.F, chunk_frames=w.C, anchor_query_mode=mode,
+                                  out_linear=out_lin)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref.cpu())
+    if split:
+        assert torch.equal(out_lin, ref_lin.cpu())
+
+
 @pytest.mark.parametrize("w", [SMALL[0], SMALL[2], SMALL[3]], ids=["tiny", "ragged", "c5_ragged"])
 def test_exported_states_match_oracle(w):
     inputs = make_inputs(w)

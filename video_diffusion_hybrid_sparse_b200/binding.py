@@ -25,7 +25,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "po
 EXPORTED = ["vdn_version", "vdn_status_string", "vdn_validate", "vdn_workspace_bytes", "vdn_plan_membership",
             "vdn_membership_device", "vdn_hybrid_attn_fwd", "vdn_stage_inputs", "vdn_state_build",
             "vdn_state_scan", "vdn_sparse_softmax", "vdn_readout_merge", "vdn_hybrid_attn_fwd_static",
-            "vdn_static_scratch_bytes"]
+            "vdn_static_scratch_bytes", "vdn_host_staging_bytes", "vdn_hybrid_attn_fwd_host"]
 
 
 class VdnError(RuntimeError):
@@ -76,8 +76,12 @@ def library() -> ctypes.CDLL:
         lib.vdn_readout_merge.argtypes = [P, P, P, P, C, P]
         lib.vdn_hybrid_attn_fwd_static.argtypes = [P, P, P, P, P, P, P, P, C, P]
         lib.vdn_static_scratch_bytes.restype = ctypes.c_size_t
+        lib.vdn_host_staging_bytes.restype = ctypes.c_size_t
+        lib.vdn_host_staging_bytes.argtypes = [C]
+        lib.vdn_hybrid_attn_fwd_host.argtypes = [P, P, P, P, P, P, P, P, P, ctypes.c_size_t, C, P]
         for name in EXPORTED:
-            if name not in ("vdn_version", "vdn_status_string", "vdn_workspace_bytes", "vdn_static_scratch_bytes"):
+            if name not in ("vdn_version", "vdn_status_string", "vdn_workspace_bytes", "vdn_static_scratch_bytes",
+                            "vdn_host_staging_bytes"):
                 getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -193,6 +197,51 @@ def hybrid_attn_fwd(q, k, v, text_k, text_v, gate_s, gate_l, *, frames: int, chu
                                          gate_s.data_ptr(), gate_l.data_ptr(), out.data_ptr(),
                                          ctypes.byref(cfg), _stream(stream))
     _check(code, "vdn_hybrid_attn_fwd")
+    return out
+
+
+_STAGING: dict = {}
+
+
+def staging_for(s: Shape, device, split: bool = False) -> torch.Tensor:
+    """A cached device staging buffer for :func:`hybrid_attn_fwd_host`."""
+    cfg = make_cfg(s)
+    if split:
+        cfg.output_mode = OUTPUT_SPLIT
+    n = library().vdn_host_staging_bytes(ctypes.byref(cfg))
+    if n == 0:
+        _check(library().vdn_validate(ctypes.byref(cfg)), "vdn_host_staging_bytes")
+    dev = torch.device(device)
+    key = (dev.index if dev.index is not None else torch.cuda.current_device())
+    buf = _STAGING.get(key)
+    if buf is None or buf.numel() < n:
+        buf = torch.empty(n, dtype=torch.uint8, device=dev)
+        _STAGING[key] = buf
+    return buf
+
+
+def hybrid_attn_fwd_host(q, k, v, text_k, text_v, gate_s, gate_l, *, frames: int, chunk_frames: int, out=None,
+                         softmax_scale: float = 0.0, rms_eps: float = -1.0, rms_weight=None, workspace=None,
+                         staging=None, stream=None, anchor_query_mode: int = ANCHOR_LOCAL,
+                         out_linear=None, device="cuda") -> torch.Tensor:
+    """The whole call on HOST tensors (contiguous CPU tensors, ideally pinned),
+    copies overlapped with the kernels inside the library.  Returns the host
+    ``out``; synchronise ``stream`` (default: the current stream of
+    ``device``) before reading it."""
+    s = shape_of(q, text_k, frames, chunk_frames)
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=q.is_pinned())
+    if workspace is None:
+        workspace = workspace_for(s, device)
+    if staging is None:
+        staging = staging_for(s, device, out_linear is not None)
+    cfg = make_cfg(s, softmax_scale=softmax_scale, rms_eps=rms_eps, rms_weight=rms_weight, workspace=workspace,
+                   anchor_query_mode=anchor_query_mode, out_linear=out_linear)
+    code = library().vdn_hybrid_attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(text_k), _ptr(text_v),
+                                              gate_s.data_ptr(), gate_l.data_ptr(), out.data_ptr(),
+                                              staging.data_ptr(), staging.numel(), ctypes.byref(cfg),
+                                              _stream(stream))
+    _check(code, "vdn_hybrid_attn_fwd_host")
     return out
 
 

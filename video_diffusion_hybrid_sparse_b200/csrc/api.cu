@@ -265,6 +265,49 @@ vdn_status check_inputs(const vdn_cfg* cfg, const Geom& g, std::initializer_list
   return s;
 }
 
+// ---------------------------------------------------------------- calls on host tensors
+
+// Device staging of vdn_hybrid_attn_fwd_host: the caller's tensors in their
+// own dtype and layout, 256-byte aligned slots.
+struct HostStaging {
+  size_t q, k, v, tk, tv, gs, gl, out, out_lin, total;
+};
+
+HostStaging host_staging(const vdn_cfg* cfg, const Geom& g) {
+  const size_t e = g.fp32_io ? 4 : 2;
+  const size_t vid = (size_t)g.B * g.N * g.H * g.d * e, txt = (size_t)g.B * g.T * g.H * g.d * e;
+  HostStaging h;
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    const size_t o = off;
+    off = align_up(off + n, 256);
+    return o;
+  };
+  h.q = take(vid);
+  h.k = take(vid);
+  h.v = take(vid);
+  h.tk = take(txt);
+  h.tv = take(txt);
+  h.gs = take(vid);
+  h.gl = take(vid);
+  h.out = take(vid);
+  h.out_lin = cfg->output_mode == VDN_OUTPUT_SPLIT ? take(vid) : h.out;
+  h.total = off;
+  return h;
+}
+
+// One non-blocking copy stream per device, created on first use.
+cudaStream_t copy_stream() {
+  static std::mutex mu;
+  static cudaStream_t streams[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
+    streams[dev] = nullptr;
+  return streams[dev];
+}
+
 }  // namespace
 }  // namespace vdn
 
@@ -393,6 +436,85 @@ vdn_status vdn_hybrid_attn_fwd(const void* q, const void* k, const void* v, cons
   if ((s = step_state_scan(cfg, g, st)) != VDN_OK) return s;
   if ((s = step_sparse_softmax(cfg, g, src, st)) != VDN_OK) return s;
   return step_readout_merge(cfg, g, src, gate_s, gate_l, out, st);
+}
+
+size_t vdn_host_staging_bytes(const vdn_cfg* cfg) {
+  Geom g;
+  return make_geom(cfg, g) == VDN_OK ? host_staging(cfg, g).total : 0;
+}
+
+vdn_status vdn_hybrid_attn_fwd_host(const void* q, const void* k, const void* v, const void* text_k,
+                                    const void* text_v, const void* gate_s, const void* gate_l, void* out,
+                                    void* staging, size_t staging_bytes, const vdn_cfg* cfg, void* stream) {
+  Geom g;
+  vdn_status s = make_geom(cfg, g);
+  if (s != VDN_OK) return s;
+  for (const void* p : {q, k, v, gate_s, gate_l, static_cast<const void*>(out)})
+    if (!p) return VDN_ERR_INVALID_ARG;
+  if (g.T > 0 && (!text_k || !text_v)) return VDN_ERR_INVALID_ARG;
+  if (cfg->output_mode == VDN_OUTPUT_SPLIT && !cfg->out_linear) return VDN_ERR_INVALID_ARG;
+  if ((cfg->debug_flags & VDN_EXPORT_STATES) && (!cfg->export_fwd || !cfg->export_bwd)) return VDN_ERR_INVALID_ARG;
+  if ((s = check_ws(cfg, g)) != VDN_OK) return s;
+  const HostStaging h = host_staging(cfg, g);
+  if (!staging || staging_bytes < h.total) return VDN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(staging) & 255u) != 0) return VDN_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaStream_t cs = copy_stream();
+  if (!cs) return VDN_ERR_CUDA;
+  uint8_t* dv = static_cast<uint8_t*>(staging);
+  const size_t e = g.fp32_io ? 4 : 2;
+  const size_t vid = (size_t)g.B * g.N * g.H * g.d * e, txt = (size_t)g.B * g.T * g.H * g.d * e;
+  cudaEvent_t ev[4] = {};  // start, k/v/text landed, q landed, gates landed
+  for (auto& x : ev)
+    if (cudaEventCreateWithFlags(&x, cudaEventDisableTiming) != cudaSuccess) x = nullptr;
+  auto finish = [&](vdn_status r) {
+    for (auto& x : ev)
+      if (x) cudaEventDestroy(x);  // released once the GPU has passed them
+    return r;
+  };
+  if (!ev[0] || !ev[1] || !ev[2] || !ev[3]) return finish(VDN_ERR_CUDA);
+  auto h2d = [&](size_t off, const void* src, size_t n) {
+    return n == 0 ? cudaSuccess : cudaMemcpyAsync(dv + off, src, n, cudaMemcpyHostToDevice, cs);
+  };
+  // Copies on the copy stream, in the order the kernels need them, so the
+  // state build runs while q lands and the softmax branch while the gates land.
+  cudaError_t ce = cudaEventRecord(ev[0], st);  // earlier work on st may still read the staging
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(cs, ev[0], 0);
+  if (ce == cudaSuccess && g.T > 0) ce = h2d(h.tk, text_k, txt);
+  if (ce == cudaSuccess && g.T > 0) ce = h2d(h.tv, text_v, txt);
+  if (ce == cudaSuccess) ce = h2d(h.k, k, vid);
+  if (ce == cudaSuccess) ce = h2d(h.v, v, vid);
+  if (ce == cudaSuccess) ce = cudaEventRecord(ev[1], cs);
+  if (ce == cudaSuccess) ce = h2d(h.q, q, vid);
+  if (ce == cudaSuccess) ce = cudaEventRecord(ev[2], cs);
+  if (ce == cudaSuccess) ce = h2d(h.gs, gate_s, vid);
+  if (ce == cudaSuccess) ce = h2d(h.gl, gate_l, vid);
+  if (ce == cudaSuccess) ce = cudaEventRecord(ev[3], cs);
+  if (ce != cudaSuccess) return finish(VDN_ERR_CUDA);
+
+  vdn_cfg c = *cfg;
+  if (c.output_mode == VDN_OUTPUT_SPLIT) c.out_linear = dv + h.out_lin;
+  const void* dq = dv + h.q;
+  const void* dk = dv + h.k;
+  const void* dvv = dv + h.v;
+  const void* dtk = g.T > 0 ? dv + h.tk : nullptr;
+  const void* dtv = g.T > 0 ? dv + h.tv : nullptr;
+  const Srcs src = kernel_srcs(&c, g, dq, dk, dvv, dtk, dtv);
+  if (cudaStreamWaitEvent(st, ev[1], 0) != cudaSuccess) return finish(VDN_ERR_CUDA);
+  if (g.staged) {  // staging converts q as well
+    if (cudaStreamWaitEvent(st, ev[2], 0) != cudaSuccess) return finish(VDN_ERR_CUDA);
+    if ((s = step_stage(&c, g, dq, dk, dvv, dtk, dtv, st)) != VDN_OK) return finish(s);
+  }
+  if ((s = step_state_build(&c, g, src, st)) != VDN_OK) return finish(s);
+  if ((s = step_state_scan(&c, g, st)) != VDN_OK) return finish(s);
+  if (cudaStreamWaitEvent(st, ev[2], 0) != cudaSuccess) return finish(VDN_ERR_CUDA);
+  if ((s = step_sparse_softmax(&c, g, src, st)) != VDN_OK) return finish(s);
+  if (cudaStreamWaitEvent(st, ev[3], 0) != cudaSuccess) return finish(VDN_ERR_CUDA);
+  if ((s = step_readout_merge(&c, g, src, dv + h.gs, dv + h.gl, dv + h.out, st)) != VDN_OK) return finish(s);
+  ce = cudaMemcpyAsync(out, dv + h.out, vid, cudaMemcpyDeviceToHost, st);
+  if (ce == cudaSuccess && c.output_mode == VDN_OUTPUT_SPLIT)
+    ce = cudaMemcpyAsync(cfg->out_linear, dv + h.out_lin, vid, cudaMemcpyDeviceToHost, st);
+  return finish(ce == cudaSuccess ? VDN_OK : VDN_ERR_CUDA);
 }
 
 }  // extern "C"

@@ -17,13 +17,13 @@ __device__ __forceinline__ float phi_f(float x) {
 // swizzle (box b at byte offset b * 16384, row r at r * 128 inside a box, the
 // 16-byte chunk index XOR-ed with r % 8).  Rows >= n_valid and columns >=
 // d_real become 0; every other element x becomes bf16(phi(x)).  Called by
-// nthreads threads with tid in [0, nthreads).
+// nthreads threads with tid in [0, nthreads).  kB chunks per thread and
+// batch: all loads first, then compute and store, so the shared-memory round
+// trips of a thread overlap (fewer when the caller keeps other registers live).
+template <int kB = 8>
 __device__ __forceinline__ void phi_tile_inplace(uint8_t* tile, int nbox, int n_valid, int d_real, int tid,
                                                  int nthreads) {
   const int nchunks = nbox * 1024;
-  // Eight chunks per batch: all loads first, then compute and store, so the
-  // shared-memory round trips of a thread overlap.
-  constexpr int kB = 8;
   for (int q0 = tid; q0 < nchunks; q0 += kB * nthreads) {
     uint4 v[kB];
     uint4* ptr[kB];
