@@ -252,6 +252,16 @@ vdn_status step_readout_merge(const vdn_cfg* cfg, const Geom& g, const Srcs& s, 
   p.out_linear = cfg->output_mode == VDN_OUTPUT_SPLIT ? cfg->out_linear : nullptr;
   p.flags = cfg->debug_flags & (VDN_OUT_SOFTMAX_ONLY | VDN_OUT_LINEAR_ONLY | VDN_OUT_LINEAR_RAW);
   p.status = status_ptr(cfg, g);
+  if (!g.fp32_io && g.d == g.Dp) {
+    // bf16 tensors without head_dim padding: every input tile by TMA
+    MergeMaps mm;
+    mm.q = m.q;
+    const long long vrows = (long long)g.B * g.N;
+    if (!make_map(&mm.os, ws(cfg, g.off_os), vrows, g.H, g.Dp) || !make_map(&mm.gs, gs, vrows, g.H, g.Dp) ||
+        !make_map(&mm.gl, gl, vrows, g.H, g.Dp))
+      return VDN_ERR_CUDA;
+    return cuda_status(launch_readout_merge_tma(mm, p, st));
+  }
   return cuda_status(launch_readout_merge(m, p, st));
 }
 

@@ -1,0 +1,343 @@
+// k4_merge_tma.cu - linear-branch readout and gated fusion of the VDN-H3
+// hybrid attention (article sections 双分支混合注意力机制 and
+// 自适应门控融合双分支输出) for bf16 tensors whose head_dim needs no padding
+// (64 or 128): every input tile arrives by TMA, so the merge reads shared
+// memory instead of waiting on scattered global loads.
+//
+// Same persistent walk as k4_readout_merge (CTA k keeps head k % H and takes
+// the 128-row tiles s, s + S, ... of stream s = k / H).  Per tile:
+//   * warp 0 (one thread) TMA-loads the q tile, and, one tile later, the
+//     tile's o_s, gate_s and gate_l tiles (128 rows x head_dim each); it
+//     bulk-copies M_c (bf16 hi/lo readout operand) when the chunk changes and
+//     prefetches the next tiles into L2;
+//   * warp 1 (one thread): D = phi(Q) M_hi^T + phi(Q) M_lo^T (M = 128,
+//     N = head_dim + 16, fp32) into one of two TMEM accumulators: numerators
+//     in the first head_dim columns, the denominator phi(q) . z after them;
+//   * warps 2-9 (256 threads) apply phi to the q tile in place (MMA operand),
+//     then finish the previous tile: each thread owns half a TMEM row, forms
+//     o_l = num / den (0 for an empty state or a GLOBAL anchor query row),
+//     exchanges the row's sum of squares with the partner half, and merges
+//     its own 8-column pieces: out = sigmoid(g_s) o_s + sigmoid(g_l) r with
+//     r = o_l / sqrt(mean(o_l^2) + eps) * gamma, reading o_s and the gates from
+//     the 128-byte-swizzled shared tiles and storing 16 bytes at a time (SPLIT:
+//     the two terms to out and out_linear).
+// Every wait is bounded; worker warps agree on giving up through barriers
+// with an OR reduction, so none is left waiting for another.
+#include "k4_common.cuh"
+#include "kernels.h"
+#include "phi.cuh"
+#include "sm100.cuh"
+
+namespace vdn {
+
+namespace {
+
+using namespace k4;
+
+template <int D>
+struct K4TLayout {
+  static constexpr int kRows = D + 16;
+  static constexpr int kTile = 128 * D * 2;   // one bf16 128-row tile (q, o_s, g_s or g_l)
+  static constexpr int kBTile = kRows * D * 2;
+  static constexpr int kA = 0;                // q tile, phi applied in place
+  static constexpr int kB = kA + kTile;       // M_c hi, lo
+  static constexpr int kG = kB + 2 * kBTile;  // o_s, g_s, g_l tiles of the tile being merged
+  static constexpr int kSs = kG + 3 * kTile;  // [2 tiles][2 halves][128] sums of squares
+  static constexpr int kBar = kSs + 4 * 128 * 4;
+  static constexpr int kBytes = kBar + 128 + 1024;
+  static constexpr int kAccCols = D + 16 <= 128 ? 128 : 256;  // one accumulator
+};
+
+enum {
+  kTAFull = 0, kTAReady = 1, kTAEmpty = 2, kTAccFull = 3, kTAccEmpty = 5, kTBFull = 7, kTBEmpty = 8,
+  kTGFull = 9, kTGEmpty = 10, kTDone = 11, kTNumBars = 12
+};
+constexpr int kTWorkers = 256;
+constexpr int kTThreads = 64 + kTWorkers;
+
+// 16-byte piece (8 bf16) of row `row`, columns [col, col + 8) of a 128-row
+// tile loaded by TMA as 64-column boxes with the 128-byte swizzle.
+__device__ __forceinline__ uint4 tile_piece(const uint8_t* tile, int row, int col) {
+  const int box = col >> 6, chunk = (col & 63) >> 3;
+  return *reinterpret_cast<const uint4*>(tile + box * 16384 + row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(kTThreads, 1)
+    k4_merge_tma(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_os,
+                 const __grid_constant__ CUtensorMap tm_gs, const __grid_constant__ CUtensorMap tm_gl,
+                 const __grid_constant__ K4Params p, int n_streams) {
+  using L = K4TLayout<D>;
+  constexpr int kCols = D + 16;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + kTNumBars * 8);
+  int* abort_flag = reinterpret_cast<int*>(smem + L::kBar + kTNumBars * 8 + 4);
+  float* ss_part = reinterpret_cast<float*>(smem + L::kSs);
+
+  const Geom& g = p.g;
+  const int tiles = (g.rows_per_chunk + 127) / 128;
+  const int head = blockIdx.x % g.H, stream = blockIdx.x / g.H;
+  const int positions = g.B * g.Nc * tiles;
+  const int n = stream < positions ? (positions - stream + n_streams - 1) / n_streams : 0;  // tiles of this CTA
+  const uint32_t warp = warp_id(), lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[kTAFull], 1);
+    mbar_init(&bars[kTAReady], kTWorkers);
+    mbar_init(&bars[kTAEmpty], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars[kTAccFull + s], 1);
+      mbar_init(&bars[kTAccEmpty + s], kTWorkers);
+    }
+    mbar_init(&bars[kTBFull], 1);
+    mbar_init(&bars[kTBEmpty], 1);
+    mbar_init(&bars[kTGFull], 1);
+    mbar_init(&bars[kTGEmpty], kTWorkers);
+    mbar_init(&bars[kTDone], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 2 * L::kAccCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const CtaAbort ab{abort_flag, p.status};
+  auto row0_of = [&](const Item4& it) { return it.b * (int)g.N + it.c * g.rows_per_chunk + it.tile * 128; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ loads
+    if (lane == 0) {
+      int prev_key = -1, b_loads = 0, a_issued = 0, g_issued = 0;
+      bool ok = true;
+      // step i: q of tile i, then o_s and the gates of tile i - 1 (they are
+      // needed one tile later, once the merge of tile i - 2 has freed the buffer)
+      for (int i = 0; i <= n && ok; ++i) {
+        if (i < n) {
+          const Item4 it = decode4(i, head, stream, n_streams, g, tiles);
+          if (it.key != prev_key) {
+            if (b_loads > 0 && !mbar_wait(&bars[kTBEmpty], (b_loads - 1) & 1, ab)) { ok = false; break; }
+            mbar_expect_tx(&bars[kTBFull], (uint32_t)(2 * L::kBTile));
+            bulk_load(smem + L::kB, p.mt + (((size_t)it.b * g.Nc + it.c) * g.H + it.h) * 2 * (size_t)L::kBTile,
+                      (uint32_t)(2 * L::kBTile), &bars[kTBFull]);
+            ++b_loads;
+            prev_key = it.key;
+          }
+          if (!mbar_wait(&bars[kTAEmpty], (i & 1) ^ 1, ab)) { ok = false; break; }
+          mbar_expect_tx(&bars[kTAFull], (uint32_t)L::kTile);
+          for (int bx = 0; bx < D / 64; ++bx)
+            tma_load_2d(smem + L::kA + bx * 16384, &tm_q, &bars[kTAFull], it.h * D + bx * 64, row0_of(it));
+          ++a_issued;
+          // warm L2 for what the next steps load
+          if (i + 1 < n) {
+            const Item4 nx = decode4(i + 1, head, stream, n_streams, g, tiles);
+            for (int bx = 0; bx < D / 64; ++bx) tma_prefetch_2d(&tm_q, nx.h * D + bx * 64, row0_of(nx));
+          }
+          for (int bx = 0; bx < D / 64; ++bx) {
+            tma_prefetch_2d(&tm_os, it.h * D + bx * 64, row0_of(it));
+            tma_prefetch_2d(&tm_gs, it.h * D + bx * 64, row0_of(it));
+            tma_prefetch_2d(&tm_gl, it.h * D + bx * 64, row0_of(it));
+          }
+        }
+        if (i >= 1) {
+          const Item4 it = decode4(i - 1, head, stream, n_streams, g, tiles);
+          if (!mbar_wait(&bars[kTGEmpty], ((i - 1) & 1) ^ 1, ab)) { ok = false; break; }
+          mbar_expect_tx(&bars[kTGFull], (uint32_t)(3 * L::kTile));
+          for (int bx = 0; bx < D / 64; ++bx) {
+            tma_load_2d(smem + L::kG + bx * 16384, &tm_os, &bars[kTGFull], it.h * D + bx * 64, row0_of(it));
+            tma_load_2d(smem + L::kG + L::kTile + bx * 16384, &tm_gs, &bars[kTGFull], it.h * D + bx * 64,
+                        row0_of(it));
+            tma_load_2d(smem + L::kG + 2 * L::kTile + bx * 16384, &tm_gl, &bars[kTGFull], it.h * D + bx * 64,
+                        row0_of(it));
+          }
+          ++g_issued;
+        }
+      }
+      if (!ok) {  // let loads in flight land before the CTA exits
+        if (a_issued > 0) mbar_drain(&bars[kTAFull], (a_issued - 1) & 1);
+        if (g_issued > 0) mbar_drain(&bars[kTGFull], (g_issued - 1) & 1);
+        if (b_loads > 0) mbar_drain(&bars[kTBFull], (b_loads - 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, kCols, 0, 0);
+      const uint64_t a_desc0 = smem_desc(smem_u32(smem + L::kA), 16, 1024, kLayoutSw128);
+      const uint64_t b_desc0 = smem_desc(smem_u32(smem + L::kB), 16, 1024, kLayoutSw128);
+      int prev_key = -1, b_loads = 0;
+      for (int i = 0; i < n; ++i) {
+        const Item4 it = decode4(i, head, stream, n_streams, g, tiles);
+        const int s = i & 1;
+        if (it.key != prev_key) {
+          ++b_loads;
+          prev_key = it.key;
+          if (!mbar_wait(&bars[kTBFull], (b_loads - 1) & 1, ab)) break;
+        }
+        if (!mbar_wait(&bars[kTAReady], i & 1, ab)) break;
+        if (!mbar_wait(&bars[kTAccEmpty + s], ((i >> 1) & 1) ^ 1, ab)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t a = a_desc0 + (uint64_t)((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4);
+            const uint64_t b =
+                b_desc0 + (uint64_t)((hl * L::kBTile + (kk >> 2) * (L::kRows * 128) + (kk & 3) * 32) >> 4);
+            mma_ss(tmem + s * L::kAccCols, a, b, idesc, (hl | kk) ? 1u : 0u);
+          }
+        mma_commit(&bars[kTAccFull + s]);
+        mma_commit(&bars[kTAEmpty]);
+        const bool key_ends = i + 1 >= n || decode4(i + 1, head, stream, n_streams, g, tiles).key != it.key;
+        if (key_ends) mma_commit(&bars[kTBEmpty]);
+      }
+      mma_commit(&bars[kTDone]);
+      mbar_drain(&bars[kTDone], 0);
+    }
+  } else {
+    // ------------------------------------------------------------ workers
+    const int tid = threadIdx.x - 64;
+    const uint32_t quarter = warp & 3, half = (warp - 2) >> 2;
+    const int row = quarter * 32 + lane;  // TMEM lane = tile row
+    const int col0 = half * (D / 2);      // this thread's columns [col0, col0 + D/2)
+    const int d = g.d;
+    const int mode = (p.flags & 1) ? 1 : ((p.flags & 6) ? 2 : 0);  // 0 merged, 1 o_s, 2 linear read
+    const bool use_gamma = p.gamma != nullptr && !(p.flags & 4);
+    const bool split = p.out_linear != nullptr;
+
+    // Finish tile j: TMEM -> o_l, RMS, merge from the shared tiles.  Returns
+    // false on a timeout (both warps of a row pair agree).
+    auto finish = [&](int j) -> bool {
+      const Item4 it = decode4(j, head, stream, n_streams, g, tiles);
+      const int s = j & 1;
+      const bool got = mbar_wait(&bars[kTAccFull + s], (j >> 1) & 1, ab);
+      if (pair_any(quarter, !got)) return false;
+      tc_fence_after();
+      const int qrow = it.c * g.rows_per_chunk + it.tile * 128 + row;
+      const bool empty = state_tokens(it.c, g) == 0 || no_linear_read(qrow / g.P, g);
+      uint32_t dr;
+      tmem_ld1(tmem_addr(tmem + s * L::kAccCols, quarter * 32, D), dr);
+      tmem_wait_ld();
+      const float inv_den = empty ? 0.f : 1.0f / __uint_as_float(dr);
+      float r[D / 2];
+#pragma unroll
+      for (int k = 0; k < D / 64; ++k) {
+        uint32_t v[32];
+        tmem_ld32(tmem_addr(tmem + s * L::kAccCols, quarter * 32, col0 + 32 * k), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[32 * k + e] = __uint_as_float(v[e]) * inv_den;
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[kTAccEmpty + s]);  // the accumulator may be overwritten now
+      float ss = 0.f;
+#pragma unroll
+      for (int a = 0; a < D / 2; ++a) ss = fmaf(r[a], r[a], ss);
+      float* ssb = ss_part + s * 256;
+      ssb[half * 128 + row] = ss;
+      pair_any(quarter, false);
+      const float inv_rms = (p.flags & 4) ? 1.0f : rsqrtf((ss + ssb[(half ^ 1) * 128 + row]) / (float)d + g.eps);
+      const bool gok = mbar_wait(&bars[kTGFull], j & 1, ab);
+      if (pair_any(quarter, !gok)) return false;
+      const int nrows = min(128, g.rows_per_chunk - it.tile * 128);
+      const size_t row_h = ((size_t)it.b * g.N + (size_t)qrow) * g.H + it.h;
+      const uint8_t* t_os = smem + L::kG;
+      const uint8_t* t_gs = smem + L::kG + L::kTile;
+      const uint8_t* t_gl = smem + L::kG + 2 * L::kTile;
+#pragma unroll
+      for (int c8 = 0; c8 < D / 16; ++c8) {
+        const int col = col0 + 8 * c8;
+        const uint4 vo = tile_piece(t_os, row, col), vs = tile_piece(t_gs, row, col), vl = tile_piece(t_gl, row, col);
+        const uint32_t ow[4] = {vo.x, vo.y, vo.z, vo.w};
+        const uint32_t sw[4] = {vs.x, vs.y, vs.z, vs.w};
+        const uint32_t lw[4] = {vl.x, vl.y, vl.z, vl.w};
+        float os[8], gs[8], gl[8], rr[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          os[2 * k] = bf16_lo(ow[k]); os[2 * k + 1] = bf16_hi(ow[k]);
+          gs[2 * k] = bf16_lo(sw[k]); gs[2 * k + 1] = bf16_hi(sw[k]);
+          gl[2 * k] = bf16_lo(lw[k]); gl[2 * k + 1] = bf16_hi(lw[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) rr[k] = r[8 * c8 + k] * inv_rms;
+        if (use_gamma) {
+          const float4 ga = __ldg(reinterpret_cast<const float4*>(p.gamma + it.h * d + col));
+          const float4 gb = __ldg(reinterpret_cast<const float4*>(p.gamma + it.h * d + col) + 1);
+          rr[0] *= ga.x; rr[1] *= ga.y; rr[2] *= ga.z; rr[3] *= ga.w;
+          rr[4] *= gb.x; rr[5] *= gb.y; rr[6] *= gb.z; rr[7] *= gb.w;
+        }
+        float o[8];
+        if (split) {
+          float ol[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            o[k] = sigmoid_f(gs[k]) * os[k];
+            ol[k] = sigmoid_f(gl[k]) * rr[k];
+          }
+          if (row < nrows) store8<false>(p.out_linear, row_h * d + col, ol);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float merged = sigmoid_f(gs[k]) * os[k] + sigmoid_f(gl[k]) * rr[k];
+            o[k] = mode == 0 ? merged : (mode == 1 ? os[k] : rr[k]);
+          }
+        }
+        if (row < nrows) store8<false>(p.out, row_h * d + col, o);
+      }
+      mbar_arrive(&bars[kTGEmpty]);  // the shared tiles may be reloaded now
+      return true;
+    };
+
+    bool ok = true;
+    for (int i = 0; i < n && ok; ++i) {
+      const bool got = mbar_wait(&bars[kTAFull], i & 1, ab);
+      if (workers_any(!got)) { ok = false; break; }
+      phi_tile_inplace(smem + L::kA, D / 64, 128, d, tid, kTWorkers);
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[kTAReady]);
+      if (i > 0) ok = !workers_any(!finish(i - 1));
+    }
+    if (ok && n > 0) finish(n - 1);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * L::kAccCols);
+  }
+}
+
+size_t k4_merge_tma_smem(int Dp) {
+  return Dp == 128 ? (size_t)K4TLayout<128>::kBytes : (size_t)K4TLayout<64>::kBytes;
+}
+
+template <int D>
+static cudaError_t launch_k4t(const MergeMaps& m, const K4Params& p, cudaStream_t st) {
+  const int smem = K4TLayout<D>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(k4_merge_tma<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int tiles = (p.g.rows_per_chunk + 127) / 128;
+  const int positions = tiles * p.g.Nc * p.g.B;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int n_streams = sms / p.g.H;
+  if (n_streams < 1) n_streams = 1;
+  if (n_streams > positions) n_streams = positions;
+  k4_merge_tma<D><<<n_streams * p.g.H, kTThreads, smem, st>>>(m.q, m.os, m.gs, m.gl, p, n_streams);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_readout_merge_tma(const MergeMaps& m, const K4Params& p, cudaStream_t st) {
+  return p.g.Dp == 128 ? launch_k4t<128>(m, p, st) : launch_k4t<64>(m, p, st);
+}
+
+}  // namespace vdn

@@ -27,6 +27,7 @@
 //     query read nothing through the states (o_l = 0).
 // Every wait is bounded; the worker warps agree on giving up through a
 // barrier with an OR reduction, so none is left waiting for another.
+#include "k4_common.cuh"
 #include "kernels.h"
 #include "phi.cuh"
 #include "sm100.cuh"
@@ -34,6 +35,8 @@
 namespace vdn {
 
 namespace {
+
+using namespace k4;
 
 template <int D>
 struct K4Layout {
@@ -54,25 +57,6 @@ enum { kAFull = 0, kAReady = 2, kAEmpty = 4, kAccFull = 6, kAccEmpty = 8, kBFull
 constexpr int kWorkers = 256;
 constexpr int kK4Threads = 64 + kWorkers;
 
-// sigmoid(x) = (1 + tanh(x / 2)) / 2 with the hardware tanh (one special-function op)
-__device__ __forceinline__ float sigmoid_f(float x) {
-  float t;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
-  return fmaf(0.5f, t, 0.5f);
-}
-
-template <bool FP32>
-__device__ __forceinline__ void store8(void* base, size_t idx, const float (&x)[8]) {
-  if constexpr (FP32) {
-    float4* p = reinterpret_cast<float4*>(static_cast<float*>(base) + idx);
-    p[0] = make_float4(x[0], x[1], x[2], x[3]);
-    p[1] = make_float4(x[4], x[5], x[6], x[7]);
-  } else {
-    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + idx) =
-        make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
-  }
-}
-
 // r staging: row-major fp32 [128][D]; the 16-byte chunk j of row r is stored
 // at chunk j ^ (r % (D/4)) so that 32 rows written column-wise, or 2 rows read
 // row-wise, spread over all banks.
@@ -80,38 +64,6 @@ template <int D>
 __device__ __forceinline__ float4* r_chunk(uint8_t* base, int row, int j) {
   constexpr int kChunks = D / 4;
   return reinterpret_cast<float4*>(base + (size_t)row * D * 4 + ((j ^ (row & (kChunks - 1))) << 4));
-}
-
-// Barrier among the 256 worker threads (id 1) that also ORs a predicate:
-// every worker leaves with the same answer.
-__device__ __forceinline__ bool workers_any(bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 256, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)pred)
-      : "memory");
-  return r != 0;
-}
-
-struct Item4 {
-  int b, h, c, tile, key;
-};
-
-// The i-th item of the CTA (head h, stream s of n_streams).
-__device__ __forceinline__ Item4 decode4(int i, int h, int s, int n_streams, const Geom& g, int tiles) {
-  Item4 it;
-  const int pos = s + i * n_streams;  // (batch, chunk, tile) position
-  it.tile = pos % tiles;
-  const int rem = pos / tiles;
-  it.c = rem % g.Nc;
-  it.b = rem / g.Nc;
-  it.h = h;
-  it.key = rem;  // (batch, chunk) of this head identifies the readout operand
-  return it;
 }
 
 }  // namespace

@@ -61,6 +61,13 @@ cudaError_t launch_state_build(const Maps& m, const K1Params& p, cudaStream_t st
 cudaError_t launch_state_scan(const K2Params& p, cudaStream_t st);
 cudaError_t launch_sparse_softmax(const Maps& m, const K3Params& p, int grid, cudaStream_t st);
 cudaError_t launch_readout_merge(const Maps& m, const K4Params& p, cudaStream_t st);
+
+// Maps of the TMA-fed readout/merge (bf16, head_dim == Dp): q, o_s and the
+// two gates as 2-D [rows, H*Dp] views like Maps.
+struct MergeMaps {
+  CUtensorMap q, os, gs, gl;
+};
+cudaError_t launch_readout_merge_tma(const MergeMaps& m, const K4Params& p, cudaStream_t st);
 cudaError_t launch_membership(const Geom& g, uint8_t* table, cudaStream_t st);
 
 size_t k3_smem_bytes(int Dp);
