@@ -13,8 +13,12 @@
 //   * warp 1 (one thread): D = phi(Q) M_hi^T + phi(Q) M_lo^T (M = 128,
 //     N = head_dim + 16, fp32) into one of two TMEM accumulators: numerators
 //     in the first head_dim columns, the denominator phi(q) . z after them;
-//   * warps 2-9 (256 threads) apply phi to the q tile in place (MMA operand),
-//     then finish the previous tile: each thread owns half a TMEM row, forms
+//     phi(Q) itself is the A operand, read from TMEM (columns of the same
+//     accumulator slot that the accumulator leaves free);
+//   * warps 2-9 (256 threads) each take half a row of the q tile from shared
+//     memory, apply phi and store it to TMEM as bf16 (the q buffer is free for
+//     the next tile's load right after), then finish the previous tile: each
+//     thread owns half a TMEM row, forms
 //     o_l = num / den (0 for an empty state or a GLOBAL anchor query row),
 //     exchanges the row's sum of squares with the partner half, and merges
 //     its own 8-column pieces: out = sigmoid(g_s) o_s + sigmoid(g_l) r with
@@ -45,13 +49,17 @@ struct K4TLayout {
   static constexpr int kSs = kG + 3 * kTile;  // [2 tiles][2 halves][128] sums of squares
   static constexpr int kBar = kSs + 4 * 128 * 4;
   static constexpr int kBytes = kBar + 128 + 1024;
-  static constexpr int kAccCols = D + 16 <= 128 ? 128 : 256;  // one accumulator
+  static constexpr int kAccCols = D + 16 <= 128 ? 128 : 256;  // one accumulator slot
+  static constexpr int kPhiCol = kAccCols - D / 2;             // phi(Q) (bf16 pairs) at the slot's end
+  static_assert(kPhiCol >= D + 16, "phi(Q) must not overlap the accumulator");
 };
 
 enum {
   kTAFull = 0, kTAReady = 1, kTAEmpty = 2, kTAccFull = 3, kTAccEmpty = 5, kTBFull = 7, kTBEmpty = 8,
   kTGFull = 9, kTGEmpty = 10, kTDone = 11, kTNumBars = 12
 };
+// kTAReady: phi(Q) of the tile is in TMEM (workers); kTAEmpty: the workers have
+// read the q tile out of shared memory (the producer may load the next one).
 constexpr int kTWorkers = 256;
 constexpr int kTThreads = 64 + kTWorkers;
 
@@ -88,7 +96,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars[kTAFull], 1);
     mbar_init(&bars[kTAReady], kTWorkers);
-    mbar_init(&bars[kTAEmpty], 1);
+    mbar_init(&bars[kTAEmpty], kTWorkers);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[kTAccFull + s], 1);
       mbar_init(&bars[kTAccEmpty + s], kTWorkers);
@@ -170,7 +178,6 @@ __global__ void __launch_bounds__(kTThreads, 1)
     // ------------------------------------------------------------ MMA
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, kCols, 0, 0);
-      const uint64_t a_desc0 = smem_desc(smem_u32(smem + L::kA), 16, 1024, kLayoutSw128);
       const uint64_t b_desc0 = smem_desc(smem_u32(smem + L::kB), 16, 1024, kLayoutSw128);
       int prev_key = -1, b_loads = 0;
       for (int i = 0; i < n; ++i) {
@@ -188,13 +195,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
         for (int hl = 0; hl < 2; ++hl)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t a = a_desc0 + (uint64_t)((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4);
             const uint64_t b =
                 b_desc0 + (uint64_t)((hl * L::kBTile + (kk >> 2) * (L::kRows * 128) + (kk & 3) * 32) >> 4);
-            mma_ss(tmem + s * L::kAccCols, a, b, idesc, (hl | kk) ? 1u : 0u);
+            mma_ts(tmem + s * L::kAccCols, tmem + s * L::kAccCols + L::kPhiCol + kk * 8, b, idesc,
+                   (hl | kk) ? 1u : 0u);
           }
         mma_commit(&bars[kTAccFull + s]);
-        mma_commit(&bars[kTAEmpty]);
         const bool key_ends = i + 1 >= n || decode4(i + 1, head, stream, n_streams, g, tiles).key != it.key;
         if (key_ends) mma_commit(&bars[kTBEmpty]);
       }
@@ -299,9 +305,29 @@ __global__ void __launch_bounds__(kTThreads, 1)
     for (int i = 0; i < n && ok; ++i) {
       const bool got = mbar_wait(&bars[kTAFull], i & 1, ab);
       if (workers_any(!got)) { ok = false; break; }
-      phi_tile_inplace(smem + L::kA, D / 64, 128, d, tid, kTWorkers);
-      fence_proxy_async_smem();
-      mbar_arrive(&bars[kTAReady]);
+      // phi of this thread's half row, bf16 pairs into the free columns of
+      // accumulator slot i % 2 (the MMA of tile i - 2, which read that slot's
+      // phi(Q), completed before finish(i - 2) returned)
+      {
+        uint32_t pk[D / 4];
+#pragma unroll
+        for (int c8 = 0; c8 < D / 16; ++c8) {
+          const uint4 v = tile_piece(smem + L::kA, row, col0 + 8 * c8);
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) pk[4 * c8 + e] = pack_bf16x2(phi_f(bf16_lo(w[e])), phi_f(bf16_hi(w[e])));
+        }
+        mbar_arrive(&bars[kTAEmpty]);  // q tile read: the next one may be loaded
+        const uint32_t base = tmem_addr(tmem + (i & 1) * L::kAccCols, quarter * 32, L::kPhiCol + col0 / 2);
+        if constexpr (D == 128) {
+          tmem_st32(base, pk);
+        } else {
+          tmem_st16(base, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars[kTAReady]);
+      }
       if (i > 0) ok = !workers_any(!finish(i - 1));
     }
     if (ok && n > 0) finish(n - 1);
