@@ -93,6 +93,8 @@ SMALL = [
     Workload("d64_fp32", 1, 9, 50, 2, 64, 7, 3, "fp32", "normal", 19),
     Workload("d128_fp32", 1, 5, 300, 1, 128, 130, 1, "fp32", "rms", 20),
     Workload("tiny_tokens", 1, 7, 1, 2, 64, 1, 1, "bf16", "normal", 21),
+    # the most chunks the scan keeps on chip (96), one-frame chunks
+    Workload("max_chunks", 1, 96, 4, 1, 64, 3, 1, "bf16", "normal", 23),
 ]
 
 
@@ -122,7 +124,8 @@ def test_branches_match_oracle(w):
 # ----------------------------------------------------------------- GLOBAL anchor queries, SPLIT output
 
 
-GLOBAL_CASES = [SMALL[i] for i in (0, 2, 3, 4, 5, 7, 10, 12)]
+GLOBAL_CASES = [SMALL[i] for i in (0, 2, 3, 4, 5, 7, 9, 10, 12, 13)] + [
+    Workload("global_b2_c3", 2, 12, 100, 2, 128, 20, 3, "bf16", "normal", 22)]
 
 
 @pytest.mark.parametrize("F,C,P,T", [(15, 1, 16, 8), (45, 5, 4, 3), (1, 1, 5, 2), (2, 1, 5, 2), (6, 6, 2, 1),
@@ -143,7 +146,7 @@ def test_global_anchor_mode_matches_oracle(w):
     assert_close(o_s.float().cpu().numpy(), ref["o_s"], f"{w.name} o_s (GLOBAL)")
 
 
-@pytest.mark.parametrize("w", [SMALL[0], SMALL[1], SMALL[3]], ids=["tiny", "small", "c5_ragged"])
+@pytest.mark.parametrize("w", [SMALL[0], SMALL[1], SMALL[3], SMALL[9]], ids=["tiny", "small", "c5_ragged", "d32"])
 def test_split_output_matches_oracle(w):
     inputs = make_inputs(w)
     dev = to_dev(inputs)
