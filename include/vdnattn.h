@@ -93,7 +93,12 @@ enum {
   VDN_OUT_SOFTMAX_ONLY = 1, /* out = o_s (no gate) */
   VDN_OUT_LINEAR_ONLY = 2,  /* out = r, the RMS-normalised linear read (no gate) */
   VDN_OUT_LINEAR_RAW = 4,   /* out = o_l, the linear read before RMSNorm */
-  VDN_EXPORT_STATES = 8     /* vdn_state_scan also writes S_F/z_F and S_B/z_B (fp32) */
+  VDN_EXPORT_STATES = 8,    /* vdn_state_scan also writes S_F/z_F and S_B/z_B (fp32) */
+  VDN_INJECT_TIMEOUT = 16   /* test of the failure path only: in the state build, the MMA thread of
+                               CTA (0, 0) first waits, with a ~2^24-cycle limit, for a barrier phase
+                               that nothing completes; it gives up, the CTA's other warps follow, the
+                               kernel writes VDN_ERR_TIMEOUT to status_word and returns.  The call's
+                               outputs are then undefined; the context stays usable. */
 };
 
 typedef struct {

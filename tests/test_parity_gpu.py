@@ -292,3 +292,26 @@ def test_global_anchor_mode_sampled_rows_768p():
                                  prob, 0, 0, rows)
         got = out[0, torch.from_numpy(rows).cuda(), h, :].float().cpu().numpy()
         assert_close(got, ref["out"], f"768p GLOBAL head {h}")
+
+
+# ----------------------------------------------------------------- failure path
+
+
+@pytest.mark.parametrize("w", [SMALL[0], Workload("inject_8tiles", 1, 6, 1024, 1, 64, 8, 1, "bf16", "normal", 24)],
+                         ids=["tiny", "eight_tiles"])
+def test_injected_timeout_reports_status_and_context_survives(w):
+    """A wait that nothing completes (VDN_INJECT_TIMEOUT: one CTA of the
+    state build, ~2^24-cycle limit) ends with VDN_ERR_TIMEOUT in the status
+    word instead of a hang or a fault, and the next call is correct."""
+    import time
+    inputs = make_inputs(w)
+    dev = to_dev(inputs)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.time()
+    run(w, dev, debug_flags=vb.INJECT_TIMEOUT, status=status)
+    assert time.time() - t0 < 30
+    assert int(status.item()) == 6
+    status.zero_()
+    out = run(w, dev, status=status)
+    assert int(status.item()) == 0
+    assert_close(out.float().cpu().numpy(), oracle_full(w, inputs)["out"], f"{w.name} after the injected timeout")

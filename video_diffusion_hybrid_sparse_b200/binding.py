@@ -18,7 +18,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvdnattn
 _lib = None
 
 VDN_BF16, VDN_FP32 = 0, 1
-OUT_SOFTMAX_ONLY, OUT_LINEAR_ONLY, OUT_LINEAR_RAW, EXPORT_STATES = 1, 2, 4, 8
+OUT_SOFTMAX_ONLY, OUT_LINEAR_ONLY, OUT_LINEAR_RAW, EXPORT_STATES, INJECT_TIMEOUT = 1, 2, 4, 8, 16
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "pointer not aligned",
           4: "workspace missing or too small", 5: "CUDA error", 6: "device wait timed out"}
 

@@ -34,7 +34,8 @@ vdn_status make_geom(const vdn_cfg* cfg, Geom& g) {
   if (cfg->frames % cfg->chunk_frames != 0) return VDN_ERR_INVALID_ARG;
   if (cfg->head_dim != 32 && cfg->head_dim != 64 && cfg->head_dim != 128) return VDN_ERR_UNSUPPORTED;
   if (cfg->dtype != VDN_BF16 && cfg->dtype != VDN_FP32) return VDN_ERR_UNSUPPORTED;
-  if (cfg->debug_flags & ~(VDN_OUT_SOFTMAX_ONLY | VDN_OUT_LINEAR_ONLY | VDN_OUT_LINEAR_RAW | VDN_EXPORT_STATES))
+  if (cfg->debug_flags &
+      ~(VDN_OUT_SOFTMAX_ONLY | VDN_OUT_LINEAR_ONLY | VDN_OUT_LINEAR_RAW | VDN_EXPORT_STATES | VDN_INJECT_TIMEOUT))
     return VDN_ERR_INVALID_ARG;
   const int Nc = cfg->frames / cfg->chunk_frames;
   if (Nc > kMaxScanChunks) return VDN_ERR_UNSUPPORTED;
@@ -193,6 +194,7 @@ vdn_status step_state_build(const vdn_cfg* cfg, const Geom& g, const Srcs& s, cu
   p.g = g;
   p.parts = reinterpret_cast<float*>(ws(cfg, g.off_parts));
   p.status = status_ptr(cfg, g);
+  p.inject_timeout = (cfg->debug_flags & VDN_INJECT_TIMEOUT) != 0;
   return cuda_status(launch_state_build(m, p, st));
 }
 

@@ -136,7 +136,12 @@ __global__ void __launch_bounds__(kK1Threads, 1)
       constexpr uint32_t idesc_v = idesc_bf16_f32(128, D, 1, 1);
       constexpr uint32_t idesc_1 = idesc_bf16_f32(128, 16, 1, 1);
       const uint32_t ones = smem_u32(smem + L::kOnes);
-      for (int i = 0; i < ntiles; ++i) {
+      // failure-path test: wait (with a short limit) for the accumulator
+      // phase, which only this thread's final commit completes; the wait runs
+      // out, the CTA gives up and the status word records the timeout
+      const bool injected = p.inject_timeout && blockIdx.x == 0 && blockIdx.y == 0 &&
+                            !mbar_wait(&bars[kAcc], 0, ab, 1ll << 24);
+      for (int i = 0; i < ntiles && !injected; ++i) {
         const int st = i % L::kStages;
         if (!mbar_wait(&bars[kPhi + st], (i / L::kStages) & 1, ab)) break;
         tc_fence_after();

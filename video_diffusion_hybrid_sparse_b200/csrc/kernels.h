@@ -26,6 +26,7 @@ struct K1Params {
   Geom g;
   float* parts;            // [n_parts, B, H, Dp+1, Dp] fp32; row Dp holds z
   int* status;
+  int inject_timeout;      // test only: CTA (0, 0) waits for a phase nothing completes (short limit)
 };
 
 struct K2Params {

@@ -161,9 +161,11 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Bounded: gives up
-// after kWaitCycles or when another warp of the CTA has given up, returning
-// false.  Every thread that calls it must act on a false return.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const CtaAbort& ab) {
+// after `limit` cycles (kWaitCycles by default) or when another warp of the CTA
+// has given up, returning false.  Every thread that calls it must act on a
+// false return.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const CtaAbort& ab,
+                                          long long limit = kWaitCycles) {
   if (mbar_test_wait(bar, parity)) return true;  // already complete: no suspension
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
@@ -172,7 +174,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     if (mbar_try_wait(bar, parity)) return true;
     if ((++n & 63u) == 0) {
       if (aborted(ab)) return false;
-      if (clock64() - t0 > kWaitCycles) {
+      if (clock64() - t0 > limit) {
         raise_abort(ab);
         return false;
       }
