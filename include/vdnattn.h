@@ -88,6 +88,15 @@ typedef enum { VDN_BF16 = 0, VDN_FP32 = 1 } vdn_dtype;
 typedef enum { VDN_ANCHOR_LOCAL = 0, VDN_ANCHOR_GLOBAL = 1 } vdn_anchor_query_mode;
 typedef enum { VDN_OUTPUT_MERGED = 0, VDN_OUTPUT_SPLIT = 1 } vdn_output_mode;
 
+/* Operand precision of the softmax branch's two contractions.  BF16 (default):
+ * bf16 operands, fp32 accumulation.  FP8: q, k, v, text_k, text_v quantised
+ * to e4m3 with one scale per (batch, head) for q, one for k and text_k, one for
+ * v and text_v (scale = max |x| / 448); P in e4m3; fp32 accumulation; o_s and
+ * everything after it as in BF16.  FP8 needs head_dim 128, bf16 tensors and
+ * tokens_per_frame % 16 == 0 (VDN_ERR_UNSUPPORTED otherwise), and a larger
+ * workspace (vdn_workspace_bytes accounts for it). */
+typedef enum { VDN_PREC_BF16 = 0, VDN_PREC_FP8 = 1 } vdn_softmax_precision;
+
 /* debug_flags: what vdn_readout_merge writes into out instead of the merge. */
 enum {
   VDN_OUT_SOFTMAX_ONLY = 1, /* out = o_s (no gate) */
@@ -121,7 +130,7 @@ typedef struct {
   float* export_fwd;        /* VDN_EXPORT_STATES: device [B, F/C, H, d+1, d] fp32; row d holds z */
   float* export_bwd;        /* same layout, backward states */
   int32_t output_mode;      /* vdn_output_mode; 0 = MERGED.  SPLIT excludes the VDN_OUT_* debug flags */
-  int32_t reserved1;        /* must be 0 */
+  int32_t softmax_precision; /* vdn_softmax_precision; 0 = BF16 */
   void* out_linear;         /* SPLIT only: device [B, N, H, d] in dtype, 16-byte aligned; else ignored */
 } vdn_cfg;
 

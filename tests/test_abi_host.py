@@ -71,8 +71,15 @@ def test_validate_rejects_unknown_dtype_and_flags():
     cfg = vb.make_cfg(shape(), debug_flags=64)
     assert lib.vdn_validate(ctypes.byref(cfg)) == 1
     cfg = vb.make_cfg(shape())
-    cfg.reserved1 = 3
+    cfg.softmax_precision = 3
     assert lib.vdn_validate(ctypes.byref(cfg)) == 1
+    # fp8 softmax: head_dim 128, bf16, tokens per frame a multiple of 16
+    assert vb.validate(shape(d=128, P=32), softmax_precision=vb.PREC_FP8) == 0
+    assert vb.validate(shape(d=64, P=32), softmax_precision=vb.PREC_FP8) == 2
+    assert vb.validate(shape(d=128, P=30), softmax_precision=vb.PREC_FP8) == 2
+    assert vb.validate(shape(d=128, P=32, fp32=True), softmax_precision=vb.PREC_FP8) == 2
+    s8 = shape(d=128, P=32)
+    assert vb.workspace_bytes(s8, vb.PREC_FP8) > vb.workspace_bytes(s8)
     for mode in (2, -1):
         cfg = vb.make_cfg(shape())
         cfg.anchor_query_mode = mode

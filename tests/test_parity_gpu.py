@@ -315,3 +315,67 @@ def test_injected_timeout_reports_status_and_context_survives(w):
     out = run(w, dev, status=status)
     assert int(status.item()) == 0
     assert_close(out.float().cpu().numpy(), oracle_full(w, inputs)["out"], f"{w.name} after the injected timeout")
+
+
+# ----------------------------------------------------------------- fp8 softmax branch
+#
+# Tolerance for softmax_precision = FP8, derived from e4m3: three mantissa
+# bits, so a rounded operand is off by at most 2^-4 of its value (RMS
+# 2^-4 / sqrt(3) ~ 3.6 %).  Each term of o_s = sum p v / sum p carries the
+# rounding of v, of p, and the perturbation of p by the rounding of q and k in
+# the logit (~5 % RMS for unit-RMS rows at head_dim 128): ~7 % RMS per term,
+# independent across keys, so o_s keeps a relative error of that order:
+# rel-L2 <= 0.1 for o_s.  The merged output is dominated by the linear branch
+# and the gates: rel-L2 <= 1e-2 as for bf16, and max-abs <= 4e-2 (the bf16
+# output rounding, up to 1.6e-2, plus sigmoid(g_s) times the o_s error).
+
+FP8_CASES = [Workload("fp8_rms", 1, 6, 256, 2, 128, 32, 1, "bf16", "rms", 25),
+             Workload("fp8_c3", 1, 9, 96, 2, 128, 40, 3, "bf16", "normal", 26),
+             Workload("fp8_b2_no_text", 2, 4, 128, 1, 128, 0, 1, "bf16", "half", 27)]
+
+
+@pytest.mark.parametrize("w", FP8_CASES, ids=[w.name for w in FP8_CASES])
+def test_fp8_softmax_matches_oracle(w):
+    inputs = make_inputs(w)
+    dev = to_dev(inputs)
+    ref = oracle_full(w, inputs)
+    out = run(w, dev, softmax_precision=vb.PREC_FP8)
+    assert_close(out.float().cpu().numpy(), ref["out"], f"{w.name} out (fp8)", abs_tol=4e-2, rel_tol=1e-2)
+    o_s = run(w, dev, softmax_precision=vb.PREC_FP8, debug_flags=vb.OUT_SOFTMAX_ONLY)
+    scale = np.abs(ref["o_s"]).max()
+    assert_close(o_s.float().cpu().numpy(), ref["o_s"], f"{w.name} o_s (fp8)", abs_tol=0.25 * scale, rel_tol=0.1)
+    again = run(w, dev, softmax_precision=vb.PREC_FP8)
+    assert torch.equal(out, again)
+
+
+def test_fp8_global_anchor_mode():
+    w = FP8_CASES[1]
+    inputs = make_inputs(w)
+    dev = to_dev(inputs)
+    ref = oracle_full(w, inputs, mode="global")
+    out = run(w, dev, softmax_precision=vb.PREC_FP8, anchor_query_mode=vb.ANCHOR_GLOBAL)
+    assert_close(out.float().cpu().numpy(), ref["out"], f"{w.name} out (fp8, GLOBAL)", abs_tol=4e-2, rel_tol=1e-2)
+
+
+def test_fp8_rejects_unsupported_shapes():
+    w = SMALL[3]  # c5_ragged: 130 tokens per frame, not a multiple of 16
+    dev = to_dev(make_inputs(w))
+    with pytest.raises(vb.VdnError) as e:
+        run(w, dev, softmax_precision=vb.PREC_FP8)
+    assert e.value.code == 2
+
+
+def test_fp8_768p_sampled_rows():
+    w = BY_NAME["768p_bf16"]
+    inputs = make_inputs(w)
+    dev = to_dev(inputs)
+    out = run(w, dev, softmax_precision=vb.PREC_FP8)
+    del dev
+    rows = sample_rows(w, np.random.default_rng(7))
+    prob = O.Problem(B=1, F=w.F, P=w.P, H=1, d=w.d, T=w.T, C=w.C)
+    for h in (0, 23):
+        x = {k: np64(t[:, :, h:h + 1, :]) for k, t in inputs.items()}
+        ref = O.hybrid_attn_rows(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], x["gate_s"], x["gate_l"],
+                                 prob, 0, 0, rows)
+        got = out[0, torch.from_numpy(rows).cuda(), h, :].float().cpu().numpy()
+        assert_close(got, ref["out"], f"768p fp8 head {h}", abs_tol=4e-2, rel_tol=1e-2)

@@ -45,7 +45,7 @@ class VdnCfg(ctypes.Structure):
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("status_word", ctypes.c_void_p),
         ("export_fwd", ctypes.c_void_p), ("export_bwd", ctypes.c_void_p),
-        ("output_mode", ctypes.c_int32), ("reserved1", ctypes.c_int32),
+        ("output_mode", ctypes.c_int32), ("softmax_precision", ctypes.c_int32),
         ("out_linear", ctypes.c_void_p),
     ]
 
@@ -107,11 +107,12 @@ class Shape:
 
 ANCHOR_LOCAL, ANCHOR_GLOBAL = 0, 1
 OUTPUT_MERGED, OUTPUT_SPLIT = 0, 1
+PREC_BF16, PREC_FP8 = 0, 1
 
 
 def make_cfg(s: Shape, *, softmax_scale: float = 0.0, rms_eps: float = -1.0, rms_weight=None,
              debug_flags: int = 0, workspace=None, status=None, export=None,
-             anchor_query_mode: int = ANCHOR_LOCAL, out_linear=None) -> VdnCfg:
+             anchor_query_mode: int = ANCHOR_LOCAL, out_linear=None, softmax_precision: int = PREC_BF16) -> VdnCfg:
     cfg = VdnCfg()
     cfg.batch, cfg.frames, cfg.tokens_per_frame = s.B, s.F, s.P
     cfg.heads, cfg.head_dim, cfg.text_tokens, cfg.chunk_frames = s.H, s.d, s.T, s.C
@@ -122,6 +123,7 @@ def make_cfg(s: Shape, *, softmax_scale: float = 0.0, rms_eps: float = -1.0, rms
     cfg.debug_flags = debug_flags
     cfg.anchor_query_mode = anchor_query_mode
     cfg.output_mode = OUTPUT_SPLIT if out_linear is not None else OUTPUT_MERGED
+    cfg.softmax_precision = softmax_precision
     cfg.out_linear = _ptr(out_linear)
     if workspace is not None:
         cfg.workspace = workspace.data_ptr()
@@ -153,19 +155,20 @@ def shape_of(q: torch.Tensor, text_k: torch.Tensor, frames: int, chunk_frames: i
     return Shape(B, frames, N // frames, H, d, text_k.shape[1], chunk_frames, q.dtype == torch.float32)
 
 
-def workspace_bytes(s: Shape) -> int:
-    n = library().vdn_workspace_bytes(ctypes.byref(make_cfg(s)))
+def workspace_bytes(s: Shape, softmax_precision: int = PREC_BF16) -> int:
+    cfg = make_cfg(s, softmax_precision=softmax_precision)
+    n = library().vdn_workspace_bytes(ctypes.byref(cfg))
     if n == 0:
-        _check(library().vdn_validate(ctypes.byref(make_cfg(s))), "vdn_workspace_bytes")
+        _check(library().vdn_validate(ctypes.byref(cfg)), "vdn_workspace_bytes")
     return n
 
 
 _WS: dict = {}
 
 
-def workspace_for(s: Shape, device) -> torch.Tensor:
+def workspace_for(s: Shape, device, softmax_precision: int = PREC_BF16) -> torch.Tensor:
     """A cached device workspace large enough for shape s."""
-    n = workspace_bytes(s)
+    n = workspace_bytes(s, softmax_precision)
     dev = torch.device(device)
     key = (dev.index if dev.index is not None else torch.cuda.current_device())
     buf = _WS.get(key)
@@ -178,7 +181,8 @@ def workspace_for(s: Shape, device) -> torch.Tensor:
 def hybrid_attn_fwd(q, k, v, text_k, text_v, gate_s, gate_l, *, frames: int, chunk_frames: int, out=None,
                     softmax_scale: float = 0.0, rms_eps: float = -1.0, rms_weight=None, debug_flags: int = 0,
                     workspace=None, status=None, export=None, stream=None,
-                    anchor_query_mode: int = ANCHOR_LOCAL, out_linear=None) -> torch.Tensor:
+                    anchor_query_mode: int = ANCHOR_LOCAL, out_linear=None,
+                    softmax_precision: int = PREC_BF16) -> torch.Tensor:
     """The whole hybrid attention call on the current CUDA stream.
 
     q, k, v, gate_s, gate_l: [B, F*P, H, d]; text_k, text_v: [B, T, H, d];
@@ -189,10 +193,11 @@ def hybrid_attn_fwd(q, k, v, text_k, text_v, gate_s, gate_l, *, frames: int, chu
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
-        workspace = workspace_for(s, q.device)
+        workspace = workspace_for(s, q.device, softmax_precision)
     cfg = make_cfg(s, softmax_scale=softmax_scale, rms_eps=rms_eps, rms_weight=rms_weight,
                    debug_flags=debug_flags, workspace=workspace, status=status, export=export,
-                   anchor_query_mode=anchor_query_mode, out_linear=out_linear)
+                   anchor_query_mode=anchor_query_mode, out_linear=out_linear,
+                   softmax_precision=softmax_precision)
     code = library().vdn_hybrid_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(text_k), _ptr(text_v),
                                          gate_s.data_ptr(), gate_l.data_ptr(), out.data_ptr(),
                                          ctypes.byref(cfg), _stream(stream))
@@ -223,7 +228,7 @@ def staging_for(s: Shape, device, split: bool = False) -> torch.Tensor:
 def hybrid_attn_fwd_host(q, k, v, text_k, text_v, gate_s, gate_l, *, frames: int, chunk_frames: int, out=None,
                          softmax_scale: float = 0.0, rms_eps: float = -1.0, rms_weight=None, workspace=None,
                          staging=None, stream=None, anchor_query_mode: int = ANCHOR_LOCAL,
-                         out_linear=None, device="cuda") -> torch.Tensor:
+                         out_linear=None, device="cuda", softmax_precision: int = PREC_BF16) -> torch.Tensor:
     """The whole call on HOST tensors (contiguous CPU tensors, ideally pinned),
     copies overlapped with the kernels inside the library.  Returns the host
     ``out``; synchronise ``stream`` (default: the current stream of
@@ -232,11 +237,11 @@ def hybrid_attn_fwd_host(q, k, v, text_k, text_v, gate_s, gate_l, *, frames: int
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, pin_memory=q.is_pinned())
     if workspace is None:
-        workspace = workspace_for(s, device)
+        workspace = workspace_for(s, device, softmax_precision)
     if staging is None:
         staging = staging_for(s, device, out_linear is not None)
     cfg = make_cfg(s, softmax_scale=softmax_scale, rms_eps=rms_eps, rms_weight=rms_weight, workspace=workspace,
-                   anchor_query_mode=anchor_query_mode, out_linear=out_linear)
+                   anchor_query_mode=anchor_query_mode, out_linear=out_linear, softmax_precision=softmax_precision)
     code = library().vdn_hybrid_attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(text_k), _ptr(text_v),
                                               gate_s.data_ptr(), gate_l.data_ptr(), out.data_ptr(),
                                               staging.data_ptr(), staging.numel(), ctypes.byref(cfg),
@@ -251,13 +256,13 @@ class Steps:
 
     def __init__(self, q, k, v, text_k, text_v, gate_s, gate_l, out, *, frames, chunk_frames, workspace=None,
                  debug_flags=0, rms_weight=None, export=None, status=None, anchor_query_mode=ANCHOR_LOCAL,
-                 out_linear=None):
+                 out_linear=None, softmax_precision=PREC_BF16):
         self.t = (q, k, v, text_k, text_v, gate_s, gate_l, out)
         self.s = shape_of(q, text_k, frames, chunk_frames)
-        self.ws = workspace if workspace is not None else workspace_for(self.s, q.device)
+        self.ws = workspace if workspace is not None else workspace_for(self.s, q.device, softmax_precision)
         self.cfg = make_cfg(self.s, workspace=self.ws, debug_flags=debug_flags, rms_weight=rms_weight,
                             export=export, status=status, anchor_query_mode=anchor_query_mode,
-                            out_linear=out_linear)
+                            out_linear=out_linear, softmax_precision=softmax_precision)
         self.lib = library()
 
     def stage(self, stream=None):

@@ -23,8 +23,13 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 vdn_status make_geom(const vdn_cfg* cfg, Geom& g) {
   if (!cfg) return VDN_ERR_INVALID_ARG;
   if (cfg->batch < 1 || cfg->frames < 1 || cfg->tokens_per_frame < 1 || cfg->heads < 1 || cfg->text_tokens < 0 ||
-      cfg->chunk_frames < 1 || cfg->reserved1 != 0)
+      cfg->chunk_frames < 1)
     return VDN_ERR_INVALID_ARG;
+  if (cfg->softmax_precision != VDN_PREC_BF16 && cfg->softmax_precision != VDN_PREC_FP8) return VDN_ERR_INVALID_ARG;
+  if (cfg->softmax_precision == VDN_PREC_FP8 &&
+      (cfg->head_dim != 128 || cfg->dtype != VDN_BF16 || cfg->tokens_per_frame % 16 != 0 ||
+       (long long)cfg->batch * cfg->heads * 5 * 4 > 48 * 1024))
+    return VDN_ERR_UNSUPPORTED;
   if (cfg->anchor_query_mode != VDN_ANCHOR_LOCAL && cfg->anchor_query_mode != VDN_ANCHOR_GLOBAL)
     return VDN_ERR_INVALID_ARG;
   if (cfg->output_mode != VDN_OUTPUT_MERGED && cfg->output_mode != VDN_OUTPUT_SPLIT) return VDN_ERR_INVALID_ARG;
@@ -83,6 +88,18 @@ vdn_status make_geom(const vdn_cfg* cfg, Geom& g) {
   }
   g.off_parts = off; off = align_up(off + (size_t)g.n_parts * g.B * g.H * (g.Dp + 1) * g.Dp * 4, 1024);
   g.off_mt = off; off = align_up(off + (size_t)g.B * g.Nc * g.H * 2 * g.mt_rows * g.Dp * 2, 1024);
+  g.fp8 = cfg->softmax_precision == VDN_PREC_FP8;
+  if (g.fp8) {
+    g.pitch_v8 = (long long)align_up((size_t)g.N, 16);
+    g.pitch_t8 = (long long)align_up((size_t)g.T, 16);
+    const size_t vid8 = (size_t)g.B * g.N * g.H * 128, txt8 = (size_t)g.B * g.T * g.H * 128;
+    g.off_q8 = off; off = align_up(off + vid8, 1024);
+    g.off_k8 = off; off = align_up(off + vid8, 1024);
+    g.off_vt8 = off; off = align_up(off + (size_t)g.B * g.H * 128 * g.pitch_v8, 1024);
+    g.off_tk8 = off; off = align_up(off + txt8, 1024);
+    g.off_tvt8 = off; off = align_up(off + (size_t)g.B * g.H * 128 * g.pitch_t8, 1024);
+    g.off_amax = off; off = align_up(off + sizeof(float) * 5 * g.B * g.H, 1024);
+  }
   g.total = off;
   return VDN_OK;
 }
@@ -139,6 +156,22 @@ bool make_map(CUtensorMap* m, const void* base, long long rows, int H, int Dp) {
   const cuuint32_t box[2] = {64, 128};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D e4m3 (byte) view [rows, cols] with the given row pitch (bytes), box 128 x
+// 128, 128-byte swizzle.
+bool make_map8(CUtensorMap* m, const void* base, long long rows, long long cols, long long pitch) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  if (rows < 1) rows = 1;
+  if (cols < 1) cols = 1;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(pitch < 16 ? 16 : pitch)};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -215,6 +248,31 @@ vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s,
   K3Params p;
   std::memset(&p, 0, sizeof(p));
   p.g = g;
+  if (g.fp8) {
+    // e4m3 operands, then the same walk with kind::f8f6f4 MMAs
+    Fp8Src src{{static_cast<const __nv_bfloat16*>(s.q), static_cast<const __nv_bfloat16*>(s.k),
+                static_cast<const __nv_bfloat16*>(s.v), static_cast<const __nv_bfloat16*>(s.tk),
+                static_cast<const __nv_bfloat16*>(s.tv)}};
+    Fp8Dst dst{ws(cfg, g.off_q8), ws(cfg, g.off_k8), ws(cfg, g.off_vt8), ws(cfg, g.off_tk8), ws(cfg, g.off_tvt8),
+               g.pitch_v8, g.pitch_t8};
+    float* amax = reinterpret_cast<float*>(ws(cfg, g.off_amax));
+    cudaError_t e = launch_fp8_quant(src, dst, g.B, g.N, g.T, g.H, amax, st);
+    if (e != cudaSuccess) return VDN_ERR_CUDA;
+    const long long vrows = (long long)g.B * g.N, trows = (long long)g.B * g.T, vtrows = (long long)g.B * g.H * 128;
+    if (!make_map8(&m.q, dst.q, vrows, (long long)g.H * 128, (long long)g.H * 128) ||
+        !make_map8(&m.k, dst.k, vrows, (long long)g.H * 128, (long long)g.H * 128) ||
+        !make_map8(&m.v, dst.vt, vtrows, g.N, g.pitch_v8))
+      return VDN_ERR_CUDA;
+    if (g.T > 0) {
+      if (!make_map8(&m.tk, dst.tk, trows, (long long)g.H * 128, (long long)g.H * 128) ||
+          !make_map8(&m.tv, dst.tvt, vtrows, g.T, g.pitch_t8))
+        return VDN_ERR_CUDA;
+    } else {
+      m.tk = m.q;
+      m.tv = m.q;
+    }
+    p.fp8_amax = amax;
+  }
   p.scale_log2 = g.scale * 1.4426950408889634f;
   p.o_s = reinterpret_cast<__nv_bfloat16*>(ws(cfg, g.off_os));
   p.status = status_ptr(cfg, g);
@@ -236,7 +294,7 @@ vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s,
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::min(p.n_items, sms);
-  return cuda_status(launch_sparse_softmax(m, p, grid, st));
+  return cuda_status(g.fp8 ? launch_sparse_softmax_fp8(m, p, grid, st) : launch_sparse_softmax(m, p, grid, st));
 }
 
 vdn_status step_readout_merge(const vdn_cfg* cfg, const Geom& g, const Srcs& s, const void* gs, const void* gl,

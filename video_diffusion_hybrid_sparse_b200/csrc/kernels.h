@@ -13,6 +13,7 @@ struct K3Params {
   Geom g;
   float scale_log2;        // softmax scale * log2(e)
   __nv_bfloat16* o_s;      // [B, N, H, Dp] bf16
+  const float* fp8_amax;   // fp8 branch: [5][B][H] maxima of q, k, v, text_k, text_v
   int* status;
   int n_items;             // sum over segments of B * H * pairs
   int n_segs;
@@ -61,6 +62,9 @@ cudaError_t launch_stage(const void* src, int fp32_in, __nv_bfloat16* dst, long 
 cudaError_t launch_state_build(const Maps& m, const K1Params& p, cudaStream_t st);
 cudaError_t launch_state_scan(const K2Params& p, cudaStream_t st);
 cudaError_t launch_sparse_softmax(const Maps& m, const K3Params& p, int grid, cudaStream_t st);
+// fp8 branch (head_dim 128): Maps of the e4m3 q, k, text_k ([rows, H * 128]
+// bytes) and of v, text_v transposed ([B * H * 128, tokens] bytes).
+cudaError_t launch_sparse_softmax_fp8(const Maps& m, const K3Params& p, int grid, cudaStream_t st);
 cudaError_t launch_readout_merge(const Maps& m, const K4Params& p, cudaStream_t st);
 
 // Maps of the TMA-fed readout/merge (bf16, head_dim == Dp): q, o_s and the
@@ -70,6 +74,20 @@ struct MergeMaps {
 };
 cudaError_t launch_readout_merge_tma(const MergeMaps& m, const K4Params& p, cudaStream_t st);
 cudaError_t launch_membership(const Geom& g, uint8_t* table, cudaStream_t st);
+
+// e4m3 operands of the fp8 softmax branch (head_dim 128): q, k, text_k in their
+// [rows, H * 128] layout, v and text_v transposed to [(b * H + h) * 128 + dd,
+// token] with row pitches pitch_v / pitch_t (multiples of 16 bytes); amax is
+// [5][B][H] (q, k, v, text_k, text_v), the scale of a tensor is amax / 448.
+struct Fp8Src {
+  const __nv_bfloat16* p[5];
+};
+struct Fp8Dst {
+  uint8_t *q, *k, *vt, *tk, *tvt;
+  long long pitch_v, pitch_t;
+};
+cudaError_t launch_fp8_quant(const Fp8Src& src, const Fp8Dst& dst, int B, long long N, int T, int H, float* amax,
+                             cudaStream_t st);
 
 size_t k3_smem_bytes(int Dp);
 

@@ -51,6 +51,9 @@ struct Geom {
   float eps;                // RMSNorm epsilon
   // workspace layout (byte offsets; each 1024-aligned)
   size_t off_status, off_os, off_q, off_k, off_v, off_tk, off_tv, off_parts, off_mt, total;
+  int fp8;                  // softmax branch with e4m3 operands
+  long long pitch_v8, pitch_t8;  // row pitches (bytes) of the transposed e4m3 v and text_v
+  size_t off_q8, off_k8, off_vt8, off_tk8, off_tvt8, off_amax;
 };
 
 VDN_HD int is_anchor(int f, int F) { return f == 0 || f == F - 1; }
