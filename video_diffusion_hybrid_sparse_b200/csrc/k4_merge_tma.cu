@@ -209,7 +209,6 @@ __global__ void __launch_bounds__(kTThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ workers
-    const int tid = threadIdx.x - 64;
     const uint32_t quarter = warp & 3, half = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;  // TMEM lane = tile row
     const int col0 = half * (D / 2);      // this thread's columns [col0, col0 + D/2)
