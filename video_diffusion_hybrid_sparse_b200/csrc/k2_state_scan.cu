@@ -7,15 +7,17 @@
 // columns a) one thread:
 //   1. sums the slice partials of every non-anchor frame into its chunk,
 //      cs[c] = sum_{f in chunk c, f not an anchor} [S|z]_f  (fp32; partials
-//      are read in batches of four for memory-level parallelism), and the text
-//      partials into t;
+//      are read in batches of kScanBatch for memory-level parallelism; parts
+//      are ordered by frame, so one register sum per chunk is kept and
+//      written out when the chunk changes), and the text partials into t;
 //   2. turns cs into running prefix sums P[c] = sum_{c' <= c} cs[c'] and forms
 //      F_c = t/2 + P[c-2],  B_c = t/2 + (P[Nc-1] - P[c+1]),  M_c = F_c + B_c
 //      (B_c is exactly t/2 for the last two chunks);
 //   3. writes M_c as a bf16 hi/lo pair (hi = bf16(M), lo = bf16(M - hi)) into
 //      the readout's B-operand image: rows n (value column; row Dp = z, rows
-//      Dp+1..Dp+15 zero), K = a, K-major with the 128-byte swizzle, so the
-//      readout copies it to shared memory with one bulk copy;
+//      Dp+1..Dp+15 zero, written by the threads of rows 0..14, one row
+//      each), K = a, K-major with the 128-byte swizzle, so the readout copies
+//      it to shared memory with one bulk copy;
 //   4. optionally exports F_c and B_c in fp32.
 // The chunk sums live in shared memory, thread-fastest ([Nc][4][threads]).
 #include "kernels.h"
@@ -24,6 +26,12 @@
 namespace vdn {
 
 namespace {
+
+#ifndef VDN_K2_BATCH
+#define VDN_K2_BATCH 10
+#endif
+constexpr int kScanBatch = VDN_K2_BATCH;  // partial loads in flight per thread
+constexpr int kScanThreads = 128;
 
 __device__ __forceinline__ uint32_t mt_offset(int n, int a, int rows) {
   // byte offset of element (row n, column a) in one K-major SW128 B-tile image
@@ -34,7 +42,7 @@ __device__ __forceinline__ uint32_t mt_offset(int n, int a, int rows) {
 
 }  // namespace
 
-__global__ void k2_state_scan(const __grid_constant__ K2Params p, int n_threads_total) {
+__global__ void __launch_bounds__(kScanThreads) k2_state_scan(const __grid_constant__ K2Params p, int n_threads_total) {
   extern __shared__ float scan_smem[];
   const Geom& g = p.g;
   const int Dp = g.Dp;
@@ -57,25 +65,36 @@ __global__ void k2_state_scan(const __grid_constant__ K2Params p, int n_threads_
 #pragma unroll
     for (int e = 0; e < 4; ++e) cs[(c * 4 + e) * T_] = 0.f;
   float t[4] = {0.f, 0.f, 0.f, 0.f};
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  int cur = -1;  // chunk held in acc
 
-  for (int p0 = 0; p0 < g.n_parts; p0 += 4) {
-    float4 x[4];
+  for (int p0 = 0; p0 < g.n_parts; p0 += kScanBatch) {
+    float4 x[kScanBatch];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      x[u] = (p0 + u < g.n_parts) ? __ldg(reinterpret_cast<const float4*>(src0 + (size_t)(p0 + u) * part_stride))
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < kScanBatch; ++u)
+      if (p0 + u < g.n_parts) x[u] = __ldg(reinterpret_cast<const float4*>(src0 + (size_t)(p0 + u) * part_stride));
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kScanBatch; ++u) {
       const int pp = p0 + u;
       if (pp >= g.n_parts) break;
       if (pp < g.n_video_parts) {
-        float* dst = cs + (part_frame(pp, g) / g.C) * 4 * T_;
-        dst[0] += x[u].x; dst[T_] += x[u].y; dst[2 * T_] += x[u].z; dst[3 * T_] += x[u].w;
+        const int ch = part_frame(pp, g) / g.C;
+        if (ch != cur) {
+          if (cur >= 0)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) cs[(cur * 4 + e) * T_] = acc[e];
+          cur = ch;
+          acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+        }
+        acc[0] += x[u].x; acc[1] += x[u].y; acc[2] += x[u].z; acc[3] += x[u].w;
       } else {
         t[0] += x[u].x; t[1] += x[u].y; t[2] += x[u].z; t[3] += x[u].w;
       }
     }
   }
+  if (cur >= 0)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) cs[(cur * 4 + e) * T_] = acc[e];
 
   // running prefix sums in place
   for (int c = 1; c < Nc; ++c)
@@ -88,6 +107,8 @@ __global__ void k2_state_scan(const __grid_constant__ K2Params p, int n_threads_
   const bool exp_row = (n < d) || (n == Dp);
   const int exp_n = (n == Dp) ? d : n;
   const uint32_t off = mt_offset(n, a4 * 4, rows);
+  const bool zero_row = n < 15;
+  const uint32_t off_z = mt_offset(Dp + 1 + (zero_row ? n : 0), a4 * 4, rows);
   for (int c = 0; c < Nc; ++c) {
     const int fl = fwd_last_chunk(c), bf = bwd_first_chunk(c);
     float Fv[4], Bv[4], M[4];
@@ -110,12 +131,9 @@ __global__ void k2_state_scan(const __grid_constant__ K2Params p, int n_threads_
     }
     *reinterpret_cast<uint2*>(tile + off) = make_uint2(hi[0], hi[1]);
     *reinterpret_cast<uint2*>(tile + tile_bytes + off) = make_uint2(lo[0], lo[1]);
-    if (n == Dp) {
-      for (int z = Dp + 1; z < rows; ++z) {  // zero padding rows
-        const uint32_t oz = mt_offset(z, a4 * 4, rows);
-        *reinterpret_cast<uint2*>(tile + oz) = make_uint2(0, 0);
-        *reinterpret_cast<uint2*>(tile + tile_bytes + oz) = make_uint2(0, 0);
-      }
+    if (zero_row) {
+      *reinterpret_cast<uint2*>(tile + off_z) = make_uint2(0, 0);
+      *reinterpret_cast<uint2*>(tile + tile_bytes + off_z) = make_uint2(0, 0);
     }
     if (p.export_fwd && exp_row) {
       const size_t base = ((((size_t)b * Nc + c) * g.H + h) * (d + 1) + exp_n) * d;
@@ -135,7 +153,7 @@ int k2_threads_per_block(int Nc) {
   // chunk sums in shared memory: Nc * 16 bytes per thread, at most ~96 KB per block
   int tpb = (96 * 1024) / (Nc * 16);
   tpb = (tpb / 32) * 32;
-  if (tpb > 256) tpb = 256;
+  if (tpb > kScanThreads) tpb = kScanThreads;
   return tpb;
 }
 
