@@ -143,10 +143,13 @@ def gpu_id_for(local_rank: int) -> str:
 
 
 def kernel_source_hash(name: str) -> str:
-    files = {"sparse_softmax": "k3_sparse_softmax.cu"}
-    path = os.path.join(ROOT, "video_diffusion_hybrid_sparse_b200", "csrc", files[name])
-    with open(path, "rb") as fh:
-        return hashlib.sha1(fh.read()).hexdigest()[:12]
+    """sha1 of the kernel's source file and of the headers it is compiled with."""
+    files = {"sparse_softmax": ["k3_sparse_softmax.cu", "sm100.cuh", "plan.h", "kernels.h"]}
+    h = hashlib.sha1()
+    for f in files[name]:
+        with open(os.path.join(ROOT, "video_diffusion_hybrid_sparse_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
 
 
 def recorded_traffic(kernel: str, workload: str):

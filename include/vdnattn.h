@@ -53,9 +53,13 @@
  *
  * Errors: every argument check happens before anything is enqueued; on an
  * error return nothing was launched.  VDN_ERR_CUDA reports a launch error
- * (cudaGetLastError).  A kernel whose bounded wait runs out (about 2 s)
- * writes VDN_ERR_TIMEOUT into *status_word (when given) and returns early;
- * that is read by the caller after synchronising.
+ * (cudaGetLastError).  A kernel whose bounded wait runs out (1 s of global
+ * time) writes VDN_ERR_TIMEOUT into *status_word (when given) and returns
+ * early; that is read by the caller after synchronising.  The first such wait
+ * also describes itself in a timeout record, 16 int32 words at byte 64 of the
+ * workspace (count of waits that ran out, kernel id, block, warp, barrier as
+ * its byte distance to the CTA's abort flag, phase parity, nanoseconds waited
+ * as two words, SM); the library never clears it, the caller may.
  */
 #ifndef VDNATTN_H
 #define VDNATTN_H
@@ -103,11 +107,15 @@ enum {
   VDN_OUT_LINEAR_ONLY = 2,  /* out = r, the RMS-normalised linear read (no gate) */
   VDN_OUT_LINEAR_RAW = 4,   /* out = o_l, the linear read before RMSNorm */
   VDN_EXPORT_STATES = 8,    /* vdn_state_scan also writes S_F/z_F and S_B/z_B (fp32) */
-  VDN_INJECT_TIMEOUT = 16   /* test of the failure path only: in the state build, the MMA thread of
-                               CTA (0, 0) first waits, with a ~2^24-cycle limit, for a barrier phase
+  VDN_INJECT_TIMEOUT = 16,  /* test of the failure path only: in the state build, the MMA thread of
+                               CTA (0, 0) first waits, with a 10-ms limit, for a barrier phase
                                that nothing completes; it gives up, the CTA's other warps follow, the
                                kernel writes VDN_ERR_TIMEOUT to status_word and returns.  The call's
                                outputs are then undefined; the context stays usable. */
+  VDN_STALL_READOUT_MMA = 32 /* test of the readout's barrier protocol only: the readout's MMA thread
+                               sleeps 50 microseconds whenever it moves to another readout operand
+                               (batch, chunk, head), letting the other warps run as far ahead as the
+                               protocol allows.  Outputs are unchanged. */
 };
 
 typedef struct {

@@ -70,6 +70,9 @@ def test_validate_rejects_unknown_dtype_and_flags():
     assert lib.vdn_validate(ctypes.byref(cfg)) == 2
     cfg = vb.make_cfg(shape(), debug_flags=64)
     assert lib.vdn_validate(ctypes.byref(cfg)) == 1
+    for flag in (vb.INJECT_TIMEOUT, vb.STALL_READOUT_MMA):
+        cfg = vb.make_cfg(shape(), debug_flags=flag)
+        assert lib.vdn_validate(ctypes.byref(cfg)) == 0
     cfg = vb.make_cfg(shape())
     cfg.softmax_precision = 3
     assert lib.vdn_validate(ctypes.byref(cfg)) == 1

@@ -255,11 +255,14 @@ def test_workload_sampled_rows(name, heads):
     w = BY_NAME[name]
     inputs = make_inputs(w)
     dev = to_dev(inputs)
+    ws = vb.workspace_for(vb.shape_of(dev["q"], dev["text_k"], w.F, w.C), dev["q"].device)
+    vb.clear_timeout_record(ws)
     status1 = torch.zeros(1, dtype=torch.int32, device="cuda")
-    out = run(w, dev, status=status1)
+    out = run(w, dev, status=status1, workspace=ws)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    out2 = run(w, dev, status=status)
-    assert int(status1.item()) == 0 and int(status.item()) == 0, "a bounded wait ran out"
+    out2 = run(w, dev, status=status, workspace=ws)
+    assert int(status1.item()) == 0 and int(status.item()) == 0, \
+        f"a bounded wait ran out: statuses {int(status1.item())}, {int(status.item())}; {vb.timeout_record(ws)}"
     same = out.view(torch.int16) == out2.view(torch.int16)
     if not bool(same.all()):
         bad = (~same).nonzero()
@@ -310,20 +313,53 @@ def test_global_anchor_mode_sampled_rows_768p():
                          ids=["tiny", "eight_tiles"])
 def test_injected_timeout_reports_status_and_context_survives(w):
     """A wait that nothing completes (VDN_INJECT_TIMEOUT: one CTA of the
-    state build, ~2^24-cycle limit) ends with VDN_ERR_TIMEOUT in the status
-    word instead of a hang or a fault, and the next call is correct."""
+    state build, 10-ms limit) ends with VDN_ERR_TIMEOUT in the status word
+    instead of a hang or a fault, the timeout record names that wait, and the
+    next call is correct."""
     import time
     inputs = make_inputs(w)
     dev = to_dev(inputs)
+    ws = vb.workspace_for(vb.shape_of(dev["q"], dev["text_k"], w.F, w.C), dev["q"].device)
+    vb.clear_timeout_record(ws)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     t0 = time.time()
-    run(w, dev, debug_flags=vb.INJECT_TIMEOUT, status=status)
+    run(w, dev, debug_flags=vb.INJECT_TIMEOUT, status=status, workspace=ws)
     assert time.time() - t0 < 30
     assert int(status.item()) == 6
+    rec = vb.timeout_record(ws)
+    assert rec["timeouts"] >= 1 and rec["kernel"] == 1 and rec["block"] == 0, rec
+    assert 10_000_000 <= rec["ns"] < 1_000_000_000, rec
+    vb.clear_timeout_record(ws)
     status.zero_()
     out = run(w, dev, status=status)
     assert int(status.item()) == 0
     assert_close(out.float().cpu().numpy(), oracle_full(w, inputs)["out"], f"{w.name} after the injected timeout")
+
+
+# The readout's MMA thread held up at every readout-operand change: the other
+# warps run as far ahead as the barrier protocol allows (in the TMA-fed
+# readout they once completed two phases of the phi-ready barrier before the
+# MMA thread waited on the first, which then waited on a third for good).
+# 37 heads put four CTAs on each head; with eight 128-row tiles per chunk each
+# CTA takes two tiles of every (batch, chunk), so the MMA thread stalls at the
+# first while the loads of the second need no new operand.  Outputs must be
+# bit-identical to an unstalled call.
+STALL_CASES = [Workload("stall_bf16", 1, 4, 1024, 37, 128, 16, 1, "bf16", "normal", 28),
+               Workload("stall_fp32", 1, 4, 1024, 37, 32, 16, 1, "fp32", "normal", 29)]
+
+
+@pytest.mark.parametrize("w", STALL_CASES, ids=[w.name for w in STALL_CASES])
+def test_readout_protocol_survives_stalled_mma_thread(w):
+    dev = to_dev(make_inputs(w))
+    ws = vb.workspace_for(vb.shape_of(dev["q"], dev["text_k"], w.F, w.C), dev["q"].device)
+    vb.clear_timeout_record(ws)
+    st0 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ref = run(w, dev, status=st0, workspace=ws)
+    st1 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = run(w, dev, status=st1, workspace=ws, debug_flags=vb.STALL_READOUT_MMA)
+    assert int(st0.item()) == 0 and int(st1.item()) == 0, vb.timeout_record(ws)
+    assert torch.equal(ref.view(torch.int16) if ref.dtype == torch.bfloat16 else ref.view(torch.int32),
+                       out.view(torch.int16) if out.dtype == torch.bfloat16 else out.view(torch.int32))
 
 
 # ----------------------------------------------------------------- fp8 softmax branch

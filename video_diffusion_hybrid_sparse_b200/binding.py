@@ -19,6 +19,7 @@ _lib = None
 
 VDN_BF16, VDN_FP32 = 0, 1
 OUT_SOFTMAX_ONLY, OUT_LINEAR_ONLY, OUT_LINEAR_RAW, EXPORT_STATES, INJECT_TIMEOUT = 1, 2, 4, 8, 16
+STALL_READOUT_MMA = 32
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "pointer not aligned",
           4: "workspace missing or too small", 5: "CUDA error", 6: "device wait timed out"}
 
@@ -206,6 +207,27 @@ def hybrid_attn_fwd(q, k, v, text_k, text_v, gate_s, gate_l, *, frames: int, chu
 
 
 _STAGING: dict = {}
+
+
+_REC_FIELDS = ("timeouts", "kernel", "block", "warp", "bar_off", "parity")
+# kernel ids in the record: 1 state build, 3 softmax (bf16), 31 softmax (fp8),
+# 4 readout + merge (TMA-fed), 41 readout + merge (general)
+
+
+def timeout_record(workspace: torch.Tensor) -> dict:
+    """The kernels' timeout record: 16 int32 words at byte 64 of the
+    workspace, describing the first bounded wait that ran out since the record
+    was cleared (kernel id, block, warp, barrier as its byte distance to the
+    CTA's abort flag, phase parity, global nanoseconds waited, SM)."""
+    w = workspace[64:128].view(torch.int32).cpu().tolist()
+    rec = dict(zip(_REC_FIELDS, w[:6]))
+    rec["ns"] = (w[6] & 0xFFFFFFFF) | (w[7] << 32)
+    rec["sm"] = w[8]
+    return rec
+
+
+def clear_timeout_record(workspace: torch.Tensor) -> None:
+    workspace[64:128].zero_()
 
 
 def staging_for(s: Shape, device, split: bool = False) -> torch.Tensor:

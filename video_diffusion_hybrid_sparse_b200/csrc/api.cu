@@ -40,7 +40,8 @@ vdn_status make_geom(const vdn_cfg* cfg, Geom& g) {
   if (cfg->head_dim != 32 && cfg->head_dim != 64 && cfg->head_dim != 128) return VDN_ERR_UNSUPPORTED;
   if (cfg->dtype != VDN_BF16 && cfg->dtype != VDN_FP32) return VDN_ERR_UNSUPPORTED;
   if (cfg->debug_flags &
-      ~(VDN_OUT_SOFTMAX_ONLY | VDN_OUT_LINEAR_ONLY | VDN_OUT_LINEAR_RAW | VDN_EXPORT_STATES | VDN_INJECT_TIMEOUT))
+      ~(VDN_OUT_SOFTMAX_ONLY | VDN_OUT_LINEAR_ONLY | VDN_OUT_LINEAR_RAW | VDN_EXPORT_STATES | VDN_INJECT_TIMEOUT |
+        VDN_STALL_READOUT_MMA))
     return VDN_ERR_INVALID_ARG;
   const int Nc = cfg->frames / cfg->chunk_frames;
   if (Nc > kMaxScanChunks) return VDN_ERR_UNSUPPORTED;
@@ -124,6 +125,13 @@ uint8_t* ws(const vdn_cfg* cfg, size_t off) { return static_cast<uint8_t*>(cfg->
 
 int* status_ptr(const vdn_cfg* cfg, const Geom& g) {
   return cfg->status_word ? cfg->status_word : reinterpret_cast<int*>(ws(cfg, g.off_status));
+}
+
+// Timeout record of the kernels' bounded waits: 16 int words at byte 64 of
+// the workspace's status slot (the workspace status word, when used, is at
+// byte 0).  Written only when a wait runs out; cleared by the caller.
+int* record_ptr(const vdn_cfg* cfg, const Geom& g) {
+  return reinterpret_cast<int*>(ws(cfg, g.off_status) + 64);
 }
 
 // ---------------------------------------------------------------- TMA descriptors
@@ -227,6 +235,7 @@ vdn_status step_state_build(const vdn_cfg* cfg, const Geom& g, const Srcs& s, cu
   p.g = g;
   p.parts = reinterpret_cast<float*>(ws(cfg, g.off_parts));
   p.status = status_ptr(cfg, g);
+  p.record = record_ptr(cfg, g);
   p.inject_timeout = (cfg->debug_flags & VDN_INJECT_TIMEOUT) != 0;
   return cuda_status(launch_state_build(m, p, st));
 }
@@ -276,6 +285,7 @@ vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s,
   p.scale_log2 = g.scale * 1.4426950408889634f;
   p.o_s = reinterpret_cast<__nv_bfloat16*>(ws(cfg, g.off_os));
   p.status = status_ptr(cfg, g);
+  p.record = record_ptr(cfg, g);
   // query segments, longest key set first (static longest-processing-time order)
   QSeg segs[kMaxSegs];
   const int n = query_segments(g, segs);
@@ -311,7 +321,9 @@ vdn_status step_readout_merge(const vdn_cfg* cfg, const Geom& g, const Srcs& s, 
   p.out = out;
   p.out_linear = cfg->output_mode == VDN_OUTPUT_SPLIT ? cfg->out_linear : nullptr;
   p.flags = cfg->debug_flags & (VDN_OUT_SOFTMAX_ONLY | VDN_OUT_LINEAR_ONLY | VDN_OUT_LINEAR_RAW);
+  p.stall_ns = (cfg->debug_flags & VDN_STALL_READOUT_MMA) ? 50000 : 0;
   p.status = status_ptr(cfg, g);
+  p.record = record_ptr(cfg, g);
   if (!g.fp32_io && g.d == g.Dp) {
     // bf16 tensors without head_dim padding: every input tile by TMA
     MergeMaps mm;

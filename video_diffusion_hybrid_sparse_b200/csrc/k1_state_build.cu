@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const CtaAbort ab{abort_flag, p.status};
+  const CtaAbort ab{abort_flag, p.status, p.record, 1};
 
   if (warp == 0) {
     if (lane == 0) {
@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
       // phase, which only this thread's final commit completes; the wait runs
       // out, the CTA gives up and the status word records the timeout
       const bool injected = p.inject_timeout && blockIdx.x == 0 && blockIdx.y == 0 &&
-                            !mbar_wait(&bars[kAcc], 0, ab, 1ll << 24);
+                            !mbar_wait(&bars[kAcc], 0, ab, 10000000ll);
       for (int i = 0; i < ntiles && !injected; ++i) {
         const int st = i % L::kStages;
         if (!mbar_wait(&bars[kPhi + st], (i / L::kStages) & 1, ab)) break;

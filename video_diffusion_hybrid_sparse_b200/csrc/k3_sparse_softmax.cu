@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const CtaAbort ab{abort_flag, p.status};
+  const CtaAbort ab{abort_flag, p.status, p.record, 3};
 
   uint8_t* sQ = smem + L::kQ;
   uint8_t* sK = smem + L::kK;

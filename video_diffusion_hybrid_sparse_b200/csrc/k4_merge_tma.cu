@@ -55,11 +55,18 @@ struct K4TLayout {
 };
 
 enum {
-  kTAFull = 0, kTAReady = 1, kTAEmpty = 2, kTAccFull = 3, kTAccEmpty = 5, kTBFull = 7, kTBEmpty = 8,
-  kTGFull = 9, kTGEmpty = 10, kTDone = 11, kTNumBars = 12
+  kTAFull = 0, kTAReady = 1, kTAEmpty = 3, kTAccFull = 4, kTAccEmpty = 6, kTBFull = 8, kTBEmpty = 9,
+  kTGFull = 10, kTGEmpty = 11, kTDone = 12, kTNumBars = 13
 };
-// kTAReady: phi(Q) of the tile is in TMEM (workers); kTAEmpty: the workers have
-// read the q tile out of shared memory (the producer may load the next one).
+// kTAReady + s: phi(Q) of a tile of accumulator slot s is in TMEM (workers);
+// kTAEmpty: the workers have read the q tile out of shared memory (the
+// producer may load the next one).  kTAReady is one barrier per slot because
+// the workers' next arrival depends only on the producer (q of the next tile),
+// not on the MMA thread having seen the previous phase: with one barrier, a
+// MMA thread held up on a readout-operand load could find two phases
+// completed and wait on the parity of a third that never comes.  Per slot,
+// the next arrival (tile i + 2) follows finish(i), which waits for the MMA of
+// tile i, so the MMA thread is never a whole phase behind.
 constexpr int kTWorkers = 256;
 constexpr int kTThreads = 64 + kTWorkers;
 
@@ -95,9 +102,9 @@ __global__ void __launch_bounds__(kTThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[kTAFull], 1);
-    mbar_init(&bars[kTAReady], kTWorkers);
     mbar_init(&bars[kTAEmpty], kTWorkers);
     for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars[kTAReady + s], kTWorkers);
       mbar_init(&bars[kTAccFull + s], 1);
       mbar_init(&bars[kTAccEmpty + s], kTWorkers);
     }
@@ -117,7 +124,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const CtaAbort ab{abort_flag, p.status};
+  const CtaAbort ab{abort_flag, p.status, p.record, 4};
   auto row0_of = [&](const Item4& it) { return it.b * (int)g.N + it.c * g.rows_per_chunk + it.tile * 128; };
 
   if (warp == 0) {
@@ -184,11 +191,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
         const Item4 it = decode4(i, head, stream, n_streams, g, tiles);
         const int s = i & 1;
         if (it.key != prev_key) {
+          if (p.stall_ns > 0 && i > 0) sleep_ns(p.stall_ns);  // debug: let the other warps run ahead
           ++b_loads;
           prev_key = it.key;
           if (!mbar_wait(&bars[kTBFull], (b_loads - 1) & 1, ab)) break;
         }
-        if (!mbar_wait(&bars[kTAReady], i & 1, ab)) break;
+        if (!mbar_wait(&bars[kTAReady + s], (i >> 1) & 1, ab)) break;
         if (!mbar_wait(&bars[kTAccEmpty + s], ((i >> 1) & 1) ^ 1, ab)) break;
         tc_fence_after();
 #pragma unroll
@@ -325,7 +333,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars[kTAReady]);
+        mbar_arrive(&bars[kTAReady + (i & 1)]);
       }
       if (i > 0) ok = !workers_any(!finish(i - 1));
     }

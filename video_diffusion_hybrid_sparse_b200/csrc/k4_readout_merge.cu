@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kK4Threads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const CtaAbort ab{abort_flag, p.status};
+  const CtaAbort ab{abort_flag, p.status, p.record, 41};
 
   if (warp == 0) {
     // ------------------------------------------------------------ loads
@@ -151,6 +151,7 @@ __global__ void __launch_bounds__(kK4Threads, 1)
         const int i = item - first, s = i & 1;
         const uint32_t ph = (i >> 1) & 1;
         if (it.key != prev_key) {
+          if (p.stall_ns > 0 && i > 0) sleep_ns(p.stall_ns);  // debug: let the other warps run ahead
           ++b_loads;
           prev_key = it.key;
           if (!mbar_wait(&bars[kBFull], (b_loads - 1) & 1, ab)) break;

@@ -15,6 +15,7 @@ struct K3Params {
   __nv_bfloat16* o_s;      // [B, N, H, Dp] bf16
   const float* fp8_amax;   // fp8 branch: [5][B][H] maxima of q, k, v, text_k, text_v
   int* status;
+  int* record;             // timeout record (workspace), may be null
   int n_items;             // sum over segments of B * H * pairs
   int n_segs;
   // query segments by decreasing KV tile count; items of segment k are
@@ -27,6 +28,7 @@ struct K1Params {
   Geom g;
   float* parts;            // [n_parts, B, H, Dp+1, Dp] fp32; row Dp holds z
   int* status;
+  int* record;             // timeout record (workspace), may be null
   int inject_timeout;      // test only: CTA (0, 0) waits for a phase nothing completes (short limit)
 };
 
@@ -48,7 +50,9 @@ struct K4Params {
   void* out;
   void* out_linear;        // SPLIT output: sigmoid(g_l) * r goes here, out gets sigmoid(g_s) * o_s
   int flags;
+  int stall_ns;            // > 0: the MMA thread sleeps this long at each readout-operand change
   int* status;
+  int* record;             // timeout record (workspace), may be null
 };
 
 // Tensor maps: 2-D bf16 views [rows, H*Dp] with a 128-row x 64-column box and

@@ -96,16 +96,52 @@ __device__ __forceinline__ float exp2_fma(float x) {
 // ------------------------------------------------------------------ abort / status
 
 // Status shared by the warps of one CTA.  A wait that runs out sets `abort`
-// (so every other waiter gives up quickly) and records VDN_ERR_TIMEOUT (6)
-// in the global status word.
+// (so every other waiter gives up quickly), records VDN_ERR_TIMEOUT (6) in
+// the global status word and describes itself in the timeout record.
 struct CtaAbort {
-  int* flag;          // shared memory
+  int* flag;           // shared memory
   int* global_status;  // device memory, may be null
+  int* record;         // device memory (kRec* words), may be null
+  int kernel;          // kernel id written into the record
 };
 
 constexpr int kStatusTimeout = 6;
-// ~2^31 SM cycles: about 1 s at 2 GHz, a few seconds at low clocks.
-constexpr long long kWaitCycles = 1ll << 31;
+// Waits are bounded in global time (%globaltimer, nanoseconds), not in SM
+// cycles: after a compute preemption a CTA may resume on another SM, whose
+// cycle counter has no relation to the one read before.
+constexpr long long kWaitNs = 1000000000ll;  // 1 s
+
+// Timeout record (int words): the first wait that ran out since the record
+// was cleared.
+enum : int {
+  kRecTimeouts = 0,  // waits that ran out
+  kRecKernel = 1,    // kernel id of the first
+  kRecBlock = 2,     // its blockIdx.x
+  kRecWarp = 3,      // its warp
+  kRecBarOff = 4,    // byte distance from its barrier to the CTA's abort flag
+  kRecParity = 5,    // the phase parity it waited for
+  kRecNs = 6,        // global nanoseconds it waited (two words, low first)
+  kRecSm = 8,        // SM it ran on
+  kRecWords = 16
+};
+
+__device__ __forceinline__ long long global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return (long long)t;
+}
+
+__device__ __forceinline__ int sm_id() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+  return (int)r;
+}
+
+// Sleep for about `ns` nanoseconds of global time (debug stalls only).
+__device__ __forceinline__ void sleep_ns(long long ns) {
+  const long long t0 = global_ns();
+  while (global_ns() - t0 < ns) __nanosleep(1000);
+}
 
 __device__ __forceinline__ bool aborted(const CtaAbort& ab) {
   return *reinterpret_cast<volatile int*>(ab.flag) != 0;
@@ -114,6 +150,22 @@ __device__ __forceinline__ bool aborted(const CtaAbort& ab) {
 __device__ __forceinline__ void raise_abort(const CtaAbort& ab) {
   *reinterpret_cast<volatile int*>(ab.flag) = 1;
   if (ab.global_status) atomicExch(ab.global_status, kStatusTimeout);
+}
+
+// Out of line: only a wait that ran out gets here.
+static __device__ __noinline__ void record_timeout(const CtaAbort& ab, const void* bar, uint32_t parity, long long ns) {
+  if (!ab.record) return;
+  if (atomicAdd(ab.record + kRecTimeouts, 1) != 0) return;
+  int* r = ab.record;
+  r[kRecKernel] = ab.kernel;
+  r[kRecBlock] = (int)blockIdx.x;
+  r[kRecWarp] = (int)(threadIdx.x >> 5);
+  r[kRecBarOff] = (int)(smem_u32(ab.flag) - smem_u32(bar));
+  r[kRecParity] = (int)parity;
+  r[kRecNs] = (int)(ns & 0xffffffffll);
+  r[kRecNs + 1] = (int)(ns >> 32);
+  r[kRecSm] = sm_id();
+  __threadfence();
 }
 
 // ------------------------------------------------------------------ mbarrier
@@ -161,20 +213,25 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Bounded: gives up
-// after `limit` cycles (kWaitCycles by default) or when another warp of the CTA
-// has given up, returning false.  Every thread that calls it must act on a
-// false return.
+// after `limit_ns` nanoseconds of global time (kWaitNs by default) or when
+// another warp of the CTA has given up, returning false.  Every thread that
+// calls it must act on a false return.  The clock is read every 64 probes
+// only, the first reading starting the count.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const CtaAbort& ab,
-                                          long long limit = kWaitCycles) {
+                                          long long limit_ns = kWaitNs) {
   if (mbar_test_wait(bar, parity)) return true;  // already complete: no suspension
   if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
+  long long g0 = 0;
   uint32_t n = 0;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((++n & 63u) == 0) {
       if (aborted(ab)) return false;
-      if (clock64() - t0 > limit) {
+      const long long g1 = global_ns();
+      if (n == 64) {
+        g0 = g1;
+      } else if (g1 - g0 > limit_ns) {
+        record_timeout(ab, bar, parity, g1 - g0);
         raise_abort(ab);
         return false;
       }
@@ -182,11 +239,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
-// Short bounded wait used only while draining on the abort path.
+// Short bounded wait (kWaitNs / 4) used only while draining on the abort path.
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
-  const long long t0 = clock64();
+  const long long t0 = global_ns();
+  uint32_t n = 0;
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > (kWaitCycles >> 2)) return;
+    if ((++n & 63u) == 0 && global_ns() - t0 > (kWaitNs >> 2)) return;
   }
 }
 
