@@ -3,7 +3,8 @@
 * the shared library loads and exports every function include/vdnattn.h declares;
 * argument validation returns the documented status codes before any CUDA call;
 * the host membership table equals the oracle's, bit for bit, on the workload
-  shapes and on edge cases (one to three frames, one chunk, many chunks).
+  shapes and on edge cases (one to three frames, one chunk, many chunks);
+* the binding reads the kernels' timeout record where and as they write it.
 """
 import ctypes
 import os
@@ -193,3 +194,28 @@ EDGE = [(1, 1), (2, 1), (2, 2), (3, 1), (3, 3), (4, 2), (5, 1), (6, 3), (15, 1),
 def test_host_membership_matches_oracle(F, C):
     np.testing.assert_array_equal(vb.plan_membership(F, C), O.membership_table(F, C))
     np.testing.assert_array_equal(vb.plan_membership(F, C, vb.ANCHOR_GLOBAL), O.membership_table(F, C, "global"))
+
+
+def test_timeout_record_reader_matches_the_kernels_layout():
+    """binding.timeout_record reads the words the kernels write (the kRec*
+    indices of csrc/sm100.cuh, at byte 64 of the workspace as api.cu places
+    them), and clear_timeout_record zeroes them."""
+    import torch
+    csrc = os.path.join(ROOT, "video_diffusion_hybrid_sparse_b200", "csrc")
+    idx = {m.group(1): int(m.group(2))
+           for m in re.finditer(r"\bkRec(\w+) = (\d+)", open(os.path.join(csrc, "sm100.cuh")).read())}
+    assert re.search(r"ws\(cfg, g\.off_status\) \+ 64\)", open(os.path.join(csrc, "api.cu")).read())
+    assert idx["Words"] * 4 <= 256 - 64  # inside the 256-byte status slot
+    ws = torch.zeros(256, dtype=torch.uint8)
+    words = ws[64:128].view(torch.int32)
+    ns = 3 * 2**32 + 123456789
+    vals = {"Timeouts": 2, "Kernel": 4, "Block": 77, "Warp": 1, "BarOff": 92, "Parity": 1, "Sm": 140}
+    for k, v in vals.items():
+        words[idx[k]] = v
+    words[idx["Ns"]] = ns & 0xFFFFFFFF if ns & 0x80000000 == 0 else (ns & 0xFFFFFFFF) - 2**32
+    words[idx["Ns"] + 1] = ns >> 32
+    rec = vb.timeout_record(ws)
+    assert rec == {"timeouts": 2, "kernel": 4, "block": 77, "warp": 1, "bar_off": 92, "parity": 1, "ns": ns,
+                   "sm": 140}
+    vb.clear_timeout_record(ws)
+    assert int(ws[64:128].sum()) == 0 and vb.timeout_record(ws)["timeouts"] == 0
