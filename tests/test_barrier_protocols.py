@@ -1,46 +1,72 @@
-"""Model check of the kernels' mbarrier protocols (host only, no GPU).
+"""Model check of the kernels' mbarrier protocols and buffer use (host only).
 
 Each role of a kernel (the TMA producer thread, the MMA thread, the groups of
-worker warps) is written out as the straight-line sequence of barrier
-operations its code performs for a given schedule of work, and every
-interleaving of the roles and of the asynchronous completions (TMA loads in
-any order, tcgen05.commit arrivals in issue order) is explored.  Barriers
-follow mbarrier semantics: a phase completes when its arrivals are in (a
-group of threads that arrives together counts as one arrival here, as does a
-TMA transaction), and a wait on parity P passes while the barrier's current
-phase has the other parity.  Two properties are checked in every reachable
-state:
+worker warps) is written out as the straight-line sequence of what its code
+does for a given schedule of work: barrier waits and arrivals, TMA loads,
+tcgen05.mma issues with the buffers they read and write, tcgen05.commit, and
+the intervals in which the warps read or write a shared-memory tile or a
+TMEM region.  Every interleaving of the roles and of the asynchronous
+completions (TMA loads in any order, commit arrivals in issue order) is
+explored.  Barriers follow mbarrier semantics: a phase completes when its
+arrivals are in (a group of threads that arrives together counts as one
+arrival here, as does a TMA transaction), and a wait on parity P passes
+while the barrier's current phase has the other parity.  A TMA load writes
+its buffer from issue to completion; an MMA reads and writes its operands
+from issue until the first commit issued after it completes (MMAs of one
+thread run in issue order, so they never conflict with one another).  In
+every reachable state the check asserts:
 
 * no deadlock: some role or completion can always move until all roles end;
 * no phase aliasing: a wait for phase p never meets a barrier that has
   completed p + 2 or more phases (it would wait on a later phase, or pass on
-  the wrong one), nor passes before phase p completed.
+  the wrong one), nor passes before phase p completed;
+* no buffer hazard: a read finds the version of the data the code means,
+  with no write to that buffer in progress, and a write overlaps no other
+  role's read or write of it.
 
 The abort paths (a wait that runs out) are not modelled.  The planted old
 protocol of the TMA-fed readout (one phi-ready barrier for both accumulator
-slots) must fail; it is the race that the per-slot barriers fixed.
+slots) must fail; it is the race that the per-slot barriers fixed.  Planted
+buffer mistakes (a loader that refills before the consumer releases, a
+release before the last read) must fail too.
 """
 from collections import namedtuple
 
 import pytest
 
-Op = namedtuple("Op", "kind bar phase")  # kind: wait / arrive / tma / commit
+Op = namedtuple("Op", "kind bar phase reads writes")
 
 
 def wait(bar, phase):
-    return Op("wait", bar, phase)
+    return Op("wait", bar, phase, (), ())
 
 
 def arrive(bar):
-    return Op("arrive", bar, None)
+    return Op("arrive", bar, None, (), ())
 
 
-def tma(bar):
-    return Op("tma", bar, None)
+def tma(bar, *writes):
+    """TMA load(s) completing on `bar`, writing (buffer, version) pairs."""
+    return Op("tma", bar, None, (), tuple(writes))
 
 
 def commit(bar):
-    return Op("commit", bar, None)
+    return Op("commit", bar, None, (), ())
+
+
+def mma(reads=(), writes=()):
+    """tcgen05.mma issues reading / writing (buffer, version) pairs (version
+    None: not checked)."""
+    return Op("mma", None, None, tuple(reads), tuple(writes))
+
+
+def beg(reads=(), writes=()):
+    """This role starts reading / writing the buffers (until `end`)."""
+    return Op("beg", None, None, tuple(reads), tuple(writes))
+
+
+def end(*bufs):
+    return Op("end", None, None, tuple(bufs), ())
 
 
 class ProtocolError(AssertionError):
@@ -49,52 +75,122 @@ class ProtocolError(AssertionError):
 
 def check(roles, max_states=3_000_000):
     """Explore every interleaving of `roles` (name -> list of Op); return the
-    number of states visited; raise ProtocolError on a deadlock or a phase
-    alias, with the trace that reaches it."""
+    number of states visited; raise ProtocolError on a deadlock, a phase
+    alias or a buffer hazard, with the trace that reaches it."""
     names = sorted(roles)
-    progs = [roles[n] for n in names]
-    bars = sorted({op.bar for p in progs for op in p})
+    progs = [list(roles[n]) for n in names]
+    bars = sorted({op.bar for p in progs for op in p if op.bar is not None})
     bid = {b: i for i, b in enumerate(bars)}
-    progs = [[(op.kind, bid[op.bar], op.phase) for op in p] for p in progs]
+    bufs = sorted({acc[0] for p in progs for op in p for acc in op.reads + op.writes}
+                  | {b for p in progs for op in p if op.kind == "end" for b in op.reads})
+    uid = {b: i for i, b in enumerate(bufs)}
 
-    start = (tuple(0 for _ in progs), tuple(0 for _ in bars), (), ())
+    def fail(msg, trace):
+        raise ProtocolError(f"{msg}: {_fmt(trace, names, bars)}")
+
+    # state: pcs, phases, pending TMAs ((bar, writes), ...), open MMA accesses
+    # (since the last commit), commit queue ((bar, accesses), ...), buffer
+    # versions, per-role open sync accesses
+    start = (tuple(0 for _ in progs), tuple(0 for _ in bars), (), (), (), tuple(None for _ in bufs),
+             tuple(() for _ in progs))
     seen = {start}
     stack = [(start, ())]
     while stack:
-        (pcs, ph, tmas, commits), trace = stack.pop()
+        state, trace = stack.pop()
+        pcs, ph, tmas, mopen, commits, ver, sync = state
+
+        def writers(u, me):
+            """Who else is writing buffer u right now (me: role index, 'tma' or 'mma')."""
+            out = [w for _, ws in tmas for (w, _) in ws if w == u]
+            if me != "mma":
+                out += [a for a in mopen if a[0] == "w" and a[1] == u]
+                out += [a for _, accs in commits for a in accs if a[0] == "w" and a[1] == u]
+            out += [a for r, accs in enumerate(sync) if r != me for a in accs if a[0] == "w" and a[1] == u]
+            return out
+
+        def users(u, me):
+            out = writers(u, me)
+            if me != "mma":
+                out += [a for a in mopen if a[1] == u]
+                out += [a for _, accs in commits for a in accs if a[1] == u]
+            out += [a for r, accs in enumerate(sync) if r != me for a in accs if a[1] == u]
+            return out
+
+        def check_access(reads, writes, me, who):
+            for b, v in reads:
+                u = uid[b]
+                if writers(u, me):
+                    fail(f"{who} reads {b} while it is being written", trace)
+                if v is not None and ver[u] != v:
+                    fail(f"{who} reads {b} expecting {v!r}, finds {ver[u]!r}", trace)
+            for b, _ in writes:
+                if users(uid[b], me):
+                    fail(f"{who} writes {b} while another role uses it", trace)
+
         moves = []
         for r, prog in enumerate(progs):
             if pcs[r] == len(prog):
                 continue
-            kind, b, p = prog[pcs[r]]
-            if kind == "wait":
+            op = prog[pcs[r]]
+            npcs = _step(pcs, r)
+            if op.kind == "wait":
+                b, p = bid[op.bar], op.phase
                 k = ph[b]
                 if k >= p + 2:
-                    raise ProtocolError(f"{names[r]} waits for phase {p} of {bars[b]}, which has completed {k} "
-                                        f"phases: {_fmt(trace, names, bars)}")
+                    fail(f"{names[r]} waits for phase {p} of {op.bar}, which has completed {k} phases", trace)
                 if (k & 1) == (p & 1):
                     continue  # blocked
                 if k < p + 1:
-                    raise ProtocolError(f"{names[r]} passes its wait for phase {p} of {bars[b]} after {k} "
-                                        f"phases: {_fmt(trace, names, bars)}")
-                moves.append(((r, None), _step(pcs, r), ph, tmas, commits))
-            elif kind == "arrive":
-                moves.append(((r, None), _step(pcs, r), _bump(ph, b), tmas, commits))
-            elif kind == "tma":
-                moves.append(((r, None), _step(pcs, r), ph, tuple(sorted(tmas + (b,))), commits))
-            else:
-                moves.append(((r, None), _step(pcs, r), ph, tmas, commits + (b,)))
-        for b in set(tmas):  # a TMA load completes: any of them, in any order
-            rest = list(tmas)
-            rest.remove(b)
-            moves.append(((None, b), pcs, _bump(ph, b), tuple(rest), commits))
-        if commits:  # commits complete in issue order
-            moves.append(((None, commits[0]), pcs, _bump(ph, commits[0]), tmas, commits[1:]))
+                    fail(f"{names[r]} passes its wait for phase {p} of {op.bar} after {k} phases", trace)
+                moves.append(((r, None), npcs, ph, tmas, mopen, commits, ver, sync))
+            elif op.kind == "arrive":
+                moves.append(((r, None), npcs, _bump(ph, bid[op.bar]), tmas, mopen, commits, ver, sync))
+            elif op.kind == "tma":
+                for b, _ in op.writes:
+                    if users(uid[b], "tma"):
+                        fail(f"{names[r]} starts a TMA load into {b} while it is in use", trace)
+                ws = tuple((uid[b], v) for b, v in op.writes)
+                moves.append(((r, None), npcs, ph, tuple(sorted(tmas + ((bid[op.bar], ws),))), mopen, commits,
+                              ver, sync))
+            elif op.kind == "mma":
+                check_access(op.reads, op.writes, "mma", names[r])
+                accs = tuple(("r", uid[b], v) for b, v in op.reads) + tuple(("w", uid[b], v) for b, v in op.writes)
+                moves.append(((r, None), npcs, ph, tmas, mopen + accs, commits, ver, sync))
+            elif op.kind == "commit":
+                moves.append(((r, None), npcs, ph, tmas, (), commits + ((bid[op.bar], mopen),), ver, sync))
+            elif op.kind == "beg":
+                check_access(op.reads, op.writes, r, names[r])
+                accs = tuple(("r", uid[b], v) for b, v in op.reads) + tuple(("w", uid[b], v) for b, v in op.writes)
+                nsync = sync[:r] + (sync[r] + accs,) + sync[r + 1:]
+                moves.append(((r, None), npcs, ph, tmas, mopen, commits, ver, nsync))
+            else:  # end: close this role's accesses to the buffers; writes take effect
+                ended = {uid[b] for b in op.reads}
+                nver = list(ver)
+                for kind, u, v in sync[r]:
+                    if u in ended and kind == "w":
+                        nver[u] = v
+                keep = tuple(a for a in sync[r] if a[1] not in ended)
+                nsync = sync[:r] + (keep,) + sync[r + 1:]
+                moves.append(((r, None), npcs, ph, tmas, mopen, commits, tuple(nver), nsync))
+        for i, (b, ws) in enumerate(tmas):  # a TMA load completes: any of them, in any order
+            if i > 0 and tmas[i - 1] == tmas[i]:
+                continue
+            nver = list(ver)
+            for u, v in ws:
+                nver[u] = v
+            moves.append(((None, b), pcs, _bump(ph, b), tmas[:i] + tmas[i + 1:], mopen, commits, tuple(nver), sync))
+        if commits:  # commits complete in issue order; their MMAs' writes take effect
+            b, accs = commits[0]
+            nver = list(ver)
+            for kind, u, v in accs:
+                if kind == "w":
+                    nver[u] = v
+            moves.append(((None, b), pcs, _bump(ph, b), tmas, mopen, commits[1:], tuple(nver), sync))
         if not moves:
             if any(pcs[r] < len(p) for r, p in enumerate(progs)):
-                blocked = [f"{names[r]} at {progs[r][pcs[r]][0]} {bars[progs[r][pcs[r]][1]]} "
-                           f"phase {progs[r][pcs[r]][2]}" for r in range(len(progs)) if pcs[r] < len(progs[r])]
-                raise ProtocolError(f"deadlock ({'; '.join(blocked)}): {_fmt(trace, names, bars)}")
+                blocked = [f"{names[r]} at {progs[r][pcs[r]].kind} {progs[r][pcs[r]].bar} "
+                           f"phase {progs[r][pcs[r]].phase}" for r in range(len(progs)) if pcs[r] < len(progs[r])]
+                fail(f"deadlock ({'; '.join(blocked)})", trace)
             continue
         for who, *nxt in moves:
             st = tuple(nxt)
@@ -124,7 +220,9 @@ def _fmt(trace, names, bars):
 # ------------------------------------------------------------------ k4_merge_tma
 # Roles as in k4_merge_tma.cu: warp 0 (loads), warp 1 (MMA), the eight worker
 # warps (one group).  keys[i] identifies the readout operand (batch, chunk) of
-# the CTA's i-th tile.
+# the CTA's i-th tile.  Buffers: Q (the q tile), G (o_s, g_s, g_l of a tile),
+# B (the operand M_c), Phi0/Phi1 and Acc0/Acc1 (TMEM columns of the two
+# accumulator slots).
 
 
 def k4_tma_roles(keys, per_slot_ready=True):
@@ -138,45 +236,51 @@ def k4_tma_roles(keys, per_slot_ready=True):
             if keys[i] != prev:
                 if b_loads > 0:
                     loads.append(wait("BEmpty", b_loads - 1))
-                loads.append(tma("BFull"))
+                loads.append(tma("BFull", ("B", keys[i])))
                 b_loads += 1
                 prev = keys[i]
             loads.append(wait("AEmpty", i - 1))  # parity (i & 1) ^ 1
-            loads.append(tma("AFull"))
+            loads.append(tma("AFull", ("Q", i)))
         if i >= 1:
             loads.append(wait("GEmpty", i - 2))  # parity ((i - 1) & 1) ^ 1
-            loads.append(tma("GFull"))
+            loads.append(tma("GFull", ("G", i - 1)))
 
-    mma, prev, b_loads = [], None, 0
+    mma_, prev, b_loads = [], None, 0
     for i in range(n):
         s = i & 1
         if keys[i] != prev:
             b_loads += 1
             prev = keys[i]
-            mma.append(wait("BFull", b_loads - 1))
-        mma.append(wait(ready(i), ready_phase(i)))
-        mma.append(wait(f"AccEmpty{s}", (i >> 1) - 1))  # parity ((i >> 1) & 1) ^ 1
-        mma.append(commit(f"AccFull{s}"))
+            mma_.append(wait("BFull", b_loads - 1))
+        mma_.append(wait(ready(i), ready_phase(i)))
+        mma_.append(wait(f"AccEmpty{s}", (i >> 1) - 1))  # parity ((i >> 1) & 1) ^ 1
+        mma_.append(mma(reads=[("B", keys[i]), (f"Phi{s}", i)], writes=[(f"Acc{s}", i)]))
+        mma_.append(commit(f"AccFull{s}"))
         if i + 1 >= n or keys[i + 1] != keys[i]:
-            mma.append(commit("BEmpty"))
-    mma += [commit("Done"), wait("Done", 0)]
+            mma_.append(commit("BEmpty"))
+    mma_ += [commit("Done"), wait("Done", 0)]
 
     workers = []
 
     def finish(j):
-        workers.extend([wait(f"AccFull{j & 1}", j >> 1), arrive(f"AccEmpty{j & 1}"), wait("GFull", j),
+        s = j & 1
+        workers.extend([wait(f"AccFull{s}", j >> 1), beg(reads=[(f"Acc{s}", j)]), end(f"Acc{s}"),
+                        arrive(f"AccEmpty{s}"), wait("GFull", j), beg(reads=[("G", j)]), end("G"),
                         arrive("GEmpty")])
 
     for i in range(n):
-        workers += [wait("AFull", i), arrive("AEmpty"), arrive(ready(i))]
+        s = i & 1
+        workers += [wait("AFull", i), beg(reads=[("Q", i)]), end("Q"), arrive("AEmpty"),
+                    beg(writes=[(f"Phi{s}", i)]), end(f"Phi{s}"), arrive(ready(i))]
         if i > 0:
             finish(i - 1)
     if n > 0:
         finish(n - 1)
-    return {"loads": loads, "mma": mma, "workers": workers}
+    return {"loads": loads, "mma": mma_, "workers": workers}
 
 
 # ------------------------------------------------------------------ k4_readout_merge
+# Buffers: A0/A1 (the double-buffered q tile, phi applied in place), B, Acc0/Acc1.
 
 
 def k4_general_roles(keys):
@@ -187,57 +291,70 @@ def k4_general_roles(keys):
         if keys[i] != prev:
             if b_loads > 0:
                 loads.append(wait("BEmpty", b_loads - 1))
-            loads.append(tma("BFull"))
+            loads.append(tma("BFull", ("B", keys[i])))
             b_loads += 1
             prev = keys[i]
-        loads += [wait(f"AEmpty{s}", (i >> 1) - 1), tma(f"AFull{s}")]
+        loads += [wait(f"AEmpty{s}", (i >> 1) - 1), tma(f"AFull{s}", (f"A{s}", i))]
 
-    mma, prev, b_loads = [], None, 0
+    mma_, prev, b_loads = [], None, 0
     for i in range(n):
         s = i & 1
         if keys[i] != prev:
             b_loads += 1
             prev = keys[i]
-            mma.append(wait("BFull", b_loads - 1))
-        mma += [wait(f"AReady{s}", i >> 1), wait(f"AccEmpty{s}", (i >> 1) - 1), commit(f"AccFull{s}"),
-                commit(f"AEmpty{s}")]
+            mma_.append(wait("BFull", b_loads - 1))
+        mma_ += [wait(f"AReady{s}", i >> 1), wait(f"AccEmpty{s}", (i >> 1) - 1),
+                 mma(reads=[("B", keys[i]), (f"A{s}", ("phi", i))], writes=[(f"Acc{s}", i)]),
+                 commit(f"AccFull{s}"), commit(f"AEmpty{s}")]
         if i + 1 >= n or keys[i + 1] != keys[i]:
-            mma.append(commit("BEmpty"))
-    mma += [commit("Done"), wait("Done", 0)]
+            mma_.append(commit("BEmpty"))
+    mma_ += [commit("Done"), wait("Done", 0)]
 
     workers = []
 
     def finish(j):
-        workers.extend([wait(f"AccFull{j & 1}", j >> 1), arrive(f"AccEmpty{j & 1}")])
+        s = j & 1
+        workers.extend([wait(f"AccFull{s}", j >> 1), beg(reads=[(f"Acc{s}", j)]), end(f"Acc{s}"),
+                        arrive(f"AccEmpty{s}")])
 
     for i in range(n):
-        workers += [wait(f"AFull{i & 1}", i >> 1), arrive(f"AReady{i & 1}")]
+        s = i & 1
+        workers += [wait(f"AFull{s}", i >> 1), beg(reads=[(f"A{s}", i)], writes=[(f"A{s}", ("phi", i))]),
+                    end(f"A{s}"), arrive(f"AReady{s}")]
         if i > 0:
             finish(i - 1)
     if n > 0:
         finish(n - 1)
-    return {"loads": loads, "mma": mma, "workers": workers}
+    return {"loads": loads, "mma": mma_, "workers": workers}
 
 
 # ------------------------------------------------------------------ k1_state_build
+# Buffers: Stage0..2 (the K and V tiles of a stage; phi is applied to K in
+# place), Acc (the TMEM accumulator of the slice).
 
 
 def k1_roles(ntiles, stages=3):
-    loads, mma, phi = [], [], []
+    loads, mma_, phi = [], [], []
     for i in range(ntiles):
         st, r = i % stages, i // stages
-        loads += [wait(f"Empty{st}", r - 1), tma(f"Full{st}")]
-        mma += [wait(f"Phi{st}", r), commit(f"Empty{st}")]
-        phi += [wait(f"Full{st}", r), arrive(f"Phi{st}")]
-    mma.append(commit("Acc"))
-    phi.append(wait("Acc", 0))
-    return {"loads": loads, "mma": mma, "phi": phi}
+        loads += [wait(f"Empty{st}", r - 1), tma(f"Full{st}", (f"Stage{st}", i))]
+        mma_ += [wait(f"Phi{st}", r), mma(reads=[(f"Stage{st}", ("phi", i))], writes=[("Acc", i)]),
+                 commit(f"Empty{st}")]
+        phi += [wait(f"Full{st}", r), beg(reads=[(f"Stage{st}", i)], writes=[(f"Stage{st}", ("phi", i))]),
+                end(f"Stage{st}"), arrive(f"Phi{st}")]
+    mma_.append(commit("Acc"))
+    phi += [wait("Acc", 0), beg(reads=[("Acc", ntiles - 1)]), end("Acc")]
+    return {"loads": loads, "mma": mma_, "phi": phi}
 
 
 # ------------------------------------------------------------------ k3_sparse_softmax / k3_fp8
 # items: (query tiles of the item, KV tiles of its key set) in the CTA's order.
 # P is handed to the MMA thread in one part (the kernels' default).  The fp8
 # kernel performs the same barrier operations (checked below on the sources).
+# Buffers: Q (the item's query tiles), K0/K1 and V0/V1 (the stages), SP0/SP1
+# (TMEM of S, with P written over it, per query tile), O0/O1 (TMEM output
+# accumulators; the softmax warps may rescale them in place before handing
+# over P, modelled at every step).
 
 
 def k3_roles(items, stages=2):
@@ -245,49 +362,61 @@ def k3_roles(items, stages=2):
     for n_item, (_, nkv) in enumerate(items):
         if n_item > 0:
             loads.append(wait("QEmpty", n_item - 1))
-        loads.append(tma("QFull"))
+        loads.append(tma("QFull", ("Q", n_item)))
         for _ in range(nkv):
             st, r = kv % stages, kv // stages
-            loads += [wait(f"KEmpty{st}", r - 1), tma(f"KFull{st}"), wait(f"VEmpty{st}", r - 1),
-                      tma(f"VFull{st}")]
+            loads += [wait(f"KEmpty{st}", r - 1), tma(f"KFull{st}", (f"K{st}", kv)), wait(f"VEmpty{st}", r - 1),
+                      tma(f"VFull{st}", (f"V{st}", kv))]
             kv += 1
 
-    mma, kv, p_cnt = [], 0, [0, 0]
+    mma_, kv, p_cnt, s_idx = [], 0, [0, 0], [0, 0]
+
+    def issue_s(t, n_item, st, kv_):
+        mma_.append(mma(reads=[("Q", n_item), (f"K{st}", kv_)], writes=[(f"SP{t}", ("S", s_idx[t]))]))
+        s_idx[t] += 1
+
     for n_item, (nt, nkv) in enumerate(items):
-        mma.append(wait("QFull", n_item))
+        mma_.append(wait("QFull", n_item))
         st = kv % stages
-        mma.append(wait(f"KFull{st}", kv // stages))
-        mma += [commit(f"SFull{t}") for t in range(nt)]
-        mma.append(commit(f"KEmpty{st}"))
+        mma_.append(wait(f"KFull{st}", kv // stages))
+        for t in range(nt):
+            issue_s(t, n_item, st, kv)
+            mma_.append(commit(f"SFull{t}"))
+        mma_.append(commit(f"KEmpty{st}"))
         for j in range(nkv):
             st, nst, has_next = kv % stages, (kv + 1) % stages, j + 1 < nkv
-            mma.append(wait(f"VFull{st}", kv // stages))
+            mma_.append(wait(f"VFull{st}", kv // stages))
             for t in range(nt):
-                mma.append(wait(f"PFull{t}", p_cnt[t]))
+                mma_.append(wait(f"PFull{t}", p_cnt[t]))
+                mma_.append(mma(reads=[(f"SP{t}", ("P", p_cnt[t])), (f"V{st}", kv)],
+                                writes=[(f"O{t}", ("O", n_item, j))]))
                 p_cnt[t] += 1
                 if not has_next:
-                    mma.append(commit(f"OFull{t}"))
+                    mma_.append(commit(f"OFull{t}"))
                 else:
                     if t == 0:
-                        mma.append(wait(f"KFull{nst}", (kv + 1) // stages))
-                    mma.append(commit(f"SFull{t}"))
-            mma.append(commit(f"VEmpty{st}"))
+                        mma_.append(wait(f"KFull{nst}", (kv + 1) // stages))
+                    issue_s(t, n_item, nst, kv + 1)
+                    mma_.append(commit(f"SFull{t}"))
+            mma_.append(commit(f"VEmpty{st}"))
             if has_next:
-                mma.append(commit(f"KEmpty{nst}"))
+                mma_.append(commit(f"KEmpty{nst}"))
             kv += 1
-        mma.append(commit("QEmpty"))
-    mma += [commit("Done"), wait("Done", 0)]
+        mma_.append(commit("QEmpty"))
+    mma_ += [commit("Done"), wait("Done", 0)]
 
-    roles = {"loads": loads, "mma": mma}
+    roles = {"loads": loads, "mma": mma_}
     for t in range(2):
         sm, s_cnt, o_cnt = [], 0, 0
-        for nt, nkv in items:
+        for n_item, (nt, nkv) in enumerate(items):
             if t >= nt:
                 continue
-            for _ in range(nkv):
-                sm += [wait(f"SFull{t}", s_cnt), arrive(f"PFull{t}")]
+            for j in range(nkv):
+                sm += [wait(f"SFull{t}", s_cnt), beg(reads=[(f"SP{t}", ("S", s_cnt))]), end(f"SP{t}"),
+                       beg(writes=[(f"O{t}", ("scaled", n_item, j))]), end(f"O{t}"),
+                       beg(writes=[(f"SP{t}", ("P", s_cnt))]), end(f"SP{t}"), arrive(f"PFull{t}")]
                 s_cnt += 1
-            sm.append(wait(f"OFull{t}", o_cnt))
+            sm += [wait(f"OFull{t}", o_cnt), beg(reads=[(f"O{t}", ("O", n_item, nkv - 1))]), end(f"O{t}")]
             o_cnt += 1
         roles[f"softmax{t}"] = sm
     return roles
@@ -355,3 +484,92 @@ def test_fp8_softmax_has_the_bf16_barrier_operations():
 
     assert ops("k3_sparse_softmax.cu") == ops("k3_fp8.cu") and len(ops("k3_fp8.cu")) > 10
     assert re.search(r"#define VDN_P_PARTS 1\b", open(os.path.join(csrc, "k3_sparse_softmax.cu")).read())
+
+
+def _drop(roles, role, pred):
+    out = dict(roles)
+    out[role] = [op for op in roles[role] if not pred(op)]
+    return out
+
+
+def _move_before(roles, role, pred_move, pred_anchor):
+    """Move every op matching pred_move to just before the preceding op that
+    matches pred_anchor."""
+    ops = list(roles[role])
+    i = 0
+    while i < len(ops):
+        if pred_move(ops[i]):
+            j = i - 1
+            while j >= 0 and not pred_anchor(ops[j]):
+                j -= 1
+            if j >= 0:
+                op = ops.pop(i)
+                ops.insert(j, op)
+        i += 1
+    out = dict(roles)
+    out[role] = ops
+    return out
+
+
+def _move_o_rescale_before_s_wait(roles):
+    ops = list(roles["softmax0"])
+    out, i = [], 0
+    while i < len(ops):
+        op = ops[i]
+        if op.kind == "wait" and op.bar == "SFull0":
+            # ops i+1..i+2 read S; ops i+3..i+4 rescale O: put the rescale first
+            out += ops[i + 3:i + 5] + [op] + ops[i + 1:i + 3]
+            i += 5
+        else:
+            out.append(op)
+            i += 1
+    roles = dict(roles)
+    roles["softmax0"] = out
+    return roles
+
+
+PLANTED = {
+    # the loader refills the q tile without waiting for the workers to release it
+    "readout_loader_skips_q_release": lambda: _drop(k4_tma_roles([0, 0, 1, 1]), "loads",
+                                                    lambda op: op.kind == "wait" and op.bar == "AEmpty"),
+    # the workers release the q tile before reading it
+    "readout_release_before_read": lambda: _move_before(
+        k4_tma_roles([0, 0, 1, 1]), "workers", lambda op: op.kind == "arrive" and op.bar == "AEmpty",
+        lambda op: op.kind == "beg" and op.reads and op.reads[0][0] == "Q"),
+    # the loader reloads o_s and the gates without waiting for the merge to finish
+    "readout_loader_skips_g_release": lambda: _drop(k4_tma_roles([0, 0, 1, 1]), "loads",
+                                                    lambda op: op.kind == "wait" and op.bar == "GEmpty"),
+    # the MMA thread reads the readout operand before its load landed
+    "readout_mma_skips_operand_load": lambda: _drop(k4_tma_roles([0, 0, 1, 1]), "mma",
+                                                    lambda op: op.kind == "wait" and op.bar == "BFull"),
+    # the general readout's MMA thread does not wait for phi
+    "general_readout_mma_skips_ready": lambda: _drop(k4_general_roles([0, 1, 1]), "mma",
+                                                     lambda op: op.kind == "wait" and op.bar.startswith("AReady")),
+    # the state build's MMA thread does not wait for phi(K)
+    "state_build_mma_skips_phi": lambda: _drop(k1_roles(4), "mma",
+                                               lambda op: op.kind == "wait" and op.bar.startswith("Phi")),
+    # the softmax MMA thread does not wait for P
+    "softmax_mma_skips_p": lambda: _drop(k3_roles([(2, 2)]), "mma",
+                                         lambda op: op.kind == "wait" and op.bar.startswith("PFull")),
+    # the loader refills a K stage before the S MMAs that read it completed
+    "softmax_loader_skips_k_release": lambda: _drop(k3_roles([(1, 3)]), "loads",
+                                                    lambda op: op.kind == "wait" and op.bar.startswith("KEmpty")),
+    # the softmax warps rescale O before the commit after S (which also
+    # covers the previous P.V into O) landed
+    "softmax_rescale_before_s": lambda: _move_o_rescale_before_s_wait(k3_roles([(1, 3)])),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PLANTED))
+def test_planted_protocol_mistake_is_caught(name):
+    with pytest.raises(ProtocolError):
+        check(PLANTED[name]())
+
+
+def test_readout_acc_release_wait_is_implied():
+    """In both readouts the MMA thread's wait for a drained accumulator slot
+    is implied by the phi-ready wait: the workers arrive on a slot's
+    phi-ready barrier for tile i + 2 only after draining tile i.  The model
+    finds no hazard without it (the kernels keep it as a safeguard)."""
+    for roles in (k4_tma_roles([0, 0, 1, 1, 1]), k4_general_roles([0, 0, 1, 1, 1])):
+        assert check(_drop(roles, "mma", lambda op: op.kind == "wait" and op.bar.startswith("AccEmpty"))) > 0
