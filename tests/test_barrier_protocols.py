@@ -573,3 +573,38 @@ def test_readout_acc_release_wait_is_implied():
     finds no hazard without it (the kernels keep it as a safeguard)."""
     for roles in (k4_tma_roles([0, 0, 1, 1, 1]), k4_general_roles([0, 0, 1, 1, 1])):
         assert check(_drop(roles, "mma", lambda op: op.kind == "wait" and op.bar.startswith("AccEmpty"))) > 0
+
+
+# The barrier operations of each kernel source, in source order, as the role
+# programs above model them.  A change to a kernel's barrier use fails here
+# until the model (and this list) is brought up to date.
+SOURCE_BARRIER_OPS = {
+    "k1_state_build.cu": "wait:kEmpty+st expect_tx:kFull+st wait:kAcc wait:kPhi+st mma_commit:kEmpty+st "
+                         "mma_commit:kAcc wait:kFull+st arrive:kPhi+st wait:kAcc",
+    "k3_sparse_softmax.cu": "wait:kQEmpty expect_tx:kQFull wait:kKEmpty+st expect_tx:kKFull+st wait:kVEmpty+st "
+                            "expect_tx:kVFull+st wait:kQFull wait:kKFull+st mma_commit:kSFull+t "
+                            "mma_commit:kKEmpty+st wait:kVFull+st wait:kPFull+2*part+t mma_commit:kOFull+t "
+                            "wait:kKFull+nst mma_commit:kSFull+t mma_commit:kVEmpty+st mma_commit:kKEmpty+nst "
+                            "mma_commit:kQEmpty mma_commit:kDone wait:kSFull+t arrive:kPFull+2*part+t "
+                            "wait:kOFull+t",
+    "k4_merge_tma.cu": "wait:kTBEmpty expect_tx:kTBFull wait:kTAEmpty expect_tx:kTAFull wait:kTGEmpty "
+                       "expect_tx:kTGFull wait:kTBFull wait:kTAReady+s wait:kTAccEmpty+s mma_commit:kTAccFull+s "
+                       "mma_commit:kTBEmpty mma_commit:kTDone wait:kTAccFull+s arrive:kTAccEmpty+s wait:kTGFull "
+                       "arrive:kTGEmpty wait:kTAFull arrive:kTAEmpty arrive:kTAReady+(i&1)",
+    "k4_readout_merge.cu": "wait:kBEmpty expect_tx:kBFull wait:kAEmpty+s expect_tx:kAFull+s wait:kBFull "
+                           "wait:kAReady+s wait:kAccEmpty+s mma_commit:kAccFull+s mma_commit:kAEmpty+s "
+                           "mma_commit:kBEmpty mma_commit:kDone4 wait:kAccFull+s arrive:kAccEmpty+s wait:kAFull+s "
+                           "arrive:kAReady+s",
+}
+
+
+@pytest.mark.parametrize("src", sorted(SOURCE_BARRIER_OPS))
+def test_model_matches_the_kernel_sources(src):
+    import os
+    import re
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                        "video_diffusion_hybrid_sparse_b200", "csrc", src)
+    pat = re.compile(r"(mbar_wait|mma_commit|mbar_arrive|mbar_expect_tx)\(&bars\[([^\]]*)\]")
+    ops = " ".join(f"{m.group(1).replace('mbar_', '')}:{m.group(2).replace(' ', '')}"
+                   for m in pat.finditer(open(path).read()))
+    assert ops == SOURCE_BARRIER_OPS[src]
