@@ -112,10 +112,14 @@ enum {
                                that nothing completes; it gives up, the CTA's other warps follow, the
                                kernel writes VDN_ERR_TIMEOUT to status_word and returns.  The call's
                                outputs are then undefined; the context stays usable. */
-  VDN_STALL_READOUT_MMA = 32 /* test of the readout's barrier protocol only: the readout's MMA thread
+  VDN_STALL_READOUT_MMA = 32, /* test of the readout's barrier protocol only: the readout's MMA thread
                                sleeps 50 microseconds whenever it moves to another readout operand
                                (batch, chunk, head), letting the other warps run as far ahead as the
                                protocol allows.  Outputs are unchanged. */
+  VDN_POISON_WS = 64          /* vdn_hybrid_attn_fwd, _host and _static first fill the workspace past its
+                               256-byte status slot with 0xFF bytes (NaN in bf16 and fp32), so that a
+                               read of scratch the call has not written would show in the output.
+                               Outputs are unchanged. */
 };
 
 typedef struct {
@@ -187,6 +191,15 @@ VDN_API vdn_status vdn_state_build(const void* k, const void* v, const void* tex
                            const void* text_v, const vdn_cfg* cfg, void* stream);
 /* Forward/backward chunk states and their sum M_c, fp32 scan. */
 VDN_API vdn_status vdn_state_scan(const vdn_cfg* cfg, void* stream);
+/* The forward and backward states S_F / z_F and S_B / z_B of every (batch,
+ * chunk, head), as fp32 [B, F/C, H, d+1, d] (row n < d: value column n of S;
+ * row d: z; column a: key feature a), recomputed by the scan on `stream`
+ * from the state partials that the last vdn_hybrid_attn_fwd or
+ * vdn_state_build on cfg->workspace left there; the readout operands are
+ * rewritten with the values they had.  fwd, bwd: device, 16-byte aligned,
+ * B*(F/C)*H*(d+1)*d floats each, caller-owned.  Same as calling
+ * vdn_state_scan with VDN_EXPORT_STATES and cfg->export_fwd/export_bwd set. */
+VDN_API vdn_status vdn_export_states(const vdn_cfg* cfg, float* fwd, float* bwd, void* stream);
 /* Block-sparse softmax branch o_s (window + anchors + text) into the workspace. */
 VDN_API vdn_status vdn_sparse_softmax(const void* q, const void* k, const void* v,
                               const void* text_k, const void* text_v,

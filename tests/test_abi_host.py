@@ -69,9 +69,9 @@ def test_validate_rejects_unknown_dtype_and_flags():
     cfg = vb.make_cfg(shape())
     cfg.dtype = 7
     assert lib.vdn_validate(ctypes.byref(cfg)) == 2
-    cfg = vb.make_cfg(shape(), debug_flags=64)
+    cfg = vb.make_cfg(shape(), debug_flags=128)
     assert lib.vdn_validate(ctypes.byref(cfg)) == 1
-    for flag in (vb.INJECT_TIMEOUT, vb.STALL_READOUT_MMA):
+    for flag in (vb.INJECT_TIMEOUT, vb.STALL_READOUT_MMA, vb.POISON_WS):
         cfg = vb.make_cfg(shape(), debug_flags=flag)
         assert lib.vdn_validate(ctypes.byref(cfg)) == 0
     cfg = vb.make_cfg(shape())
@@ -148,6 +148,9 @@ def test_call_errors_before_any_launch():
     assert lib.vdn_hybrid_attn_fwd(*args, ctypes.byref(cfg), None) == 1
     assert lib.vdn_state_scan(ctypes.byref(cfg), None) == 1
     cfg.debug_flags = 0
+    assert lib.vdn_export_states(ctypes.byref(cfg), None, p, None) == 1  # no buffer
+    assert lib.vdn_export_states(ctypes.byref(cfg), p + 4, p, None) == 3  # misaligned
+    assert lib.vdn_export_states(ctypes.byref(vb.make_cfg(s)), p, p, None) == 4  # no workspace
     assert lib.vdn_plan_membership(ctypes.byref(cfg), None) == 1
     cfg.output_mode = vb.OUTPUT_SPLIT  # SPLIT without its second output buffer
     assert lib.vdn_hybrid_attn_fwd(*args, ctypes.byref(cfg), None) == 1

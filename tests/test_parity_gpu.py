@@ -424,3 +424,41 @@ def test_fp8_768p_sampled_rows():
                                  prob, 0, 0, rows)
         got = out[0, torch.from_numpy(rows).cuda(), h, :].float().cpu().numpy()
         assert_close(got, ref["out"], f"768p fp8 head {h}", abs_tol=4e-2, rel_tol=1e-2)
+
+
+# ----------------------------------------------------------------- workspace poison, state export after a call
+#
+# VDN_POISON_WS fills the workspace past its status slot with 0xFF (NaN in
+# bf16 and fp32) before the call: an output that differs from an unpoisoned
+# call on the same workspace would mean that some kernel read scratch the call
+# had not written.
+
+
+@pytest.mark.parametrize("w,prec", [(SMALL[0], vb.PREC_BF16), (SMALL[2], vb.PREC_BF16), (SMALL[3], vb.PREC_BF16),
+                                    (FP8_CASES[0], vb.PREC_FP8), (FP8_CASES[2], vb.PREC_FP8)],
+                         ids=["tiny_fp32", "ragged_b2", "c5_ragged", "fp8_rms", "fp8_b2_no_text"])
+def test_poisoned_workspace_changes_nothing(w, prec):
+    dev = to_dev(make_inputs(w))
+    ws = vb.workspace_for(vb.shape_of(dev["q"], dev["text_k"], w.F, w.C), dev["q"].device, prec)
+    st0 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ref = run(w, dev, status=st0, workspace=ws, softmax_precision=prec)
+    st1 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = run(w, dev, status=st1, workspace=ws, softmax_precision=prec, debug_flags=vb.POISON_WS)
+    assert int(st0.item()) == 0 and int(st1.item()) == 0
+    word = torch.int32 if out.dtype == torch.float32 else torch.int16
+    assert torch.equal(ref.view(word), out.view(word))
+
+
+@pytest.mark.parametrize("w", [SMALL[0], SMALL[3]], ids=["tiny", "c5_ragged"])
+def test_export_states_after_a_call_equals_export_during_it(w):
+    dev = to_dev(make_inputs(w))
+    ws = vb.workspace_for(vb.shape_of(dev["q"], dev["text_k"], w.F, w.C), dev["q"].device)
+    nc = w.F // w.C
+    fwd = torch.zeros((w.B, nc, w.H, w.d + 1, w.d), dtype=torch.float32, device="cuda")
+    bwd = torch.zeros_like(fwd)
+    run(w, dev, workspace=ws, debug_flags=vb.EXPORT_STATES, export=(fwd, bwd))
+    run(w, dev, workspace=ws)
+    fwd2, bwd2 = torch.full_like(fwd, float("nan")), torch.full_like(bwd, float("nan"))
+    vb.export_states(vb.shape_of(dev["q"], dev["text_k"], w.F, w.C), ws, fwd2, bwd2)
+    torch.cuda.synchronize()
+    assert torch.equal(fwd, fwd2) and torch.equal(bwd, bwd2)

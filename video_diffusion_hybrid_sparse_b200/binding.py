@@ -19,14 +19,14 @@ _lib = None
 
 VDN_BF16, VDN_FP32 = 0, 1
 OUT_SOFTMAX_ONLY, OUT_LINEAR_ONLY, OUT_LINEAR_RAW, EXPORT_STATES, INJECT_TIMEOUT = 1, 2, 4, 8, 16
-STALL_READOUT_MMA = 32
+STALL_READOUT_MMA, POISON_WS = 32, 64
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "pointer not aligned",
           4: "workspace missing or too small", 5: "CUDA error", 6: "device wait timed out"}
 
 EXPORTED = ["vdn_version", "vdn_status_string", "vdn_validate", "vdn_workspace_bytes", "vdn_plan_membership",
             "vdn_membership_device", "vdn_hybrid_attn_fwd", "vdn_stage_inputs", "vdn_state_build",
             "vdn_state_scan", "vdn_sparse_softmax", "vdn_readout_merge", "vdn_hybrid_attn_fwd_static",
-            "vdn_static_scratch_bytes", "vdn_host_staging_bytes", "vdn_hybrid_attn_fwd_host"]
+            "vdn_static_scratch_bytes", "vdn_host_staging_bytes", "vdn_hybrid_attn_fwd_host", "vdn_export_states"]
 
 
 class VdnError(RuntimeError):
@@ -73,6 +73,7 @@ def library() -> ctypes.CDLL:
         lib.vdn_stage_inputs.argtypes = [P, P, P, P, P, C, P]
         lib.vdn_state_build.argtypes = [P, P, P, P, C, P]
         lib.vdn_state_scan.argtypes = [C, P]
+        lib.vdn_export_states.argtypes = [C, P, P, P]
         lib.vdn_sparse_softmax.argtypes = [P, P, P, P, P, C, P]
         lib.vdn_readout_merge.argtypes = [P, P, P, P, C, P]
         lib.vdn_hybrid_attn_fwd_static.argtypes = [P, P, P, P, P, P, P, P, C, P]
@@ -204,6 +205,15 @@ def hybrid_attn_fwd(q, k, v, text_k, text_v, gate_s, gate_l, *, frames: int, chu
                                          ctypes.byref(cfg), _stream(stream))
     _check(code, "vdn_hybrid_attn_fwd")
     return out
+
+
+def export_states(s: Shape, workspace: torch.Tensor, fwd: torch.Tensor, bwd: torch.Tensor, *, stream=None,
+                  softmax_precision: int = PREC_BF16) -> None:
+    """S_F / z_F and S_B / z_B ([B, F/C, H, d+1, d] fp32 each) recomputed from
+    the state partials that the last call on `workspace` left there."""
+    cfg = make_cfg(s, workspace=workspace, softmax_precision=softmax_precision)
+    _check(library().vdn_export_states(ctypes.byref(cfg), fwd.data_ptr(), bwd.data_ptr(), _stream(stream)),
+           "vdn_export_states")
 
 
 _STAGING: dict = {}

@@ -41,7 +41,7 @@ vdn_status make_geom(const vdn_cfg* cfg, Geom& g) {
   if (cfg->dtype != VDN_BF16 && cfg->dtype != VDN_FP32) return VDN_ERR_UNSUPPORTED;
   if (cfg->debug_flags &
       ~(VDN_OUT_SOFTMAX_ONLY | VDN_OUT_LINEAR_ONLY | VDN_OUT_LINEAR_RAW | VDN_EXPORT_STATES | VDN_INJECT_TIMEOUT |
-        VDN_STALL_READOUT_MMA))
+        VDN_STALL_READOUT_MMA | VDN_POISON_WS))
     return VDN_ERR_INVALID_ARG;
   const int Nc = cfg->frames / cfg->chunk_frames;
   if (Nc > kMaxScanChunks) return VDN_ERR_UNSUPPORTED;
@@ -125,6 +125,12 @@ uint8_t* ws(const vdn_cfg* cfg, size_t off) { return static_cast<uint8_t*>(cfg->
 
 int* status_ptr(const vdn_cfg* cfg, const Geom& g) {
   return cfg->status_word ? cfg->status_word : reinterpret_cast<int*>(ws(cfg, g.off_status));
+}
+
+// VDN_POISON_WS: 0xFF over the workspace past the 256-byte status slot.
+cudaError_t poison_ws(const vdn_cfg* cfg, const Geom& g, cudaStream_t st) {
+  if (!(cfg->debug_flags & VDN_POISON_WS) || g.total <= 256) return cudaSuccess;
+  return cudaMemsetAsync(ws(cfg, 256), 0xFF, g.total - 256, st);
 }
 
 // Timeout record of the kernels' bounded waits: 16 int words at byte 64 of
@@ -480,6 +486,16 @@ vdn_status vdn_state_scan(const vdn_cfg* cfg, void* stream) {
   return step_state_scan(cfg, g, static_cast<cudaStream_t>(stream));
 }
 
+vdn_status vdn_export_states(const vdn_cfg* cfg, float* fwd, float* bwd, void* stream) {
+  if (!cfg || !fwd || !bwd) return VDN_ERR_INVALID_ARG;
+  if (((reinterpret_cast<uintptr_t>(fwd) | reinterpret_cast<uintptr_t>(bwd)) & 15u) != 0) return VDN_ERR_ALIGNMENT;
+  vdn_cfg c = *cfg;
+  c.debug_flags |= VDN_EXPORT_STATES;
+  c.export_fwd = fwd;
+  c.export_bwd = bwd;
+  return vdn_state_scan(&c, stream);
+}
+
 vdn_status vdn_sparse_softmax(const void* q, const void* k, const void* v, const void* text_k, const void* text_v,
                               const vdn_cfg* cfg, void* stream) {
   Geom g;
@@ -513,6 +529,7 @@ vdn_status vdn_hybrid_attn_fwd(const void* q, const void* k, const void* v, cons
   if ((cfg->debug_flags & VDN_EXPORT_STATES) && (!cfg->export_fwd || !cfg->export_bwd)) return VDN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Srcs src = kernel_srcs(cfg, g, q, k, v, text_k, text_v);
+  if (poison_ws(cfg, g, st) != cudaSuccess) return VDN_ERR_CUDA;
   if ((s = step_stage(cfg, g, q, k, v, text_k, text_v, st)) != VDN_OK) return s;
   if ((s = step_state_build(cfg, g, src, st)) != VDN_OK) return s;
   if ((s = step_state_scan(cfg, g, st)) != VDN_OK) return s;
@@ -560,6 +577,7 @@ vdn_status vdn_hybrid_attn_fwd_host(const void* q, const void* k, const void* v,
   };
   // Copies on the copy stream, in the order the kernels need them, so the
   // state build runs while q lands and the softmax branch while the gates land.
+  if (poison_ws(cfg, g, st) != cudaSuccess) return finish(VDN_ERR_CUDA);
   cudaError_t ce = cudaEventRecord(ev[0], st);  // earlier work on st may still read the staging
   if (ce == cudaSuccess) ce = cudaStreamWaitEvent(cs, ev[0], 0);
   if (ce == cudaSuccess && g.T > 0) ce = h2d(h.tk, text_k, txt);
