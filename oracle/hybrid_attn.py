@@ -26,7 +26,7 @@ Source of every step: the VDN-H3 article "VDN-Minimax-H3 ... 11.23 秒生成
 * each branch gets its own input-dependent sigmoid gate; the linear output is
   RMS-normalised before its element-wise gate; the two are summed.
 
-Readings of points the page leaves open (each also listed in the design doc):
+Readings of points the page leaves open:
 chunk size C is a parameter (5 in the chunking sentence, 1 in the frame-7
 example); the window is clipped at the sequence ends; anchor frames as queries
 follow the same rule as every other frame (LOCAL, the default) -- the other
