@@ -438,7 +438,7 @@ def test_checker_finds_a_planted_deadlock_and_alias():
                   "c": [wait("X", 0), arrive("Y"), wait("X", 1)]}) > 0
 
 
-READOUT_KEYS = [[0, 0, 0, 0], [0, 0, 1, 1], [0, 1, 1, 2], [0, 1, 2, 3], [0, 0, 0, 1, 1]]
+READOUT_KEYS = [[0, 0, 0, 0], [0, 0, 1, 1], [0, 1, 1, 2], [0, 1, 2, 3], [0, 0, 0, 1, 1], [0, 0, 1, 1, 2, 2]]
 
 
 @pytest.mark.parametrize("keys", READOUT_KEYS, ids=["".join(map(str, k)) for k in READOUT_KEYS])
@@ -463,7 +463,8 @@ def test_state_build_protocol(ntiles):
     assert check(k1_roles(ntiles)) > 0
 
 
-K3_SCHEDULES = [[(2, 1)], [(2, 3)], [(1, 2)], [(2, 2), (2, 1)], [(2, 1), (1, 2)], [(1, 1), (2, 2), (1, 1)]]
+K3_SCHEDULES = [[(2, 1)], [(2, 3)], [(2, 4)], [(1, 2)], [(2, 2), (2, 1)], [(2, 1), (1, 2)], [(1, 1), (2, 2), (1, 1)],
+                [(2, 3), (1, 2), (2, 1)], [(2, 2), (2, 2), (2, 2)]]
 
 
 @pytest.mark.parametrize("items", K3_SCHEDULES, ids=[str(s) for s in K3_SCHEDULES])
