@@ -295,6 +295,45 @@ def _pins_hold():
             failed.append("pairwise " + mode)
         if not np.array_equal(O.membership_table(prob.F, prob.C, mode), table_from_masks(prob)):
             failed.append("membership " + mode)
+    failed += _epilogue_pins_failed()
+    return failed
+
+
+def _epilogue_pins_failed():
+    """Closed forms of the scale, RMSNorm, sigmoid and merge (pages, sections
+    双分支混合注意力机制 and 自适应门控融合双分支输出): torch's own default SDPA
+    scale; RMS of an RMSNorm output is 1, it is scale-free, gamma multiplies
+    it, and a constant row c with eps e gives c / sqrt(c^2 + e); sigmoid(0) =
+    1/2 and sigmoid(ln 3) = 3/4; gates of +-ln 3 weigh the branches 3/4 and
+    1/4, and saturated gates select one branch."""
+    failed = []
+    prob, x = problem_inputs(6, 3, 1, 8, 2, 2, seed=5)
+    mask = torch.from_numpy(BF.softmax_mask(prob))
+    kt = torch.from_numpy(np.concatenate([x["k"][0], x["text_k"][0]], axis=0).transpose(1, 0, 2).copy())
+    vt = torch.from_numpy(np.concatenate([x["v"][0], x["text_v"][0]], axis=0).transpose(1, 0, 2).copy())
+    qt = torch.from_numpy(np.asarray(x["q"][0]).transpose(1, 0, 2).copy())
+    sdpa = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask).numpy().transpose(1, 0, 2)
+    if not np.allclose(O.softmax_branch(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], prob)[0], sdpa,
+                       rtol=1e-10, atol=1e-10):
+        failed.append("default scale")
+    rng = np.random.default_rng(5)
+    v = rng.normal(size=(6, 16))
+    gam = rng.uniform(0.5, 1.5, 16)
+    r = O.rms_norm(v, 0.0)
+    if not np.allclose(np.mean(r * r, axis=-1), 1.0):
+        failed.append("rms unit")
+    if not np.allclose(O.rms_norm(3.0 * v, 0.0), r) or not np.allclose(O.rms_norm(v, 0.0, gam), r * gam):
+        failed.append("rms scale / gamma")
+    if not np.allclose(O.rms_norm(np.ones((2, 16)), 3.0), 0.5):
+        failed.append("rms eps")
+    if not (np.isclose(O.sigmoid(0.0), 0.5) and np.isclose(O.sigmoid(np.log(3.0)), 0.75)):
+        failed.append("sigmoid")
+    o_s, o_r = rng.normal(size=(4, 8)), rng.normal(size=(4, 8))
+    g = np.full((4, 8), np.log(3.0))
+    if not np.allclose(O.merge(o_s, o_r, g, -g), 0.75 * o_s + 0.25 * o_r):
+        failed.append("merge weights")
+    if not np.allclose(O.merge(o_s, o_r, g * 0 + 60, g * 0 - 60), o_s):
+        failed.append("merge saturation")
     return failed
 
 
@@ -319,6 +358,16 @@ MUTATIONS = {
     "phi_plain_exp": ("phi", lambda x: np.exp(np.asarray(x, np.float64))),
     "softmax_frames_drop_last_anchor": ("softmax_frames",
                                         lambda f, F, C, mode="local": sorted(set(O.window_frames(f, F, C)) | {0})),
+    "rms_eps_outside_sqrt": ("rms_norm", lambda x, eps, gamma=None: (lambda x: x / (np.sqrt(
+        np.mean(x * x, axis=-1, keepdims=True)) + eps) * (1.0 if gamma is None else gamma))(np.asarray(x, float))),
+    "rms_sum_not_mean": ("rms_norm", lambda x, eps, gamma=None: (lambda x: x / np.sqrt(
+        np.sum(x * x, axis=-1, keepdims=True) + eps) * (1.0 if gamma is None else gamma))(np.asarray(x, float))),
+    "rms_gamma_ignored": ("rms_norm", lambda x, eps, gamma=None: (lambda x: x / np.sqrt(
+        np.mean(x * x, axis=-1, keepdims=True) + eps))(np.asarray(x, float))),
+    "sigmoid_sign": ("sigmoid", lambda x: 1.0 / (1.0 + np.exp(np.asarray(x, float)))),
+    "gates_swapped": ("merge", lambda o_s, r, g_s, g_l: O.sigmoid(g_l) * o_s + O.sigmoid(g_s) * r),
+    "forward_state_off_by_one": ("forward_frames", lambda f, F, C, mode="local": [
+        g for g in range(F) if g // C <= f // C - 1 and g not in O.anchor_frames(F)]),
 }
 
 
@@ -330,6 +379,15 @@ def test_planted_mistake_is_caught(name, monkeypatch):
     assert _pins_hold() == []
     monkeypatch.setattr(O, fn_name, bad)
     assert _pins_hold() != [], f"planted mistake {name} went unnoticed"
+
+
+def test_planted_wrong_default_scale_is_caught(monkeypatch):
+    """A default softmax scale of 1/d instead of 1/sqrt(d) fails the pin
+    against torch's own default SDPA scale."""
+    assert _pins_hold() == []
+    monkeypatch.setattr(O.Problem, "softmax_scale",
+                        property(lambda self: 1.0 / self.d if self.scale is None else float(self.scale)))
+    assert "default scale" in _pins_hold()
 
 
 # ---------------------------------------------------------------- GLOBAL anchor queries, SPLIT output
