@@ -14,8 +14,9 @@ independent replica of the same workload (no data-path collective) and the
 timing is the max over ranks.
 
 ``--impl reference`` times the fp64 CPU oracle (the method's definition) on
-the host cores, on a bounded sample of the same workload, scaled to the
-metric's unit.
+the host cores: each step is one pass over a bounded sample of one call of the
+same workload (the whole call for the small workloads), and the value is the
+sample's algorithmic FLOPs over its measured time.
 """
 from __future__ import annotations
 
@@ -80,28 +81,65 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    """SM clock and clock-event reasons sampled every 10 ms while the timed
+    region runs (NVML, read-only queries), so that a region of a few hundred
+    milliseconds still yields dozens of samples.  Falls back to nvidia-smi at
+    its 200-ms floor when NVML cannot be loaded."""
 
-    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
-              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
-              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
+    SMI_FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+                  "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+                  "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
 
-    def __init__(self, gpu_id: str):
-        self.gpu_id = gpu_id
-        self.proc = None
+    def __init__(self, gpu_id: str, period_s: float = 0.01):
+        self.gpu_id, self.period = gpu_id, period_s
+        self.samples, self.max_mhz, self.source = [], None, None
+        self.proc = self.thread = None
+
+    def _nvml_handle(self):
+        import pynvml
+
+        pynvml.nvmlInit()
+        if self.gpu_id.isdigit():
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(int(self.gpu_id))
+        return pynvml, pynvml.nvmlDeviceGetHandleByUUID(self.gpu_id)
 
     def __enter__(self):
+        import threading
+
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            nv, h = self._nvml_handle()
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.stop = threading.Event()
+
+            def loop():
+                while not self.stop.is_set():
+                    try:
+                        self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)), int(get_reasons(h))))
+                    except Exception:  # noqa: BLE001 - a failed read only loses a sample
+                        pass
+                    self.stop.wait(self.period)
+
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            self.source = "nvml, 10 ms"
+        except Exception:  # noqa: BLE001 - NVML missing: nvidia-smi instead
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.SMI_FIELDS),
+                     "--format=csv,noheader,nounits", "-lms", "200"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.source = "nvidia-smi, 200 ms"
+            except OSError:
+                self.proc = None
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -109,25 +147,25 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            for ln in out.splitlines():
+                f = [x.strip() for x in ln.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    mhz, self.max_mhz = float(f[1]), float(f[2])
+                except ValueError:
+                    continue
+                mask = 0
+                for (_, bit), val in zip(self.REASONS.items(), f[5:9]):
+                    if val.lower().startswith("active"):
+                        mask |= bit
+                self.samples.append((mhz, mask))
 
     def summary(self):
-        sms, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sms.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for nm, val in zip(names, f[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sms)}
+        sms = [m for m, _ in self.samples]
+        reasons = sorted({nm for _, mask in self.samples for nm, bit in self.REASONS.items() if mask & bit})
+        return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(sms), "sampler": self.source}
 
 
 def gpu_id_for(local_rank: int) -> str:
@@ -169,43 +207,82 @@ def recorded_traffic(kernel: str, workload: str):
 
 # ---------------------------------------------------------------- CPU baseline (oracle)
 
+# Workloads small enough for the whole oracle call to be the sample (under a
+# second on the host): their CPU baseline is a full, exactly timed call.
+FULL_CALL_TOKENS = 15 * 256 * 8
 
-class CpuBaseline:
-    """The fp64 oracle timed on a bounded sample of the workload, scaled to one
-    whole call.  Per head the call costs the frame states plus, per query
-    frame, the softmax rows, readout, RMSNorm and merge; a query frame's cost
-    is taken proportional to the number of keys it scores (window + anchors +
-    text), from the frames actually timed.  The sample is head 0: its frame
-    states and the given query frames."""
+
+def sample_flops(w, heads: int, frames, with_states: bool) -> float:
+    """Algorithmic FLOPs of the sampled work: for each sampled head, the frame
+    and text states (if built) and, per sampled query frame, its softmax pairs
+    and its linear readout -- the same counting as :func:`work`."""
+    anchors = len({0, w.F - 1})
+    per_head = 0.0
+    if with_states:
+        per_head += 2.0 * w.d * (w.d + 1) * (w.P * (w.F - anchors) + w.T)
+    for f in frames:
+        keys = w.P * len(softmax_key_frames(f // w.C, w.F, w.C)) + w.T
+        per_head += 4.0 * w.d * w.P * keys + 2.0 * w.d * (w.d + 1) * w.P
+    return per_head * heads * w.B
+
+
+class OracleSample:
+    """The fp64 oracle, as it stands, timed on a bounded sample of one call of
+    the workload.  Small workloads: the sample is the whole call (all batches,
+    heads and frames).  Large ones: batch 0, head 0 -- its frame and text
+    states and the query rows of its first, middle and last frames (softmax
+    rows, readout, RMSNorm, merge), about 1-3 s of host time at 768p.  The
+    value is the sample's algorithmic FLOPs over its measured time; nothing
+    is extrapolated into it."""
 
     def __init__(self, w, inputs):
-        from oracle import hybrid_attn as O  # only this leg imports the oracle
+        from oracle import hybrid_attn as O  # only the CPU-baseline legs import the oracle
 
         self.O, self.w = O, w
         self.cores = len(os.sched_getaffinity(0))
-        self.x = {k: t[:, :, 0:1, :].to(torch.float64).numpy() for k, t in inputs.items()}
-        self.prob = O.Problem(B=1, F=w.F, P=w.P, H=1, d=w.d, T=w.T, C=w.C)
-        t0 = time.perf_counter()
-        self.cache = {(0, 0): O.frame_states(self.x["k"], self.x["v"], self.prob, 0, 0)}
-        self.t_states = time.perf_counter() - t0
-        self.keys = [w.P * len(softmax_key_frames(f // w.C, w.F, w.C)) + w.T for f in range(w.F)]
+        self.full = w.N * w.H * w.B <= FULL_CALL_TOKENS
+        if self.full:
+            self.x = {k: t.to(torch.float64).numpy() for k, t in inputs.items()}
+            self.prob = O.Problem(B=w.B, F=w.F, P=w.P, H=w.H, d=w.d, T=w.T, C=w.C)
+            self.frames = list(range(w.F))
+            self.flops = work(w)["softmax_flops"] + work(w)["linear_flops"]
+            self.desc = "fp64 oracle, the whole call (all %d heads, all %d frames)" % (w.H, w.F)
+        else:
+            self.x = {k: t[0:1, :, 0:1, :].to(torch.float64).numpy() for k, t in inputs.items()}
+            self.prob = O.Problem(B=1, F=w.F, P=w.P, H=1, d=w.d, T=w.T, C=w.C)
+            self.frames = sorted({0, (w.F // w.C // 2) * w.C, w.F - 1})
+            self.rows = np.concatenate([np.arange(f * w.P, (f + 1) * w.P) for f in self.frames])
+            self.flops = sample_flops(w, 1, self.frames, True) / w.B
+            self.desc = ("fp64 oracle, batch 0 head 0 of %d: frame and text states plus the query rows of frames "
+                         "%s (softmax, readout, RMSNorm, merge)" % (w.H, self.frames))
 
-    def interior_frame(self):
-        return (self.w.F // self.w.C // 2) * self.w.C
-
-    def time_frames(self, frames):
-        """Seconds per key-weighted frame from timing the given query frames."""
+    def run(self) -> float:
+        """Seconds for one pass over the sample."""
         x, O = self.x, self.O
-        spent, keys = 0.0, 0
-        for f in frames:
-            rows = np.arange(f * self.w.P, (f + 1) * self.w.P)
-            t0 = time.perf_counter()
+        t0 = time.perf_counter()
+        if self.full:
+            O.hybrid_attn(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], x["gate_s"], x["gate_l"], self.prob)
+        else:
             O.hybrid_attn_rows(x["q"], x["k"], x["v"], x["text_k"], x["text_v"], x["gate_s"], x["gate_l"],
-                               self.prob, 0, 0, rows, frame_state_cache=self.cache)
-            spent += time.perf_counter() - t0
-            keys += self.keys[f]
-        per_head = self.t_states + spent / keys * sum(self.keys)
-        return per_head * self.w.H * self.w.B, spent
+                               self.prob, 0, 0, self.rows)
+        return time.perf_counter() - t0
+
+    def record(self, secs: float) -> dict:
+        call = work(self.w)["softmax_flops"] + work(self.w)["linear_flops"]
+        value = self.flops / secs / 1e12
+        return {"value": value, "unit": "TFLOP/s", "cores": self.cores, "kind": "oracle", "sample": self.desc,
+                "sample_s": secs, "sample_tflop": self.flops / 1e12,
+                "ms_per_call_extrapolated": None if self.full else call / (value * 1e12) * 1e3}
+
+
+def full_oracle_calls(names=("tiny_fp32", "small_bf16")) -> dict:
+    """Whole oracle calls of the small workloads, each timed exactly (ms)."""
+    out = {}
+    for name in names:
+        w = BY_NAME[name]
+        s = OracleSample(w, make_inputs(w))
+        out[name] = s.run() * 1e3
+    return out
 
 
 # ---------------------------------------------------------------- main
@@ -250,34 +327,33 @@ def barrier(world):
 def run_reference(args, w, world, rank):
     if rank != 0:
         return
-    wk = work(w)
-    flops = (wk["softmax_flops"] + wk["linear_flops"]) * world
-    cb = CpuBaseline(w, make_inputs(w))
-    frame = cb.interior_frame()
-    per_step = []
+    cb = OracleSample(w, make_inputs(w))
+    secs = []
     for i in range(args.warmup + args.steps):
-        est_s, _ = cb.time_frames([frame])
+        t = cb.run()
         if i >= args.warmup:
-            per_step.append(est_s)
-    est = statistics.median(per_step)
-    value = flops / est / 1e12
+            secs.append(t)
+    med = statistics.median(secs)
+    rec = cb.record(med)
+    value = rec["value"]
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": med * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(w, world),
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cb.cores, "kind": "oracle",
-                         "sample": "fp64 oracle; each step times head 0's query frame %d (softmax rows, readout, "
-                                   "RMSNorm, merge); with head 0's frame states it is scaled by key count to all "
-                                   "frames and heads of one call" % frame},
+        "config": config_of(w, world, args.precision),
+        "step": "one pass of the oracle over the sample below (a bounded part of one call of the workload)",
+        "cpu_baseline": rec,
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def config_of(w, world):
-    return {"workload": w.name, "B": w.B, "F": w.F, "P": w.P, "H": w.H, "d": w.d, "T": w.T, "C": w.C,
-            "dtype": w.dtype, "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"}
+def config_of(w, world, precision="bf16"):
+    c = {"workload": w.name, "B": w.B, "F": w.F, "P": w.P, "H": w.H, "d": w.d, "T": w.T, "C": w.C,
+         "dtype": w.dtype, "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas x{world}"}
+    if precision != "bf16":
+        c["softmax_precision"] = precision
+    return c
 
 
 def run_ours(args, w, world, rank, local):
@@ -366,7 +442,7 @@ def run_ours(args, w, world, rank, local):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp8 (e4m3 softmax operands)" if fp8 else "bf16", "data": "synthetic",
-        "config": dict(config_of(w, world), softmax_precision=args.precision),
+        "config": config_of(w, world, args.precision),
         "roofline": {"bound": "tensor", "kernel": "sparse_softmax" + (" (incl. e4m3 quantisation)" if fp8 else ""),
                      "achieved": achieved, "peak": tc_peak,
                      "unit": "TFLOP/s", "frac": achieved / tc_peak, "traffic": None if fp8 else traffic,
@@ -382,14 +458,10 @@ def run_ours(args, w, world, rank, local):
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = CpuBaseline(w, dev_t)
-        frames = sorted({0, cb.interior_frame(), w.F - 1})
-        est_s, spent = cb.time_frames(frames)
-        line["cpu_baseline"] = {"value": flops_call / est_s / 1e12, "unit": "TFLOP/s", "cores": cb.cores,
-                                "kind": "oracle", "ms_per_call_est": est_s * 1e3, "sampled_s": spent + cb.t_states,
-                                "sample": "fp64 oracle: head 0's frame states and query frames %s (softmax rows, "
-                                          "readout, RMSNorm, merge), scaled by key count to all frames and heads "
-                                          "of one call" % frames}
+        cb = OracleSample(w, dev_t)
+        rec = cb.record(min(cb.run() for _ in range(3 if cb.full else 1)))
+        rec["full_call_ms"] = full_oracle_calls()
+        line["cpu_baseline"] = rec
     if rank == 0:
         print(json.dumps(line), flush=True)
 

@@ -220,11 +220,17 @@ VDN_API vdn_status vdn_readout_merge(const void* q, const void* gate_s, const vo
  * GPU that loads the library holds until the process exits.  The first call on
  * a device (with that device current) looks up the array's device address
  * with cudaGetSymbolAddress; make that first call before any stream capture.
- * Nothing is allocated.  Returns VDN_ERR_WORKSPACE, before any CUDA call, when
+ * The address is cached with the id of the CUDA context it was looked up in
+ * and is valid only there: after cudaDeviceReset (or any replacement of the
+ * context) the next call looks it up again, and that call too should precede
+ * any capture.  Nothing is allocated.  Returns VDN_ERR_WORKSPACE when
  * vdn_workspace_bytes(cfg) exceeds the static size (it fits, e.g., 15 frames
- * x 256 tokens x 8 heads x head_dim 64).  All calls on a device share the one
- * array: calls whose GPU work overlaps race and must be ordered by the caller.
- * The status slot of the array is cleared on every call. */
+ * x 256 tokens x 8 heads x head_dim 64); every argument error (sizes,
+ * missing or misaligned pointers, including cfg->status_word and
+ * cfg->rms_weight) is returned before any CUDA call, with nothing queued.
+ * All calls on a device share the one array: calls whose GPU work overlaps
+ * race and must be ordered by the caller.  The status slot of the array is
+ * cleared on every call. */
 VDN_API vdn_status vdn_hybrid_attn_fwd_static(const void* q, const void* k, const void* v,
                                               const void* text_k, const void* text_v,
                                               const void* gate_s, const void* gate_l, void* out,

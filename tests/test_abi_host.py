@@ -12,6 +12,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 from oracle import hybrid_attn as O
 from video_diffusion_hybrid_sparse_b200 import binding as vb
@@ -158,6 +159,29 @@ def test_call_errors_before_any_launch():
     assert lib.vdn_hybrid_attn_fwd_static(*args, ctypes.byref(cfg), None) == 1
     cfg.out_linear = p + 4
     assert lib.vdn_hybrid_attn_fwd(*args, ctypes.byref(cfg), None) == 3
+
+
+def test_static_call_checks_every_pointer_before_any_cuda_call():
+    """vdn_hybrid_attn_fwd_static clears its status slot on the stream before
+    the regular path runs, so every pointer rule must be checked first.  On a
+    host without a GPU any CUDA call fails (VDN_ERR_CUDA): an alignment or
+    argument status therefore shows that the check came before it."""
+    lib = vb.library()
+    s = shape()
+    p = 1 << 20
+    args = [p] * 8
+    cfg = vb.make_cfg(s)
+    cfg.status_word = p + 2  # not 4-byte aligned
+    assert lib.vdn_hybrid_attn_fwd_static(*args, ctypes.byref(cfg), None) == 3
+    cfg = vb.make_cfg(s)
+    cfg.rms_weight = p + 8  # not 16-byte aligned
+    assert lib.vdn_hybrid_attn_fwd_static(*args, ctypes.byref(cfg), None) == 3
+    cfg = vb.make_cfg(s)
+    bad = list(args)
+    bad[6] = p + 4  # gate_l misaligned
+    assert lib.vdn_hybrid_attn_fwd_static(*bad, ctypes.byref(cfg), None) == 3
+    if not torch.cuda.is_available():  # well-formed call: it reaches the CUDA runtime, which has no device here
+        assert lib.vdn_hybrid_attn_fwd_static(*args, ctypes.byref(vb.make_cfg(s)), None) == 5
 
 
 def test_host_call_errors_before_any_copy():

@@ -14,15 +14,21 @@
 // array until the process exits.  Host code cannot pass the array's name to a
 // kernel (on the host it is only a stand-in symbol), so the first call on each
 // device, with that device current, looks up its device address with
-// cudaGetSymbolAddress and caches it; that first call should therefore come
-// before any stream capture.  The call then runs the regular whole-call path
-// with cfg->workspace replaced by that address.  Nothing is allocated:
-// no cudaMalloc, cudaFree or allocating library routine is called.
+// cudaGetSymbolAddress and caches it together with the id of the CUDA context
+// it was looked up in; that first call should therefore come before any
+// stream capture.  The address is only valid in that context: if the context
+// is replaced (cudaDeviceReset, or a primary context released and made again)
+// the module is loaded afresh, the array may move, and the next call looks
+// the address up again (and should again precede any capture).  The call
+// then runs the regular whole-call path with cfg->workspace replaced by that
+// address.  Nothing is allocated: no cudaMalloc, cudaFree or allocating
+// library routine is called.
 //
 // All calls on a device share the one array and it keeps the last call's
 // contents; the status slot at its start is cleared on every call.  Calls
 // whose GPU work overlaps (two streams, or two host threads without
 // ordering) race on the array: the caller must order them.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -37,20 +43,55 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+struct CachedAddress {
+  unsigned long long ctx_id;  // id of the context the address belongs to (0: none yet)
+  void* addr;
+};
 
-// Device address of g_static_scratch on the current device (looked up once per device).
+std::mutex g_mu;
+CachedAddress g_scratch[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion(name, &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
+
+// Id of the context current on this thread; 0 when there is none yet.
+bool current_ctx_id(unsigned long long* id) {
+  static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return false;
+  *id = 0;
+  return !ctx || get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_static_scratch in the current device's current context
+// (looked up once per device, and again whenever that context has changed).
 vdn_status scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return VDN_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
+  unsigned long long id = 0;
+  if (!current_ctx_id(&id)) return VDN_ERR_CUDA;
+  CachedAddress& c = g_scratch[dev];
+  if (id == 0 || c.ctx_id != id || !c.addr) {
+    void* p = nullptr;  // the lookup makes the device's primary context current if none was
     if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return VDN_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+    if (!current_ctx_id(&id) || id == 0) return VDN_ERR_CUDA;
+    c.ctx_id = id;
+    c.addr = p;
   }
-  *out = g_scratch_addr[dev];
+  *out = c.addr;
   return VDN_OK;
 }
 
@@ -72,8 +113,9 @@ extern "C" VDN_API vdn_status vdn_hybrid_attn_fwd_static(const void* q, const vo
   if (valid != VDN_OK) return valid;
   // Problems whose scratch does not fit the static array are rejected before any CUDA call.
   if (vdn_workspace_bytes(&c) > kStaticScratchBytes) return VDN_ERR_WORKSPACE;
-  // Same pointer rules as the regular call, checked here because the status
-  // slot is cleared on the stream before that call runs.
+  // Every pointer rule of the regular call, checked here because the status
+  // slot is cleared on the stream before that call runs: an error return
+  // means nothing was queued and no CUDA call was made.
   for (const void* p : {q, k, v, gate_s, gate_l, static_cast<const void*>(out)})
     if (bad_ptr(p)) return p ? VDN_ERR_ALIGNMENT : VDN_ERR_INVALID_ARG;
   if (cfg->text_tokens > 0)
@@ -82,6 +124,8 @@ extern "C" VDN_API vdn_status vdn_hybrid_attn_fwd_static(const void* q, const vo
   if (cfg->output_mode == VDN_OUTPUT_SPLIT && bad_ptr(cfg->out_linear))
     return cfg->out_linear ? VDN_ERR_ALIGNMENT : VDN_ERR_INVALID_ARG;
   if ((cfg->debug_flags & VDN_EXPORT_STATES) && (!cfg->export_fwd || !cfg->export_bwd)) return VDN_ERR_INVALID_ARG;
+  if (cfg->status_word && (reinterpret_cast<uintptr_t>(cfg->status_word) & 3u) != 0) return VDN_ERR_ALIGNMENT;
+  if (cfg->rms_weight && (reinterpret_cast<uintptr_t>(cfg->rms_weight) & 15u) != 0) return VDN_ERR_ALIGNMENT;
   void* scratch = nullptr;
   const vdn_status s = scratch_address(&scratch);
   if (s != VDN_OK) return s;
