@@ -106,9 +106,10 @@ enum {
   VDN_OUT_SOFTMAX_ONLY = 1, /* out = o_s (no gate) */
   VDN_OUT_LINEAR_ONLY = 2,  /* out = r, the RMS-normalised linear read (no gate) */
   VDN_OUT_LINEAR_RAW = 4,   /* out = o_l, the linear read before RMSNorm */
-  VDN_EXPORT_STATES = 8,    /* vdn_state_scan also writes S_F/z_F and S_B/z_B (fp32) */
+  VDN_EXPORT_STATES = 8,    /* the scan (vdn_state_scan, or the one inside vdn_softmax_and_scan and
+                               the whole calls) also writes S_F/z_F and S_B/z_B (fp32) */
   VDN_INJECT_TIMEOUT = 16,  /* test of the failure path only: in the state build, the MMA thread of
-                               CTA (0, 0) first waits, with a 10-ms limit, for a barrier phase
+                               CTA 0 first waits, with a 10-ms limit, for a barrier phase
                                that nothing completes; it gives up, the CTA's other warps follow, the
                                kernel writes VDN_ERR_TIMEOUT to status_word and returns.  The call's
                                outputs are then undefined; the context stays usable. */
@@ -169,24 +170,32 @@ VDN_API vdn_status vdn_plan_membership(const vdn_cfg* cfg, uint8_t* table);
  * table_dev is DEVICE memory of F*F bytes.  stream is a cudaStream_t. */
 VDN_API vdn_status vdn_membership_device(const vdn_cfg* cfg, uint8_t* table_dev, void* stream);
 
-/* Whole call: staging (fp32 or head_dim 32 only), state build, scan, sparse
- * softmax, readout + merge, all on stream.  out: [B, N, H, d] in dtype (and
- * cfg->out_linear under VDN_OUTPUT_SPLIT). */
+/* Whole call: staging (fp32 or head_dim 32 only), state build, sparse
+ * softmax with the forward/backward scan in the same kernel, readout + merge,
+ * all on stream.  out: [B, N, H, d] in dtype (and cfg->out_linear under
+ * VDN_OUTPUT_SPLIT). */
 VDN_API vdn_status vdn_hybrid_attn_fwd(const void* q, const void* k, const void* v,
                                const void* text_k, const void* text_v,
                                const void* gate_s, const void* gate_l, void* out,
                                const vdn_cfg* cfg, void* stream);
 
 /* The steps of vdn_hybrid_attn_fwd, for callers that schedule them
- * separately (e.g. the linear steps on a second stream).  Run in this order:
- * vdn_stage_inputs (required first when dtype is fp32 or head_dim is 32;
- * otherwise a no-op), then vdn_state_build -> vdn_state_scan, and
- * vdn_sparse_softmax, in either order, then vdn_readout_merge.  Each reads
- * what the earlier steps left in the workspace. */
+ * separately.  vdn_stage_inputs (required first when dtype is fp32 or
+ * head_dim is 32; otherwise a no-op), then either
+ *   vdn_state_build -> vdn_softmax_and_scan -> vdn_readout_merge
+ * (the sequence of the whole call: the scan runs in otherwise idle warps of
+ * the softmax kernel), or, with the linear steps independent of the softmax
+ * branch (e.g. on a second stream),
+ *   vdn_state_build -> vdn_state_scan, and vdn_sparse_softmax, in either
+ *   order, then vdn_readout_merge.
+ * Each reads what the earlier steps left in the workspace. */
 VDN_API vdn_status vdn_stage_inputs(const void* q, const void* k, const void* v,
                             const void* text_k, const void* text_v,
                             const vdn_cfg* cfg, void* stream);
-/* Per-frame-slice partial states [S | z] = phi(K)^T [V | 1] (tensor cores). */
+/* Partial states [S | z] = phi(K)^T [V | 1] (tensor cores): for every state
+ * segment (the non-anchor frames of one chunk, or the text) of every (batch,
+ * head), one partial per state-build CTA whose equal share of the tiles meets
+ * the segment. */
 VDN_API vdn_status vdn_state_build(const void* k, const void* v, const void* text_k,
                            const void* text_v, const vdn_cfg* cfg, void* stream);
 /* Forward/backward chunk states and their sum M_c, fp32 scan. */
@@ -204,6 +213,13 @@ VDN_API vdn_status vdn_export_states(const vdn_cfg* cfg, float* fwd, float* bwd,
 VDN_API vdn_status vdn_sparse_softmax(const void* q, const void* k, const void* v,
                               const void* text_k, const void* text_v,
                               const vdn_cfg* cfg, void* stream);
+/* vdn_sparse_softmax and, in the same kernel, vdn_state_scan: must follow
+ * vdn_state_build on the same workspace (stream order).  Errors as
+ * vdn_sparse_softmax, plus VDN_ERR_INVALID_ARG for VDN_EXPORT_STATES without
+ * export buffers. */
+VDN_API vdn_status vdn_softmax_and_scan(const void* q, const void* k, const void* v,
+                                        const void* text_k, const void* text_v,
+                                        const vdn_cfg* cfg, void* stream);
 /* phi(Q) M_c readout, RMSNorm, gates and merge into out. */
 VDN_API vdn_status vdn_readout_merge(const void* q, const void* gate_s, const void* gate_l,
                              void* out, const vdn_cfg* cfg, void* stream);

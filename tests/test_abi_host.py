@@ -57,7 +57,8 @@ def shape(**kw):
     (dict(T=-1), 1),
     (dict(B=0), 1),
     (dict(P=0), 1),
-    (dict(F=200, C=1), 2),         # more chunks than the scan keeps on chip
+    (dict(F=200, C=1), 0),         # 200 chunks: within the 256 the kernel parameters carry
+    (dict(F=257, C=1), 2),         # more chunks than the kernel parameters carry
     (dict(d=32, fp32=True), 0),
     (dict(d=128, F=60, C=5, P=4032, H=24, T=512), 0),
 ])

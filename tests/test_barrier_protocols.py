@@ -329,27 +329,37 @@ def k4_general_roles(keys):
 
 
 # ------------------------------------------------------------------ k1_state_build
+# pieces: tiles of each run of the CTA's range that lies in one state segment.
 # Buffers: Stage0..2 (the K and V tiles of a stage; phi is applied to K in
-# place), Acc (the TMEM accumulator of the slice).
+# place), Acc0/Acc1 (the two TMEM accumulators, one per piece in turn).
 
 
-def k1_roles(ntiles, stages=3):
-    loads, mma_, phi = [], [], []
-    for i in range(ntiles):
-        st, r = i % stages, i // stages
-        loads += [wait(f"Empty{st}", r - 1), tma(f"Full{st}", (f"Stage{st}", i))]
-        mma_ += [wait(f"Phi{st}", r), mma(reads=[(f"Stage{st}", ("phi", i))], writes=[("Acc", i)]),
-                 commit(f"Empty{st}")]
-        phi += [wait(f"Full{st}", r), beg(reads=[(f"Stage{st}", i)], writes=[(f"Stage{st}", ("phi", i))]),
-                end(f"Stage{st}"), arrive(f"Phi{st}")]
-    mma_.append(commit("Acc"))
-    phi += [wait("Acc", 0), beg(reads=[("Acc", ntiles - 1)]), end("Acc")]
-    return {"loads": loads, "mma": mma_, "phi": phi}
+def k1_roles(pieces, stages=3):
+    loads, mma_, phi, epi = [], [], [], []
+    i = 0
+    for pc, n in enumerate(pieces):
+        a = pc & 1
+        for k in range(n):
+            st, r = i % stages, i // stages
+            loads += [wait(f"Empty{st}", r - 1), tma(f"Full{st}", (f"Stage{st}", i))]
+            phi += [wait(f"Full{st}", r), beg(reads=[(f"Stage{st}", i)], writes=[(f"Stage{st}", ("phi", i))]),
+                    end(f"Stage{st}"), arrive(f"Phi{st}")]
+            if k == 0:
+                mma_.append(wait(f"AccEmpty{a}", (pc >> 1) - 1))
+            mma_ += [wait(f"Phi{st}", r), mma(reads=[(f"Stage{st}", ("phi", i))], writes=[(f"Acc{a}", (pc, k))]),
+                     commit(f"Empty{st}")]
+            if k == n - 1:
+                mma_.append(commit(f"AccFull{a}"))
+            i += 1
+        epi += [wait(f"AccFull{a}", pc >> 1), beg(reads=[(f"Acc{a}", (pc, n - 1))]), end(f"Acc{a}"),
+                arrive(f"AccEmpty{a}")]
+    mma_ += [commit("Done"), wait("Done", 0)]
+    return {"loads": loads, "mma": mma_, "phi": phi, "epilogue": epi}
 
 
 # ------------------------------------------------------------------ k3_sparse_softmax / k3_fp8
 # items: (query tiles of the item, KV tiles of its key set) in the CTA's order.
-# P is handed to the MMA thread in one part (the kernels' default).  The fp8
+# P is handed to the MMA thread in one piece per tile.  The fp8
 # kernel performs the same barrier operations (checked below on the sources).
 # Buffers: Q (the item's query tiles), K0/K1 and V0/V1 (the stages), SP0/SP1
 # (TMEM of S, with P written over it, per query tile), O0/O1 (TMEM output
@@ -458,9 +468,12 @@ def test_general_readout_protocol(keys):
     assert check(k4_general_roles(keys)) > 0
 
 
-@pytest.mark.parametrize("ntiles", [1, 2, 3, 4, 7])
-def test_state_build_protocol(ntiles):
-    assert check(k1_roles(ntiles)) > 0
+K1_PIECES = [[1], [4], [7], [1, 1], [2, 3], [3, 1, 2], [1, 1, 1, 1], [2, 1, 1, 2]]
+
+
+@pytest.mark.parametrize("pieces", K1_PIECES, ids=[str(p) for p in K1_PIECES])
+def test_state_build_protocol(pieces):
+    assert check(k1_roles(pieces)) > 0
 
 
 K3_SCHEDULES = [[(2, 1)], [(2, 3)], [(2, 4)], [(1, 2)], [(2, 2), (2, 1)], [(2, 1), (1, 2)], [(1, 1), (2, 2), (1, 1)],
@@ -484,7 +497,6 @@ def test_fp8_softmax_has_the_bf16_barrier_operations():
         return pat.findall(open(os.path.join(csrc, f)).read())
 
     assert ops("k3_sparse_softmax.cu") == ops("k3_fp8.cu") and len(ops("k3_fp8.cu")) > 10
-    assert re.search(r"#define VDN_P_PARTS 1\b", open(os.path.join(csrc, "k3_sparse_softmax.cu")).read())
 
 
 def _drop(roles, role, pred):
@@ -547,8 +559,15 @@ PLANTED = {
     "general_readout_mma_skips_ready": lambda: _drop(k4_general_roles([0, 1, 1]), "mma",
                                                      lambda op: op.kind == "wait" and op.bar.startswith("AReady")),
     # the state build's MMA thread does not wait for phi(K)
-    "state_build_mma_skips_phi": lambda: _drop(k1_roles(4), "mma",
+    "state_build_mma_skips_phi": lambda: _drop(k1_roles([4]), "mma",
                                                lambda op: op.kind == "wait" and op.bar.startswith("Phi")),
+    # the state build's MMA thread starts a piece in an accumulator still being read out
+    "state_build_mma_skips_acc_release": lambda: _drop(k1_roles([1, 1, 1]), "mma",
+                                                       lambda op: op.kind == "wait" and op.bar.startswith("AccEmpty")),
+    # the read-out releases an accumulator before reading it
+    "state_build_release_before_read": lambda: _move_before(
+        k1_roles([1, 1, 1]), "epilogue", lambda op: op.kind == "arrive" and op.bar.startswith("AccEmpty"),
+        lambda op: op.kind == "beg"),
     # the softmax MMA thread does not wait for P
     "softmax_mma_skips_p": lambda: _drop(k3_roles([(2, 2)]), "mma",
                                          lambda op: op.kind == "wait" and op.bar.startswith("PFull")),
@@ -580,13 +599,14 @@ def test_readout_acc_release_wait_is_implied():
 # programs above model them.  A change to a kernel's barrier use fails here
 # until the model (and this list) is brought up to date.
 SOURCE_BARRIER_OPS = {
-    "k1_state_build.cu": "wait:kEmpty+st expect_tx:kFull+st wait:kAcc wait:kPhi+st mma_commit:kEmpty+st "
-                         "mma_commit:kAcc wait:kFull+st arrive:kPhi+st wait:kAcc",
+    "k1_state_build.cu": "wait:kEmpty+st expect_tx:kFull+st wait:kAccFull wait:kAccEmpty+a wait:kPhi+st "
+                         "mma_commit:kEmpty+st mma_commit:kAccFull+a mma_commit:kDone wait:kFull+st arrive:kPhi+st "
+                         "wait:kAccFull+buf arrive:kAccEmpty+buf",
     "k3_sparse_softmax.cu": "wait:kQEmpty expect_tx:kQFull wait:kKEmpty+st expect_tx:kKFull+st wait:kVEmpty+st "
                             "expect_tx:kVFull+st wait:kQFull wait:kKFull+st mma_commit:kSFull+t "
-                            "mma_commit:kKEmpty+st wait:kVFull+st wait:kPFull+2*part+t mma_commit:kOFull+t "
+                            "mma_commit:kKEmpty+st wait:kVFull+st wait:kPFull+t mma_commit:kOFull+t "
                             "wait:kKFull+nst mma_commit:kSFull+t mma_commit:kVEmpty+st mma_commit:kKEmpty+nst "
-                            "mma_commit:kQEmpty mma_commit:kDone wait:kSFull+t arrive:kPFull+2*part+t "
+                            "mma_commit:kQEmpty mma_commit:kDone wait:kSFull+t arrive:kPFull+t "
                             "wait:kOFull+t",
     "k4_merge_tma.cu": "wait:kTBEmpty expect_tx:kTBFull wait:kTAEmpty expect_tx:kTAFull wait:kTGEmpty "
                        "expect_tx:kTGFull wait:kTBFull wait:kTAReady+s wait:kTAccEmpty+s mma_commit:kTAccFull+s "

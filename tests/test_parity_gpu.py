@@ -180,7 +180,15 @@ def test_host_tensor_call_equals_device_call(w, mode, split):
         assert torch.equal(out_lin, ref_lin.cpu())
 
 
-@pytest.mark.parametrize("w", [SMALL[0], SMALL[2], SMALL[3]], ids=["tiny", "ragged", "c5_ragged"])
+# Exported forward/backward states against the oracle's: relative L2 4e-3.
+# The states are fp32 sums of phi(k) v^T with phi(k) rounded to bf16 for the
+# tensor cores (relative rounding <= 2^-9, about 1.1e-3 RMS per term,
+# unbiased), so the relative error of a state is about 1e-3; fp32 inputs add
+# their own rounding to bf16 before phi.
+STATE_TOL = 4e-3
+
+
+@pytest.mark.parametrize("w", [SMALL[0], SMALL[2], SMALL[3], SMALL[1]], ids=["tiny", "ragged", "c5_ragged", "small"])
 def test_exported_states_match_oracle(w):
     inputs = make_inputs(w)
     dev = to_dev(inputs)
@@ -190,16 +198,25 @@ def test_exported_states_match_oracle(w):
     bwd = torch.zeros_like(fwd)
     run(w, dev, debug_flags=vb.EXPORT_STATES, export=(fwd, bwd))
     fwd, bwd = fwd.cpu().numpy(), bwd.cpu().numpy()
+    worst = 0.0
     for b in range(w.B):
         for h in range(w.H):
             st = ref["states"][(b, h)]
             # exported layout: row a' < d holds S[:, a'] (value column a'), row d holds z
             ref_f = np.concatenate([st["SF"].transpose(0, 2, 1), st["zF"][:, None, :]], axis=1)
             ref_b = np.concatenate([st["SB"].transpose(0, 2, 1), st["zB"][:, None, :]], axis=1)
-            assert rel_l2(fwd[b, :, h], ref_f) <= 1e-2
-            assert rel_l2(bwd[b, :, h], ref_b) <= 1e-2
+            ef, eb = rel_l2(fwd[b, :, h], ref_f), rel_l2(bwd[b, :, h], ref_b)
+            worst = max(worst, ef, eb)
+            assert ef <= STATE_TOL and eb <= STATE_TOL, (b, h, ef, eb)
             if w.T > 0:  # chunk 0's forward state holds nothing but half of the text state
-                assert rel_l2(fwd[b, 0, h, :w.d, :], 0.5 * st["S_t"].T) <= 1e-2
+                assert rel_l2(fwd[b, 0, h, :w.d, :], 0.5 * st["S_t"].T) <= STATE_TOL
+            # the states that hold no video frame are the same half text state, bit for bit:
+            # forward of chunks 0 and 1, backward of the last two chunks
+            half_t = fwd[b, 0, h]
+            for c in range(min(2, nc)):
+                assert np.array_equal(fwd[b, c, h], half_t), f"forward state of chunk {c} holds video"
+                assert np.array_equal(bwd[b, nc - 1 - c, h], half_t), f"backward state of chunk {nc - 1 - c} holds video"
+    print(f"{w.name}: worst state rel-L2 {worst:.2e}")
 
 
 def test_rms_weight_gamma():
@@ -226,6 +243,27 @@ def test_steps_equal_whole_call_and_deterministic():
     assert torch.equal(out, a)
 
 
+@pytest.mark.parametrize("w,mode", [(BY_NAME["small_bf16"], 0), (SMALL[3], 0), (SMALL[3], 1), (SMALL[0], 0),
+                                    (SMALL[9], 0)], ids=["small", "c5_ragged", "c5_ragged_global", "tiny_fp32", "d32"])
+def test_scan_inside_softmax_equals_separate_scan(w, mode):
+    """The forward/backward scan run by the softmax kernel's idle warps and the
+    scan launched on its own write the same readout operands: the outputs of
+    the two step sequences are bit-identical."""
+    dev = to_dev(make_inputs(w))
+    outs = []
+    for seq in ("all", "all_separate"):
+        out = torch.full_like(dev["q"], float("nan"))
+        steps = vb.Steps(dev["q"], dev["k"], dev["v"], dev["text_k"], dev["text_v"], dev["gate_s"], dev["gate_l"],
+                         out, frames=w.F, chunk_frames=w.C, anchor_query_mode=mode,
+                         workspace=torch.empty(vb.workspace_bytes(vb.shape_of(dev["q"], dev["text_k"], w.F, w.C)),
+                                               dtype=torch.uint8, device="cuda"))
+        getattr(steps, seq)()
+        torch.cuda.synchronize()
+        outs.append(out)
+    word = torch.int32 if outs[0].dtype == torch.float32 else torch.int16
+    assert torch.equal(outs[0].view(word), outs[1].view(word))
+
+
 def test_status_word_stays_clear():
     w = SMALL[2]
     dev = to_dev(make_inputs(w))
@@ -249,8 +287,8 @@ def sample_rows(w: Workload, rng, n_random=24):
     return np.array(sorted(rows))
 
 
-@pytest.mark.parametrize("name,heads", [("chunk5_bf16", [0, 15]), ("768p_bf16", [0, 23]),
-                                        ("768p_long_bf16", [7])])
+@pytest.mark.parametrize("name,heads", [("chunk5_bf16", [0, 7, 15]), ("768p_bf16", [0, 4, 9, 14, 19, 23]),
+                                        ("768p_long_bf16", [0, 7, 23])])
 def test_workload_sampled_rows(name, heads):
     w = BY_NAME[name]
     inputs = make_inputs(w)

@@ -25,7 +25,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "po
 
 EXPORTED = ["vdn_version", "vdn_status_string", "vdn_validate", "vdn_workspace_bytes", "vdn_plan_membership",
             "vdn_membership_device", "vdn_hybrid_attn_fwd", "vdn_stage_inputs", "vdn_state_build",
-            "vdn_state_scan", "vdn_sparse_softmax", "vdn_readout_merge", "vdn_hybrid_attn_fwd_static",
+            "vdn_state_scan", "vdn_sparse_softmax", "vdn_softmax_and_scan", "vdn_readout_merge",
+            "vdn_hybrid_attn_fwd_static",
             "vdn_static_scratch_bytes", "vdn_host_staging_bytes", "vdn_hybrid_attn_fwd_host", "vdn_export_states"]
 
 
@@ -75,6 +76,7 @@ def library() -> ctypes.CDLL:
         lib.vdn_state_scan.argtypes = [C, P]
         lib.vdn_export_states.argtypes = [C, P, P, P]
         lib.vdn_sparse_softmax.argtypes = [P, P, P, P, P, C, P]
+        lib.vdn_softmax_and_scan.argtypes = [P, P, P, P, P, C, P]
         lib.vdn_readout_merge.argtypes = [P, P, P, P, C, P]
         lib.vdn_hybrid_attn_fwd_static.argtypes = [P, P, P, P, P, P, P, P, C, P]
         lib.vdn_static_scratch_bytes.restype = ctypes.c_size_t
@@ -315,12 +317,25 @@ class Steps:
         _check(self.lib.vdn_sparse_softmax(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(tk), _ptr(tv),
                                            ctypes.byref(self.cfg), _stream(stream)), "vdn_sparse_softmax")
 
+    def softmax_and_scan(self, stream=None):
+        q, k, v, tk, tv = self.t[:5]
+        _check(self.lib.vdn_softmax_and_scan(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(tk), _ptr(tv),
+                                             ctypes.byref(self.cfg), _stream(stream)), "vdn_softmax_and_scan")
+
     def readout_merge(self, stream=None):
         q, gs, gl, out = self.t[0], self.t[5], self.t[6], self.t[7]
         _check(self.lib.vdn_readout_merge(q.data_ptr(), gs.data_ptr(), gl.data_ptr(), out.data_ptr(),
                                           ctypes.byref(self.cfg), _stream(stream)), "vdn_readout_merge")
 
     def all(self, stream=None):
+        """The whole call's sequence (the scan inside the softmax kernel)."""
+        self.stage(stream)
+        self.state_build(stream)
+        self.softmax_and_scan(stream)
+        self.readout_merge(stream)
+
+    def all_separate(self, stream=None):
+        """The same result with the scan as a kernel of its own."""
         self.stage(stream)
         self.state_build(stream)
         self.state_scan(stream)

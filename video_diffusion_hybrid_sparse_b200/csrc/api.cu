@@ -14,7 +14,7 @@
 namespace vdn {
 namespace {
 
-constexpr int kMaxScanChunks = 96;  // chunk sums of the scan live in shared memory
+constexpr int kMaxScanChunks = kMaxChunks;  // state segments carried in kernel parameters
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -64,10 +64,12 @@ vdn_status make_geom(const vdn_cfg* cfg, Geom& g) {
   g.N = N;
   g.fp32_io = cfg->dtype == VDN_FP32;
   g.staged = g.fp32_io || g.d != g.Dp;
-  g.n_slices = (g.P + kSliceTokens - 1) / kSliceTokens;
-  g.n_video_parts = (g.F - n_anchor(g.F)) * g.n_slices;
-  g.n_text_parts = (g.T + kSliceTokens - 1) / kSliceTokens;
-  g.n_parts = g.n_video_parts + g.n_text_parts;
+  {
+    StatePlan sp;
+    build_state_plan(g, sp);
+    g.n_state_segs = sp.n_segs;
+    g.n_part_slots = (long long)g.B * g.H * sp.n_segs * sp.cmax;
+  }
   g.rows_per_chunk = g.C * g.P;
   g.n_pairs = (g.rows_per_chunk + 2 * kBlockM - 1) / (2 * kBlockM);
   g.mt_rows = g.Dp + 16;
@@ -87,7 +89,9 @@ vdn_status make_geom(const vdn_cfg* cfg, Geom& g) {
     g.off_tk = off; off = align_up(off + txt, 1024);
     g.off_tv = off; off = align_up(off + txt, 1024);
   }
-  g.off_parts = off; off = align_up(off + (size_t)g.n_parts * g.B * g.H * (g.Dp + 1) * g.Dp * 4, 1024);
+  const size_t state_bytes = (size_t)(g.Dp + 1) * g.Dp * 4;
+  g.off_parts = off; off = align_up(off + (size_t)g.n_part_slots * state_bytes, 1024);
+  g.off_segst = off; off = align_up(off + (size_t)g.B * g.H * g.n_state_segs * state_bytes, 1024);
   g.off_mt = off; off = align_up(off + (size_t)g.B * g.Nc * g.H * 2 * g.mt_rows * g.Dp * 2, 1024);
   g.fp8 = cfg->softmax_precision == VDN_PREC_FP8;
   if (g.fp8) {
@@ -233,31 +237,73 @@ vdn_status step_stage(const vdn_cfg* cfg, const Geom& g, const void* q, const vo
   return cuda_status(e);
 }
 
+// 8-byte counter of the scan units the softmax kernel has handed out, at byte
+// 128 of the workspace's status slot.
+unsigned long long* scan_counter_ptr(const vdn_cfg* cfg, const Geom& g) {
+  return reinterpret_cast<unsigned long long*>(ws(cfg, g.off_status) + 128);
+}
+
 vdn_status step_state_build(const vdn_cfg* cfg, const Geom& g, const Srcs& s, cudaStream_t st) {
-  if (g.n_parts == 0) return VDN_OK;
-  Maps m;
-  if (!make_maps(m, g, s)) return VDN_ERR_CUDA;
   K1Params p;
   p.g = g;
+  build_state_plan(g, p.sp);
+  Maps m;
+  if (!make_maps(m, g, s)) return VDN_ERR_CUDA;
   p.parts = reinterpret_cast<float*>(ws(cfg, g.off_parts));
   p.status = status_ptr(cfg, g);
   p.record = record_ptr(cfg, g);
   p.inject_timeout = (cfg->debug_flags & VDN_INJECT_TIMEOUT) != 0;
+  p.scan_counter = scan_counter_ptr(cfg, g);
   return cuda_status(launch_state_build(m, p, st));
 }
 
-vdn_status step_state_scan(const vdn_cfg* cfg, const Geom& g, cudaStream_t st) {
-  K2Params p;
-  p.g = g;
-  p.parts = reinterpret_cast<const float*>(ws(cfg, g.off_parts));
-  p.mt = ws(cfg, g.off_mt);
+void make_scan_args(const vdn_cfg* cfg, const Geom& g, ScanArgs& sa) {
+  sa.g = g;
+  build_state_plan(g, sa.sp);
+  sa.parts = reinterpret_cast<const float*>(ws(cfg, g.off_parts));
+  sa.segst = reinterpret_cast<float*>(ws(cfg, g.off_segst));
+  sa.mt = ws(cfg, g.off_mt);
   const bool exp = (cfg->debug_flags & VDN_EXPORT_STATES) != 0;
-  p.export_fwd = exp ? cfg->export_fwd : nullptr;
-  p.export_bwd = exp ? cfg->export_bwd : nullptr;
-  return cuda_status(launch_state_scan(p, st));
+  sa.export_fwd = exp ? cfg->export_fwd : nullptr;
+  sa.export_bwd = exp ? cfg->export_bwd : nullptr;
 }
 
-vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s, cudaStream_t st) {
+vdn_status step_state_scan(const vdn_cfg* cfg, const Geom& g, cudaStream_t st) {
+  ScanArgs sa;
+  make_scan_args(cfg, g, sa);
+  return cuda_status(launch_state_scan(sa, st));
+}
+
+// Work items of the softmax kernel.  Block 0: the segments that read every
+// frame (GLOBAL anchor rows), the longest items, first.  Block 1: the chunk
+// segments in chunk order, so that the items the persistent CTAs run at the
+// same time share a head's keys and values (and neighbouring chunks two of
+// their three window chunks).  Each block is ordered (batch, head, segment,
+// pair).
+void plan_items(const Geom& g, K3Params& p) {
+  QSeg segs[kMaxSegs];
+  const int n = query_segments(g, segs);
+  int k = 0, nb = 0;
+  p.blk_seg0[0] = 0;
+  for (int blk = 0; blk < 2; ++blk) {
+    const int k0 = k;
+    for (int i = 0; i < n; ++i)
+      if ((segs[i].c == kAllFrames) == (blk == 0)) p.segs[k++] = segs[i];
+    if (k > k0) p.blk_seg0[++nb] = k;
+  }
+  p.n_blocks = nb;
+  p.seg_pair0[0] = 0;
+  for (int i = 0; i < k; ++i)
+    p.seg_pair0[i + 1] = p.seg_pair0[i] + (p.segs[i].nrows + 2 * kBlockM - 1) / (2 * kBlockM);
+  p.blk_item0[0] = 0;
+  for (int b = 0; b < nb; ++b)
+    p.blk_item0[b + 1] = p.blk_item0[b] + g.B * g.H * (p.seg_pair0[p.blk_seg0[b + 1]] - p.seg_pair0[p.blk_seg0[b]]);
+  p.n_items = p.blk_item0[nb];
+}
+
+// The softmax branch; with do_scan, the kernel's otherwise idle warps also
+// run the forward/backward scan of the state partials in the workspace.
+vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s, cudaStream_t st, bool do_scan) {
   Maps m;
   if (!make_maps(m, g, s)) return VDN_ERR_CUDA;
   K3Params p;
@@ -292,20 +338,10 @@ vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s,
   p.o_s = reinterpret_cast<__nv_bfloat16*>(ws(cfg, g.off_os));
   p.status = status_ptr(cfg, g);
   p.record = record_ptr(cfg, g);
-  // query segments, longest key set first (static longest-processing-time order)
-  QSeg segs[kMaxSegs];
-  const int n = query_segments(g, segs);
-  std::stable_sort(segs, segs + n, [&](const QSeg& a, const QSeg& b) {
-    return seg_kv_tiles(a.c, g) > seg_kv_tiles(b.c, g);
-  });
-  p.n_segs = n;
-  p.seg_item0[0] = 0;
-  for (int k = 0; k < n; ++k) {
-    p.segs[k] = segs[k];
-    const int pairs = (segs[k].nrows + 2 * kBlockM - 1) / (2 * kBlockM);
-    p.seg_item0[k + 1] = p.seg_item0[k] + g.B * g.H * pairs;
-  }
-  p.n_items = p.seg_item0[n];
+  plan_items(g, p);
+  p.do_scan = do_scan ? 1 : 0;
+  p.scan_counter = scan_counter_ptr(cfg, g);
+  if (do_scan) make_scan_args(cfg, g, p.scan);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -503,7 +539,20 @@ vdn_status vdn_sparse_softmax(const void* q, const void* k, const void* v, const
   if (s != VDN_OK) return s;
   s = check_inputs(cfg, g, {q, k, v}, {text_k, text_v});
   if (s != VDN_OK) return s;
-  return step_sparse_softmax(cfg, g, kernel_srcs(cfg, g, q, k, v, text_k, text_v), static_cast<cudaStream_t>(stream));
+  return step_sparse_softmax(cfg, g, kernel_srcs(cfg, g, q, k, v, text_k, text_v), static_cast<cudaStream_t>(stream),
+                             false);
+}
+
+vdn_status vdn_softmax_and_scan(const void* q, const void* k, const void* v, const void* text_k, const void* text_v,
+                                const vdn_cfg* cfg, void* stream) {
+  Geom g;
+  vdn_status s = make_geom(cfg, g);
+  if (s != VDN_OK) return s;
+  s = check_inputs(cfg, g, {q, k, v}, {text_k, text_v});
+  if (s != VDN_OK) return s;
+  if ((cfg->debug_flags & VDN_EXPORT_STATES) && (!cfg->export_fwd || !cfg->export_bwd)) return VDN_ERR_INVALID_ARG;
+  return step_sparse_softmax(cfg, g, kernel_srcs(cfg, g, q, k, v, text_k, text_v), static_cast<cudaStream_t>(stream),
+                             true);
 }
 
 vdn_status vdn_readout_merge(const void* q, const void* gate_s, const void* gate_l, void* out, const vdn_cfg* cfg,
@@ -532,8 +581,7 @@ vdn_status vdn_hybrid_attn_fwd(const void* q, const void* k, const void* v, cons
   if (poison_ws(cfg, g, st) != cudaSuccess) return VDN_ERR_CUDA;
   if ((s = step_stage(cfg, g, q, k, v, text_k, text_v, st)) != VDN_OK) return s;
   if ((s = step_state_build(cfg, g, src, st)) != VDN_OK) return s;
-  if ((s = step_state_scan(cfg, g, st)) != VDN_OK) return s;
-  if ((s = step_sparse_softmax(cfg, g, src, st)) != VDN_OK) return s;
+  if ((s = step_sparse_softmax(cfg, g, src, st, true)) != VDN_OK) return s;  // the scan runs inside
   return step_readout_merge(cfg, g, src, gate_s, gate_l, out, st);
 }
 
@@ -606,9 +654,8 @@ vdn_status vdn_hybrid_attn_fwd_host(const void* q, const void* k, const void* v,
     if ((s = step_stage(&c, g, dq, dk, dvv, dtk, dtv, st)) != VDN_OK) return finish(s);
   }
   if ((s = step_state_build(&c, g, src, st)) != VDN_OK) return finish(s);
-  if ((s = step_state_scan(&c, g, st)) != VDN_OK) return finish(s);
   if (cudaStreamWaitEvent(st, ev[2], 0) != cudaSuccess) return finish(VDN_ERR_CUDA);
-  if ((s = step_sparse_softmax(&c, g, src, st)) != VDN_OK) return finish(s);
+  if ((s = step_sparse_softmax(&c, g, src, st, true)) != VDN_OK) return finish(s);  // the scan runs inside
   if (cudaStreamWaitEvent(st, ev[3], 0) != cudaSuccess) return finish(VDN_ERR_CUDA);
   if ((s = step_readout_merge(&c, g, src, dv + h.gs, dv + h.gl, dv + h.out, st)) != VDN_OK) return finish(s);
   ce = cudaMemcpyAsync(out, dv + h.out, vid, cudaMemcpyDeviceToHost, st);

@@ -1,22 +1,35 @@
-// k1_state_build.cu - per-slice linear-attention states of the VDN-H3 linear
-// branch (article section 双分支混合注意力机制: the frame-wise linear memory).
+// k1_state_build.cu - linear-attention states of the VDN-H3 linear branch
+// (article section 双分支混合注意力机制: the frame-wise linear memory).
 //
-// For one slice of up to 2048 key tokens of one non-anchor frame (or of the
-// text), one batch and one head, it computes on the tensor cores
+// For every (batch, head) and state segment -- the non-anchor frames of one
+// chunk, or the text -- the states are
 //
 //     [S | z] = phi(K)^T [V | 1],   S: d x d,  z: d,   phi = elu + 1,
 //
-// with bf16 operands and fp32 accumulation in TMEM.  Anchor frames get no
-// state (no state ever reads them).  The output partial is stored transposed,
-// part[b_col][a] with row Dp holding z, which is the K-major order the
+// computed on the tensor cores with bf16 operands and fp32 accumulation in
+// TMEM.  Anchor frames get no state (no state ever reads them).
+//
+// Work split (stream-K): the 128-token tiles of every (batch, head, segment)
+// form one list, (batch, head)-major; the grid is one wave of CTAs and CTA k
+// takes the k-th of `grid` equal contiguous ranges of that list, so every SM
+// streams the same number of tiles.  A CTA accumulates over the run of its
+// tiles that lies in one segment (a "piece") and writes that run's sum as one
+// partial to the segment's slot for this CTA; the scan adds a segment's
+// partials.  Partials are stored transposed, part[n][a] with row n = value
+// column (row Dp holds z) and a = phi(k) slot, which is the K-major order the
 // readout consumes.
 //
-// Per 128-token tile: TMA brings the K tile and the V tile (128-byte swizzle);
-// sixteen warps apply phi in place on the K tile (zeroing rows past the slice and
-// padded head_dim columns) and fence it to the async proxy; one thread issues
-//   D[:, 0:Dp]    += phi(K)^T V      (A and B both MN-major, M = 128 = head_dim slots)
-//   D[:, Dp:Dp+16] += phi(K)^T 1     (B = a block of ones)
-// Three pipeline stages keep the HBM stream busy.
+// Roles (22 warps):
+//   * warp 0 (one thread): TMA loads of the K and V tiles (128-byte swizzle),
+//     three stages;
+//   * warps 2-17: phi in place on the K tile (rows past the segment and padded
+//     head_dim columns zeroed), fenced to the async proxy;
+//   * warp 1 (one thread): D[:, 0:Dp] += phi(K)^T V and D[:, Dp:Dp+16] +=
+//     phi(K)^T 1 (both operands MN-major, M = 128 head_dim slots; B = a block
+//     of bf16 ones gives z) into one of two TMEM accumulators, one per piece
+//     in turn, so a piece's read-out overlaps the next piece's products;
+//   * warps 18-21: read a finished accumulator (TMEM lane = phi slot) and
+//     store the partial.
 #include "kernels.h"
 #include "phi.cuh"
 #include "sm100.cuh"
@@ -35,11 +48,43 @@ struct K1Layout {
   static constexpr int kOnesBytes = 4096;
   static constexpr int kBar = kOnes + kOnesBytes;
   static constexpr int kBytes = kBar + 256 + 1024;
+  static constexpr int kCols = D + 16;                     // accumulator columns: values, z (+ padding)
+  static constexpr int kAccCols = kCols <= 128 ? 128 : 256;  // one accumulator slot
 };
 
-enum { kFull = 0, kPhi = 3, kEmpty = 6, kAcc = 9, kNumBars1 = 10 };
-constexpr int kPhiThreads = 512;  // warps 2..17
-constexpr int kK1Threads = 64 + kPhiThreads;
+enum { kFull = 0, kPhi = 3, kEmpty = 6, kAccFull = 9, kAccEmpty = 11, kDone = 13, kNumBars1 = 14 };
+constexpr int kPhiWarps = 16;        // warps 2..17
+constexpr int kPhiThreads = 32 * kPhiWarps;
+constexpr int kEpiWarp0 = 2 + kPhiWarps;  // warps 18..21
+constexpr int kK1Threads = 32 * (kEpiWarp0 + 4);
+
+// Tile `t` of this CTA's range, decoded.
+struct SbTile {
+  int bh, seg, row, n_valid;
+  bool text;
+};
+
+__device__ __forceinline__ SbTile sb_tile(long long t, const Geom& g, const StatePlan& sp) {
+  SbTile r;
+  r.bh = (int)(t / sp.tiles_per_bh);
+  const int lt = (int)(t - (long long)r.bh * sp.tiles_per_bh);
+  r.seg = sb_seg_of(lt, sp);
+  const int tis = lt - sp.seg_tile0[r.seg];
+  r.text = r.seg >= sp.n_vsegs;
+  const int b = r.bh / g.H;
+  r.row = (r.text ? b * g.T : b * (int)g.N) + sp.seg_row0[r.seg] + tis * 128;
+  r.n_valid = min(128, sp.seg_rows[r.seg] - tis * 128);
+  return r;
+}
+
+// The CTA's tile t ends its piece (the next tile is in another segment, or the range ends).
+__device__ __forceinline__ bool piece_ends(long long t, long long t_end, const StatePlan& sp) {
+  if (t + 1 >= t_end) return true;
+  const int bh = (int)(t / sp.tiles_per_bh), bh1 = (int)((t + 1) / sp.tiles_per_bh);
+  if (bh != bh1) return true;
+  const int lt1 = (int)(t + 1 - (long long)bh * sp.tiles_per_bh);
+  return sb_seg_of(lt1, sp) != sb_seg_of(lt1 - 1, sp);
+}
 
 }  // namespace
 
@@ -49,8 +94,6 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                    const __grid_constant__ CUtensorMap tm_tk, const __grid_constant__ CUtensorMap tm_tv,
                    const __grid_constant__ K1Params p) {
   using L = K1Layout<D>;
-  constexpr int kCols = D + 16;
-  constexpr int kAlloc = kCols <= 128 ? 128 : 256;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
@@ -58,37 +101,24 @@ __global__ void __launch_bounds__(kK1Threads, 1)
   int* abort_flag = reinterpret_cast<int*>(smem + L::kBar + kNumBars1 * 8 + 4);
 
   const Geom& g = p.g;
-  // (batch, head) is the fastest grid index: CTAs that run together read
-  // whole [H, d] token rows of k and v rather than scattered 256-byte pieces
-  const int bh = blockIdx.x;
-  const int part = blockIdx.y;
-  const int b = bh / g.H, h = bh % g.H;
+  const StatePlan& sp = p.sp;
+  const long long t_begin = sp.grid > 0 ? sb_range_start(blockIdx.x, sp) : 0;
+  const long long t_end = sp.grid > 0 ? sb_range_start(blockIdx.x + 1, sp) : 0;
+  const int ntiles = (int)(t_end - t_begin);
   const uint32_t warp = warp_id(), lane = lane_id();
 
-  // token range of this part
-  const bool text = part >= g.n_video_parts;
-  int row0, ntok;
-  if (!text) {
-    const int f = part_frame(part, g);
-    const int s = part % g.n_slices;
-    row0 = b * (int)g.N + f * g.P + s * kSliceTokens;
-    ntok = min(kSliceTokens, g.P - s * kSliceTokens);
-  } else {
-    const int tp = part - g.n_video_parts;
-    row0 = b * g.T + tp * kSliceTokens;
-    ntok = min(kSliceTokens, g.T - tp * kSliceTokens);
-  }
-  const int ntiles = (ntok + 127) / 128;
-  const CUtensorMap* mk = text ? &tm_tk : &tm_k;
-  const CUtensorMap* mv = text ? &tm_tv : &tm_v;
-
+  if (threadIdx.x == 0 && blockIdx.x == 0 && p.scan_counter) *p.scan_counter = 0ull;
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&bars[kFull + s], 1);
       mbar_init(&bars[kPhi + s], kPhiThreads);
       mbar_init(&bars[kEmpty + s], 1);
     }
-    mbar_init(&bars[kAcc], 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&bars[kAccFull + a], 1);
+      mbar_init(&bars[kAccEmpty + a], 128);
+    }
+    mbar_init(&bars[kDone], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -102,7 +132,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
   }
   fence_proxy_async_smem();
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kAlloc);
+    tmem_alloc(tmem_slot, 2 * L::kAccCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -112,6 +142,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
   const CtaAbort ab{abort_flag, p.status, p.record, 1};
 
   if (warp == 0) {
+    // ------------------------------------------------------------ loads
     if (lane == 0) {
       int i = 0;
       bool ok = true;
@@ -119,12 +150,16 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         const int st = i % L::kStages;
         const uint32_t ph = (i / L::kStages) & 1;
         if (!mbar_wait(&bars[kEmpty + st], ph ^ 1, ab)) { ok = false; break; }
+        const SbTile tl = sb_tile(t_begin + i, g, sp);
+        const int h = tl.bh % g.H;
+        const CUtensorMap* mk = tl.text ? &tm_tk : &tm_k;
+        const CUtensorMap* mv = tl.text ? &tm_tv : &tm_v;
         mbar_expect_tx(&bars[kFull + st], (D / 64) * 16384 * 2);
         uint8_t* sa = smem + st * L::kStage;
         uint8_t* sb = sa + L::kATile;
         for (int bx = 0; bx < D / 64; ++bx) {
-          tma_load_2d(sa + bx * 16384, mk, &bars[kFull + st], h * D + bx * 64, row0 + i * 128);
-          tma_load_2d(sb + bx * 16384, mv, &bars[kFull + st], h * D + bx * 64, row0 + i * 128);
+          tma_load_2d(sa + bx * 16384, mk, &bars[kFull + st], h * D + bx * 64, tl.row);
+          tma_load_2d(sb + bx * 16384, mv, &bars[kFull + st], h * D + bx * 64, tl.row);
         }
       }
       if (!ok)
@@ -132,83 +167,106 @@ __global__ void __launch_bounds__(kK1Threads, 1)
           mbar_drain(&bars[kFull + k % L::kStages], (k / L::kStages) & 1);
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA
     if (lane == 0) {
       constexpr uint32_t idesc_v = idesc_bf16_f32(128, D, 1, 1);
       constexpr uint32_t idesc_1 = idesc_bf16_f32(128, 16, 1, 1);
       const uint32_t ones = smem_u32(smem + L::kOnes);
-      // failure-path test: wait (with a short limit) for the accumulator
-      // phase, which only this thread's final commit completes; the wait runs
-      // out, the CTA gives up and the status word records the timeout
-      const bool injected = p.inject_timeout && blockIdx.x == 0 && blockIdx.y == 0 &&
-                            !mbar_wait(&bars[kAcc], 0, ab, 10000000ll);
+      // failure-path test: wait (with a short limit) for the first
+      // accumulator phase, which only this thread's own commit completes; the
+      // wait runs out, the CTA gives up and the status word records the timeout
+      const bool injected = p.inject_timeout && blockIdx.x == 0 && !mbar_wait(&bars[kAccFull], 0, ab, 10000000ll);
+      int piece = 0;
+      bool first = true;  // first tile of the current piece
       for (int i = 0; i < ntiles && !injected; ++i) {
         const int st = i % L::kStages;
+        const int a = piece & 1;
+        if (first && !mbar_wait(&bars[kAccEmpty + a], ((piece >> 1) & 1) ^ 1, ab)) break;
         if (!mbar_wait(&bars[kPhi + st], (i / L::kStages) & 1, ab)) break;
         tc_fence_after();
+        const uint32_t acc = tmem + a * L::kAccCols;
         const uint32_t sa = smem_u32(smem + st * L::kStage);
         const uint32_t sb = sa + L::kATile;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = smem_desc(sa + kk * 2048, 16384, 1024, kLayoutSw128);
+          const uint64_t da = smem_desc(sa + kk * 2048, 16384, 1024, kLayoutSw128);
           const uint64_t bv = smem_desc(sb + kk * 2048, 16384, 1024, kLayoutSw128);
           const uint64_t b1 = smem_desc(ones, 256, 256, kLayoutNone);
-          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          mma_ss(tmem, a, bv, idesc_v, acc);
-          mma_ss(tmem + D, a, b1, idesc_1, acc);
+          const uint32_t accum = (!first || kk > 0) ? 1u : 0u;
+          mma_ss(acc, da, bv, idesc_v, accum);
+          mma_ss(acc + D, da, b1, idesc_1, accum);
         }
         mma_commit(&bars[kEmpty + st]);
+        first = piece_ends(t_begin + i, t_end, sp);
+        if (first) {
+          mma_commit(&bars[kAccFull + a]);
+          ++piece;
+        }
       }
-      mma_commit(&bars[kAcc]);
+      // every MMA of this thread completes before TMEM is released
+      mma_commit(&bars[kDone]);
     }
-  } else {
-    // warps 2..17: phi workers; warps 2..5 then read the accumulator out
+  } else if (warp < kEpiWarp0) {
+    // ------------------------------------------------------------ phi workers
     const int tid = threadIdx.x - 64;
-    bool ok = true;
     for (int i = 0; i < ntiles; ++i) {
       const int st = i % L::kStages;
       const bool got = mbar_wait(&bars[kFull + st], (i / L::kStages) & 1, ab);
-      if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
-      phi_tile_inplace(smem + st * L::kStage, D / 64, ntok - i * 128, g.d, tid, kPhiThreads);
+      if (__any_sync(0xffffffffu, !got)) break;
+      const SbTile tl = sb_tile(t_begin + i, g, sp);
+      phi_tile_inplace<D / 64 * 1024 / kPhiThreads>(smem + st * L::kStage, D / 64, tl.n_valid, g.d, tid, kPhiThreads);
       fence_proxy_async_smem();
       mbar_arrive(&bars[kPhi + st]);
     }
-    if (ok && warp < 6) {
-      const bool got = mbar_wait(&bars[kAcc], 0, ab);
-      if (!__any_sync(0xffffffffu, !got)) {
-        tc_fence_after();
-        const uint32_t quarter = warp & 3;
-        const int a = quarter * 32 + lane;  // TMEM lane = head_dim slot of phi(k)
-        float* dst = p.parts + (((size_t)part * g.B + b) * g.H + h) * (size_t)(D + 1) * D;
+  } else {
+    // ------------------------------------------------------------ read-out of finished pieces
+    const uint32_t quarter = warp & 3;
+    const int a = quarter * 32 + lane;  // TMEM lane = head_dim slot of phi(k)
+    int piece = 0;
+    for (int i = 0; i < ntiles; ++i) {
+      if (!piece_ends(t_begin + i, t_end, sp)) continue;
+      const int buf = piece & 1;
+      const bool got = mbar_wait(&bars[kAccFull + buf], (piece >> 1) & 1, ab);
+      if (__any_sync(0xffffffffu, !got)) break;
+      tc_fence_after();
+      const SbTile tl = sb_tile(t_begin + i, g, sp);
+      // this CTA's contributor index within the segment
+      const long long seg_first = (long long)tl.bh * sp.tiles_per_bh + sp.seg_tile0[tl.seg];
+      const int u = (int)blockIdx.x - sb_cta_of(seg_first, sp);
+      float* dst = p.parts + sb_slot(tl.bh, tl.seg, u, sp) * (long long)(D + 1) * D;
+      const uint32_t acc = tmem + buf * L::kAccCols;
 #pragma unroll
-        for (int i = 0; i < kCols / 16; ++i) {
-          uint32_t r[16];
-          tmem_ld16(tmem_addr(tmem, quarter * 32, 16 * i), r);
-          tmem_wait_ld();
-          if (a < D) {
-            if (16 * i < D) {
+      for (int c = 0; c < L::kCols / 16; ++c) {
+        uint32_t r[16];
+        tmem_ld16(tmem_addr(acc, quarter * 32, 16 * c), r);
+        tmem_wait_ld();
+        if (a < D) {
+          if (16 * c < D) {
 #pragma unroll
-              for (int e = 0; e < 16; ++e) dst[(size_t)(16 * i + e) * D + a] = __uint_as_float(r[e]);
-            } else {
-              dst[(size_t)D * D + a] = __uint_as_float(r[0]);  // z
-            }
+            for (int e = 0; e < 16; ++e) dst[(size_t)(16 * c + e) * D + a] = __uint_as_float(r[e]);
+          } else {
+            dst[(size_t)D * D + a] = __uint_as_float(r[0]);  // z
           }
         }
       }
+      tc_fence_before();
+      mbar_arrive(&bars[kAccEmpty + buf]);
+      ++piece;
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 1) {
-    // every MMA of this CTA completed (kAcc) before the columns are released
-    mbar_drain(&bars[kAcc], 0);
-    tmem_dealloc(tmem, kAlloc);
+    // every MMA of this CTA completed (kDone) before the columns are released
+    mbar_drain(&bars[kDone], 0);
+    tmem_dealloc(tmem, 2 * L::kAccCols);
   }
 }
 
 cudaError_t launch_state_build(const Maps& m, const K1Params& p, cudaStream_t st) {
-  dim3 grid(p.g.B * p.g.H, p.g.n_parts);
-  if (p.g.n_parts == 0) return cudaSuccess;
+  // one CTA even without tiles: it zeroes the scan counter
+  const int grid = p.sp.grid > 0 ? p.sp.grid : 1;
   if (p.g.Dp == 128) {
     const int smem = K1Layout<128>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(k1_state_build<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

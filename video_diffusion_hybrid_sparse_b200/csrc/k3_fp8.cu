@@ -15,12 +15,16 @@
 //    cancels in o_s = v_scale * O / l.
 // V enters transposed (rows = head_dim, keys contiguous), so both operands of
 // P.V are K-major.
+#include "k3_common.cuh"
 #include "kernels.h"
+#include "scan.cuh"
 #include "sm100.cuh"
 
 namespace vdn {
 
 namespace {
+
+using namespace k3;
 
 template <int D>
 struct K3Layout {
@@ -38,10 +42,7 @@ struct K3Layout {
 // work per KV tile halves and the exponential unit is the tighter limit, so
 // one pair in eight goes to the FMA pipe (measured 1.7 % faster at 768p than
 // none, and than one in four).
-#ifndef VDN_FP8_POLY_EVERY
-#define VDN_FP8_POLY_EVERY 8
-#endif
-constexpr int kPolyEvery = VDN_FP8_POLY_EVERY;
+constexpr int kPolyEvery = 8;
 
 // two fp32 to e4m3 (round to nearest even, saturate), a in the low byte
 __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
@@ -55,56 +56,7 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&r)[4])
                "r"(r[2]), "r"(r[3])
                : "memory");
 }
-__host__ __device__ constexpr bool poly_pair(int e) {
-  return kPolyEvery > 0 && (e % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
-}
-
-// P of one tile can be handed to the MMA warp in kPParts column groups, so that
-// the P·V products of the first keys run while the later keys are
-// exponentiated.  One group is fastest on B200 (2 and 4 add MMA-warp waits
-// that cost more than the overlap gains).
-#ifndef VDN_P_PARTS
-#define VDN_P_PARTS 1
-#endif
-constexpr int kPParts = VDN_P_PARTS;
-static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P parts");
-
-struct Item {
-  int b, h, c, pair, ntiles;
-  int row0;   // first query row of the item within the batch
-  int nrows;  // rows of the item's query segment from row0 on (the tiles mask rows past it)
-};
-
-__device__ __forceinline__ Item decode_item(int item, const K3Params& p) {
-  const Geom& g = p.g;
-  // segment k with seg_item0[k] <= item < seg_item0[k + 1]
-  int lo = 0, hi = p.n_segs - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (p.seg_item0[mid] <= item) lo = mid;
-    else hi = mid - 1;
-  }
-  const QSeg sg = p.segs[lo];
-  const int n_pairs = (sg.nrows + 2 * kBlockM - 1) / (2 * kBlockM);
-  Item it;
-  int rem = item - p.seg_item0[lo];
-  const int per_b = g.H * n_pairs;
-  it.b = rem / per_b;
-  rem -= it.b * per_b;
-  it.h = rem / n_pairs;
-  it.pair = rem - it.h * n_pairs;
-  it.c = sg.c;
-  it.row0 = sg.row0 + it.pair * 2 * kBlockM;
-  it.nrows = sg.nrows - it.pair * 2 * kBlockM;
-  it.ntiles = it.nrows > kBlockM ? 2 : 1;
-  return it;
-}
-
-// Barrier slots.
-enum {
-  kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = 4, kVFull = 6, kVEmpty = 8,
-  kSFull = 10, kPFull = 12, kOFull = 12 + 2 * kPParts, kDone = kOFull + 2, kNumBars = kDone + 1
-};
+__host__ __device__ constexpr bool poly_pair(int e) { return e % kPolyEvery == kPolyEvery - 1; }
 
 }  // namespace
 
@@ -136,7 +88,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars[kSFull + t], 1);
-      for (int part = 0; part < kPParts; ++part) mbar_init(&bars[kPFull + 2 * part + t], kBlockM);
+      mbar_init(&bars[kPFull + t], kBlockM);
       mbar_init(&bars[kOFull + t], 1);
     }
     mbar_init(&bars[kDone], 1);
@@ -219,16 +171,13 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk) mma_ss_f8(d_tmem, qd + 2 * kk, kd + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
       };
-      // O_t += P_t·V over the keys of P part `part`
-      auto issue_pv = [&](int t, int st, int part, bool acc) {
+      // O_t += P_t·V over the 128 keys of the tile
+      auto issue_pv = [&](int t, int st, bool acc) {
         const uint32_t d_tmem = tmem + 256 + t * D;
         const uint64_t vd = v_desc0 + (uint64_t)((st * L::kTile) >> 4);
-        constexpr int kPer = kBlockN / 32 / kPParts;
 #pragma unroll
-        for (int k = 0; k < kPer; ++k) {
-          const int kk = part * kPer + k;  // 32 keys: 8 TMEM columns of P, 32 bytes of a V^T row
+        for (int kk = 0; kk < kBlockN / 32; ++kk)  // 32 keys: 8 TMEM columns of P, 32 bytes of a V^T row
           mma_ts_f8(d_tmem, tmem + t * 128 + kk * 8, vd + 2 * kk, idesc_pv, (acc || kk > 0) ? 1u : 0u);
-        }
       };
 
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++item_cnt) {
@@ -251,12 +200,9 @@ __global__ void __launch_bounds__(384, 1)
           const bool has_next = j + 1 < nkv;
           if (!mbar_wait(&bars[kVFull + st], (kv_cnt / L::kStages) & 1, ab)) { ok = false; break; }
           for (int t = 0; t < it.ntiles; ++t) {
-            for (int part = 0; part < kPParts; ++part) {
-              if (!mbar_wait(&bars[kPFull + 2 * part + t], p_cnt[t] & 1, ab)) { ok = false; break; }
-              tc_fence_after();
-              issue_pv(t, st, part, j > 0);
-            }
-            if (!ok) break;
+            if (!mbar_wait(&bars[kPFull + t], p_cnt[t] & 1, ab)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(t, st, j > 0);
             ++p_cnt[t];
             if (!has_next) mma_commit(&bars[kOFull + t]);
             if (has_next) {
@@ -280,7 +226,11 @@ __global__ void __launch_bounds__(384, 1)
       mma_commit(&bars[kDone]);
       mbar_drain(&bars[kDone], 0);
     }
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ linear-branch scan (no barriers)
+    if (p.do_scan)
+      scan_range(p.scan, (long long)blockIdx.x * 64 + (threadIdx.x - 64), (long long)gridDim.x * 64);
+  } else {
     // ------------------------------------------------------------ softmax warpgroups
     const int t = (warp - 4) >> 2;
     const uint32_t quarter = warp & 3;
@@ -385,27 +335,24 @@ __global__ void __launch_bounds__(384, 1)
               else pk[e >> 1] = pr;
             }
             tmem_st4(tmem_addr(tmem, lane_base, t * 128 + 4 * i), pk);
-            if ((i + 1) % (8 / kPParts) == 0) {
-              const int part = (i + 1) / (8 / kPParts) - 1;
-              if (part == 0 && rescale) {
-                // O_t is quiescent here: S_t(j) completing implies PV_t(j-1)
-                // completed, and PV_t(j) starts only after this part arrives.
+          }
+          if (rescale) {
+            // O_t is quiescent here: S_t(j) completing implies PV_t(j-1)
+            // completed, and PV_t(j) starts only after P_t(j) is handed over.
 #pragma unroll 1
-                for (int c = 0; c < D / 16; ++c) {
-                  uint32_t o[16];
-                  const uint32_t ta = tmem_addr(tmem, lane_base, 256 + t * D + 16 * c);
-                  tmem_ld16(ta, o);
-                  tmem_wait_ld();
+            for (int c = 0; c < D / 16; ++c) {
+              uint32_t o[16];
+              const uint32_t ta = tmem_addr(tmem, lane_base, 256 + t * D + 16 * c);
+              tmem_ld16(ta, o);
+              tmem_wait_ld();
 #pragma unroll
-                  for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                  tmem_st16(ta, o);
-                }
-              }
-              tmem_wait_st();
-              tc_fence_before();
-              mbar_arrive(&bars[kPFull + 2 * part + t]);
+              for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st16(ta, o);
             }
           }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&bars[kPFull + t]);
           {
             float l0, l1, l2, l3;
             f32x2_unpack(lsum0, l0, l1);

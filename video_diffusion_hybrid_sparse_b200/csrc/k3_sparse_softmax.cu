@@ -8,7 +8,7 @@
 //    one (batch, head, query segment), a segment being the rows of one chunk
 //    (under the GLOBAL anchor reading the rows of frames 0 and F-1 are
 //    segments of their own whose key set is every frame); items are handed
-//    out statically in an order sorted by KV tile count (longest first);
+//    out statically, (batch, head)-major (k3_common.cuh says why);
 //  * only the KV tiles of the item's key set are enumerated: at most three
 //    merged video token ranges plus the text range, 128 keys per tile; the
 //    last tile of a range is masked past the range end;
@@ -20,21 +20,37 @@
 //    (warp w reads TMEM lanes 32*(w%4)..+31); each thread owns one query row
 //    (TMEM lane), so row max and row sum are in-thread; P is written back as
 //    bf16 over the first half of S's columns;
-//  * online softmax with a lazy rescale: the running max only moves (and O is
-//    rescaled in TMEM) when a tile's max exceeds it by more than 8 in log2
-//    units; the final 1/l is applied in the epilogue;
-//  * TMEM: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
+//  * TMEM: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D);
+//  * when asked to, warps 2-3 (idle in the attention itself) and, after their
+//    last item, the softmax warps run the forward/backward scan of the linear
+//    branch (scan.cuh), taking units from a counter in the workspace (zeroed
+//    by the state build), so CTAs that finish their items early do most of
+//    the scan's tail.
+//
+// Online softmax.  The running max m moves only when a tile's max exceeds it
+// by more than 8 (log2 units; O is then rescaled in TMEM and the final 1/l
+// is applied in the epilogue), so P <= 2^8.  Of every eight key pairs, the
+// pairs in kEmuPairs get 2^x from a cubic on the FMA pipe (exp2x2_fma) and
+// the others from the special-function unit: at head_dim 128 a 128-key tile
+// costs the SFU as many cycles as the tensor core, so moving part of the
+// exponentials to the FMA pipe leaves the SFU slack to absorb the hand-offs
+// between the roles.  Masked keys (past the end of a key range) get s = -inf:
+// a weight of 0 from the SFU, below 2^-126 from the FMA-pipe form.
 //
 // The MMA issue order per KV tile j is PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), so
 // the tensor core works on one tile while the other tile's softmax runs.  A
 // commit after S_t(j+1) also covers PV_t(j), so when the softmax of tile t sees
 // S_t(j+1) its O_t is quiescent and may be rescaled.
+#include "k3_common.cuh"
 #include "kernels.h"
+#include "scan.cuh"
 #include "sm100.cuh"
 
 namespace vdn {
 
 namespace {
+
+using namespace k3;
 
 template <int D>
 struct K3Layout {
@@ -47,70 +63,51 @@ struct K3Layout {
   static constexpr int kBytes = kBar + 256 + 1024;  // + barriers + alignment slack
 };
 
-// With kPolyEvery = n > 0, one column pair in n is exponentiated on the FMA
-// pipe instead of the special-function unit.  Off by default: on B200 the
-// FMA-pipe form costs more cycles per step than it saves on the MUFU (the
-// softmax warps are latency-bound, and the extra instructions lower the
-// clock under the power cap).
-#ifndef VDN_POLY_EVERY
-#define VDN_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = VDN_POLY_EVERY;
-__host__ __device__ constexpr bool poly_pair(int e) {
-  return kPolyEvery > 0 && (e % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
-}
+constexpr int kThreads = 384;  // warp 0 loads, warp 1 MMA, warps 2-3 scan, warps 4-11 softmax
 
-// P of one tile can be handed to the MMA warp in kPParts column groups, so that
-// the P·V products of the first keys run while the later keys are
-// exponentiated.  One group is fastest on B200 (2 and 4 add MMA-warp waits
-// that cost more than the overlap gains).
-#ifndef VDN_P_PARTS
-#define VDN_P_PARTS 1
-#endif
-constexpr int kPParts = VDN_P_PARTS;
-static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P parts");
+// Key pairs (bit e of each group of eight) exponentiated on the FMA pipe.
+constexpr uint32_t kEmuPairs = 0x0u;
 
-struct Item {
-  int b, h, c, pair, ntiles;
-  int row0;   // first query row of the item within the batch
-  int nrows;  // rows of the item's query segment from row0 on (the tiles mask rows past it)
-};
-
-__device__ __forceinline__ Item decode_item(int item, const K3Params& p) {
-  const Geom& g = p.g;
-  // segment k with seg_item0[k] <= item < seg_item0[k + 1]
-  int lo = 0, hi = p.n_segs - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (p.seg_item0[mid] <= item) lo = mid;
-    else hi = mid - 1;
+// Exponentials of one 16-key group: P (bf16 pairs) and the row sum (two
+// packed partial sums).
+__device__ __forceinline__ void exp_group(const uint32_t* s, uint64_t sl2x2, uint64_t negm, uint32_t (&pk)[8],
+                                          uint64_t& l0, uint64_t& l1) {
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const uint64_t x = f32x2_fma(f32x2_pack(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), sl2x2, negm);
+    uint64_t pp;
+    if ((kEmuPairs >> e) & 1u) {
+      pp = exp2x2_fma(x);
+    } else {
+      float x0, x1;
+      f32x2_unpack(x, x0, x1);
+      pp = f32x2_pack(ex2_approx(x0), ex2_approx(x1));
+    }
+    if (e & 1) l1 = f32x2_add(l1, pp);
+    else l0 = f32x2_add(l0, pp);
+    float p0, p1;
+    f32x2_unpack(pp, p0, p1);
+    pk[e] = pack_bf16x2(p0, p1);
   }
-  const QSeg sg = p.segs[lo];
-  const int n_pairs = (sg.nrows + 2 * kBlockM - 1) / (2 * kBlockM);
-  Item it;
-  int rem = item - p.seg_item0[lo];
-  const int per_b = g.H * n_pairs;
-  it.b = rem / per_b;
-  rem -= it.b * per_b;
-  it.h = rem / n_pairs;
-  it.pair = rem - it.h * n_pairs;
-  it.c = sg.c;
-  it.row0 = sg.row0 + it.pair * 2 * kBlockM;
-  it.nrows = sg.nrows - it.pair * 2 * kBlockM;
-  it.ntiles = it.nrows > kBlockM ? 2 : 1;
-  return it;
 }
 
-// Barrier slots.
-enum {
-  kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = 4, kVFull = 6, kVEmpty = 8,
-  kSFull = 10, kPFull = 12, kOFull = 12 + 2 * kPParts, kDone = kOFull + 2, kNumBars = kDone + 1
-};
+// Scan units taken 32 at a time (one per lane) from the workspace counter
+// until none is left.
+__device__ __forceinline__ void scan_dynamic(const K3Params& p, uint32_t lane) {
+  const long long units = scan_units(p.g);
+  while (true) {
+    long long base = 0;
+    if (lane == 0) base = (long long)atomicAdd(p.scan_counter, 32ull);
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (base >= units) break;
+    if (base + lane < units) scan_unit(p.scan, base + lane);
+  }
+}
 
 }  // namespace
 
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     k3_sparse_softmax(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_tk,
                       const __grid_constant__ CUtensorMap tm_tv, const __grid_constant__ K3Params p) {
@@ -136,14 +133,14 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars[kSFull + t], 1);
-      for (int part = 0; part < kPParts; ++part) mbar_init(&bars[kPFull + 2 * part + t], kBlockM);
+      mbar_init(&bars[kPFull + t], kBlockM);
       mbar_init(&bars[kOFull + t], 1);
     }
     mbar_init(&bars[kDone], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 2) {
+  if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -223,17 +220,14 @@ __global__ void __launch_bounds__(384, 1)
           mma_ss(d_tmem, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
-      // O_t += P_t·V over the keys of P part `part`
-      auto issue_pv = [&](int t, int st, int part, bool acc) {
+      // O_t += P_t·V over the 128 keys of the tile
+      auto issue_pv = [&](int t, int st, bool acc) {
         const uint32_t d_tmem = tmem + 256 + t * D;
         const uint64_t vd = v_desc0 + (uint64_t)((st * L::kTile) >> 4);
-        constexpr int kPer = kBlockN / 16 / kPParts;
 #pragma unroll
-        for (int k = 0; k < kPer; ++k) {
-          const int kk = part * kPer + k;
+        for (int kk = 0; kk < kBlockN / 16; ++kk)
           mma_ts(d_tmem, tmem + t * 128 + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
                  (acc || kk > 0) ? 1u : 0u);
-        }
       };
 
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++item_cnt) {
@@ -256,12 +250,9 @@ __global__ void __launch_bounds__(384, 1)
           const bool has_next = j + 1 < nkv;
           if (!mbar_wait(&bars[kVFull + st], (kv_cnt / L::kStages) & 1, ab)) { ok = false; break; }
           for (int t = 0; t < it.ntiles; ++t) {
-            for (int part = 0; part < kPParts; ++part) {
-              if (!mbar_wait(&bars[kPFull + 2 * part + t], p_cnt[t] & 1, ab)) { ok = false; break; }
-              tc_fence_after();
-              issue_pv(t, st, part, j > 0);
-            }
-            if (!ok) break;
+            if (!mbar_wait(&bars[kPFull + t], p_cnt[t] & 1, ab)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(t, st, j > 0);
             ++p_cnt[t];
             if (!has_next) mma_commit(&bars[kOFull + t]);
             if (has_next) {
@@ -285,16 +276,21 @@ __global__ void __launch_bounds__(384, 1)
       mma_commit(&bars[kDone]);
       mbar_drain(&bars[kDone], 0);
     }
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ forward/backward scan
+    if (p.do_scan) scan_dynamic(p, lane);
+  } else {
     // ------------------------------------------------------------ softmax warpgroups
     const int t = (warp - 4) >> 2;
     const uint32_t quarter = warp & 3;
     const int row = quarter * 32 + lane;  // query row of the tile == TMEM lane
     const uint32_t lane_base = quarter * 32;
     const float sl2 = p.scale_log2;
+    const uint64_t sl2x2 = f32x2_pack(sl2, sl2);
     uint32_t s_cnt = 0, o_cnt = 0;
+    bool ok = true;
 
-    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       // only the key set and the tile count live across the KV loop; the
       // epilogue decodes the item again (fewer registers held in the loop)
       int seg_c, ntiles;
@@ -305,120 +301,90 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (t >= ntiles) continue;
       float m_run = 0.f, l_run = 0.f;
-      bool ok = true;
       // keys left in the current key range (video ranges, then text); only
       // these scalars live across the loop, the ranges are re-derived at
       // range ends
       const int nkv = seg_kv_tiles(seg_c, g);
       int range = 0, left = seg_range_len(seg_c, g, 0);
-      {
-        for (int j = 0; j < nkv; ++j) {
-          while (left == 0) left = seg_range_len(seg_c, g, ++range);
-          const int n_valid = min(kBlockN, left);
-          left -= n_valid;
-          const bool got = mbar_wait(&bars[kSFull + t], s_cnt & 1, ab);
-          if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
-          ++s_cnt;
-          tc_fence_after();
-          uint32_t s[128];
+      for (int j = 0; j < nkv; ++j) {
+        while (left == 0) left = seg_range_len(seg_c, g, ++range);
+        const int n_valid = min(kBlockN, left);
+        left -= n_valid;
+        const bool got = mbar_wait(&bars[kSFull + t], s_cnt & 1, ab);
+        if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
+        ++s_cnt;
+        tc_fence_after();
+        const uint32_t s_addr = tmem_addr(tmem, lane_base, t * 128);  // S_t, then P_t over its first half
+        uint32_t s[128];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t (&chunk)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32 * i]);
-            tmem_ld32(tmem_addr(tmem, lane_base, t * 128 + 32 * i), chunk);
-          }
-          tmem_wait_ld();
-          if (n_valid < kBlockN) {
+        for (int i = 0; i < 4; ++i) tmem_ld32(s_addr + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * i]));
+        tmem_wait_ld();
+        if (n_valid < kBlockN) {
 #pragma unroll
-            for (int i = 0; i < 128; ++i)
-              if (i >= n_valid) s[i] = __float_as_uint(-INFINITY);
-          }
-          // row max: four independent fmax3 chains
-          float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+          for (int i = 0; i < 128; ++i)
+            if (i >= n_valid) s[i] = __float_as_uint(-INFINITY);
+        }
+        // row max: four independent fmax3 chains
+        float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < 128; i += 8) {
-            a0 = fmax3(a0, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
-            a1 = fmax3(a1, __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
-            a2 = fmax3(a2, __uint_as_float(s[i + 4]), __uint_as_float(s[i + 5]));
-            a3 = fmax3(a3, __uint_as_float(s[i + 6]), __uint_as_float(s[i + 7]));
-          }
-          const float mx = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
-          const float mxs = mx * sl2;
-          // lazy rescale: move the running max only when this tile's max is
-          // more than 2^8 above it (O is rescaled below, once P is stored)
-          float alpha = 1.0f;
-          bool rescale = false;
-          if (j == 0) {
+        for (int i = 0; i < 128; i += 8) {
+          a0 = fmax3(a0, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
+          a1 = fmax3(a1, __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
+          a2 = fmax3(a2, __uint_as_float(s[i + 4]), __uint_as_float(s[i + 5]));
+          a3 = fmax3(a3, __uint_as_float(s[i + 6]), __uint_as_float(s[i + 7]));
+        }
+        const float mxs = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * sl2;
+        // lazy rescale: move the running max only when this tile's max is
+        // more than 2^8 above it (O is rescaled below, once P is stored)
+        float alpha = 1.0f;
+        bool rescale = false;
+        if (j == 0) {
+          m_run = mxs;
+        } else {
+          const bool need = mxs > m_run + 8.0f;
+          rescale = __any_sync(0xffffffffu, need);
+          if (need) {
+            alpha = ex2_approx(m_run - mxs);
             m_run = mxs;
-          } else {
-            const bool need = mxs > m_run + 8.0f;
-            rescale = __any_sync(0xffffffffu, need);
-            if (need) {
-              alpha = ex2_approx(m_run - mxs);
-              m_run = mxs;
-            }
-          }
-          l_run *= alpha;
-          // p = 2^(s * scale * log2(e) - m): the exponent argument and the
-          // row sum in packed f32x2; P goes to TMEM 8 columns (16 keys) at a
-          // time, which keeps the live registers under the 168 of a 384-thread
-          // CTA (no spills).
-          const uint64_t sl2x2 = f32x2_pack(sl2, sl2);
-          const uint64_t negm = f32x2_pack(-m_run, -m_run);
-          uint64_t lsum0 = f32x2_pack(0.f, 0.f), lsum1 = lsum0;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            uint32_t pk[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const uint64_t sx = f32x2_pack(__uint_as_float(s[16 * i + 2 * e]), __uint_as_float(s[16 * i + 2 * e + 1]));
-              float x0, x1;
-              f32x2_unpack(f32x2_fma(sx, sl2x2, negm), x0, x1);
-              float p0, p1;
-              if (poly_pair(e)) {
-                p0 = exp2_fma(x0);
-                p1 = exp2_fma(x1);
-              } else {
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
-              }
-              if (e & 1) lsum1 = f32x2_add(lsum1, f32x2_pack(p0, p1));
-              else lsum0 = f32x2_add(lsum0, f32x2_pack(p0, p1));
-              pk[e] = pack_bf16x2(p0, p1);
-            }
-            tmem_st8(tmem_addr(tmem, lane_base, t * 128 + 8 * i), pk);
-            if ((i + 1) % (8 / kPParts) == 0) {
-              const int part = (i + 1) / (8 / kPParts) - 1;
-              if (part == 0 && rescale) {
-                // O_t is quiescent here: S_t(j) completing implies PV_t(j-1)
-                // completed, and PV_t(j) starts only after this part arrives.
-#pragma unroll 1
-                for (int c = 0; c < D / 16; ++c) {
-                  uint32_t o[16];
-                  const uint32_t ta = tmem_addr(tmem, lane_base, 256 + t * D + 16 * c);
-                  tmem_ld16(ta, o);
-                  tmem_wait_ld();
-#pragma unroll
-                  for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                  tmem_st16(ta, o);
-                }
-              }
-              tmem_wait_st();
-              tc_fence_before();
-              mbar_arrive(&bars[kPFull + 2 * part + t]);
-            }
-          }
-          {
-            float l0, l1, l2, l3;
-            f32x2_unpack(lsum0, l0, l1);
-            f32x2_unpack(lsum1, l2, l3);
-            l_run += (l0 + l1) + (l2 + l3);
           }
         }
+        // p = 2^(s * scale * log2(e) - m); P goes to TMEM 8 columns (16 keys)
+        // at a time, which keeps the live registers within the 168 of a
+        // 384-thread CTA
+        uint64_t l0 = f32x2_pack(0.f, 0.f), l1 = l0;
+        const uint64_t negm = f32x2_pack(-m_run, -m_run);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          uint32_t pk[8];
+          exp_group(&s[16 * i], sl2x2, negm, pk, l0, l1);
+          tmem_st8(s_addr + 8 * i, pk);
+        }
+        if (rescale) {
+          // O_t is quiescent here: S_t(j) completing implies PV_t(j-1)
+          // completed, and PV_t(j) starts only after P_t(j) is handed over.
+#pragma unroll 1
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t o[16];
+            const uint32_t ta = tmem_addr(tmem, lane_base, 256 + t * D + 16 * c);
+            tmem_ld16(ta, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st16(ta, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars[kPFull + t]);
+        float c0, c1, c2, c3;
+        f32x2_unpack(l0, c0, c1);
+        f32x2_unpack(l1, c2, c3);
+        l_run = l_run * alpha + ((c0 + c1) + (c2 + c3));
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue: o_s = O / l
       const bool got = mbar_wait(&bars[kOFull + t], o_cnt & 1, ab);
-      if (__any_sync(0xffffffffu, !got)) break;
+      if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
       ++o_cnt;
       tc_fence_after();
       const float inv_l = 1.0f / l_run;
@@ -444,12 +410,14 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
     }
+    // the scan's tail: warps that finish their items early take the remaining units
+    if (ok && p.do_scan) scan_dynamic(p, lane);
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem, 512);
+  if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 size_t k3_smem_bytes(int Dp) {
@@ -463,7 +431,7 @@ static cudaError_t launch_k3(const Maps& m, const K3Params& p, int grid, cudaStr
   const size_t smem = k3_smem_bytes(D);
   cudaError_t e = cudaFuncSetAttribute(k3_sparse_softmax<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k3_sparse_softmax<D><<<grid, 384, smem, st>>>(m.q, m.k, m.v, m.tk, m.tv, p);
+  k3_sparse_softmax<D><<<grid, kThreads, smem, st>>>(m.q, m.k, m.v, m.tk, m.tv, p);
   return cudaGetLastError();
 }
 
@@ -472,4 +440,3 @@ cudaError_t launch_sparse_softmax(const Maps& m, const K3Params& p, int grid, cu
 }
 
 }  // namespace vdn
-

@@ -345,7 +345,7 @@ __global__ void __launch_bounds__(kK4Threads, 1)
       }
       const bool got = mbar_wait(&bars[kAFull + s], (i >> 1) & 1, ab);
       if (workers_any(!got)) { ok = false; break; }
-      phi_tile_inplace(smem + L::kA + s * L::kATile, D / 64, 128, d, tid, kWorkers);
+      phi_tile_inplace<D / 64 * 1024 / kWorkers>(smem + L::kA + s * L::kATile, D / 64, 128, d, tid, kWorkers);
       fence_proxy_async_smem();
       mbar_arrive(&bars[kAReady + s]);
       if (item > first) ok = finish(item - 1, (i - 1) & 1);

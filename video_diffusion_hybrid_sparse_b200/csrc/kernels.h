@@ -9,6 +9,18 @@
 
 namespace vdn {
 
+// The forward/backward scan (scan.cuh): partials in, segment states, the
+// readout operands M_c and (optionally) the exported F_c / B_c out.
+struct ScanArgs {
+  Geom g;
+  StatePlan sp;
+  const float* parts;      // state-build partial slots [n_part_slots, Dp+1, Dp] fp32 (row Dp holds z)
+  float* segst;            // segment states [B * H * n_segs, Dp+1, Dp] fp32
+  uint8_t* mt;             // readout B-tiles (hi, lo) per (b, chunk, head)
+  float* export_fwd;       // optional [B, Nc, H, d+1, d]
+  float* export_bwd;
+};
+
 struct K3Params {
   Geom g;
   float scale_log2;        // softmax scale * log2(e)
@@ -16,28 +28,30 @@ struct K3Params {
   const float* fp8_amax;   // fp8 branch: [5][B][H] maxima of q, k, v, text_k, text_v
   int* status;
   int* record;             // timeout record (workspace), may be null
-  int n_items;             // sum over segments of B * H * pairs
-  int n_segs;
-  // query segments by decreasing KV tile count; items of segment k are
-  // [seg_item0[k], seg_item0[k + 1]), ordered (batch, head, pair)
+  int n_items;             // all work items
+  // Work items come in blocks of query segments; block k holds segments
+  // [blk_seg0[k], blk_seg0[k + 1]) and items [blk_item0[k], blk_item0[k + 1]),
+  // ordered (batch, head, segment, pair of 128-row query tiles).  seg_pair0
+  // is the running count of pairs over all segments (pairs of segment i are
+  // seg_pair0[i] .. seg_pair0[i + 1]).
+  int n_blocks;
+  int blk_seg0[kMaxSegs + 1];
+  int blk_item0[kMaxSegs + 1];
   QSeg segs[kMaxSegs];
-  int seg_item0[kMaxSegs + 1];
+  int seg_pair0[kMaxSegs + 1];
+  int do_scan;             // the kernel also runs the forward/backward scan (scan below)
+  unsigned long long* scan_counter;  // next scan unit to take (workspace; zeroed by the state build)
+  ScanArgs scan;
 };
 
 struct K1Params {
   Geom g;
-  float* parts;            // [n_parts, B, H, Dp+1, Dp] fp32; row Dp holds z
+  StatePlan sp;
+  float* parts;            // partial slots [n_part_slots, Dp+1, Dp] fp32; row Dp holds z
   int* status;
   int* record;             // timeout record (workspace), may be null
-  int inject_timeout;      // test only: CTA (0, 0) waits for a phase nothing completes (short limit)
-};
-
-struct K2Params {
-  Geom g;
-  const float* parts;
-  uint8_t* mt;             // readout B-tiles (hi, lo) per (b, chunk, head)
-  float* export_fwd;       // optional [B, Nc, H, d+1, d]
-  float* export_bwd;
+  int inject_timeout;      // test only: CTA 0 waits for a phase nothing completes (short limit)
+  unsigned long long* scan_counter;  // zeroed by CTA 0 for the scan of the softmax kernel that follows
 };
 
 struct K4Params {
@@ -64,7 +78,7 @@ struct Maps {
 cudaError_t launch_stage(const void* src, int fp32_in, __nv_bfloat16* dst, long long rows, int H, int d, int Dp,
                          cudaStream_t st);
 cudaError_t launch_state_build(const Maps& m, const K1Params& p, cudaStream_t st);
-cudaError_t launch_state_scan(const K2Params& p, cudaStream_t st);
+cudaError_t launch_state_scan(const ScanArgs& sa, cudaStream_t st);
 cudaError_t launch_sparse_softmax(const Maps& m, const K3Params& p, int grid, cudaStream_t st);
 // fp8 branch (head_dim 128): Maps of the e4m3 q, k, text_k ([rows, H * 128]
 // bytes) and of v, text_v transposed ([B * H * 128, tokens] bytes).

@@ -19,7 +19,9 @@ __device__ __forceinline__ float phi_f(float x) {
 // d_real become 0; every other element x becomes bf16(phi(x)).  Called by
 // nthreads threads with tid in [0, nthreads).  kB chunks per thread and
 // batch: all loads first, then compute and store, so the shared-memory round
-// trips of a thread overlap (fewer when the caller keeps other registers live).
+// trips of a thread overlap; with kB = nbox * 1024 / nthreads every thread
+// takes exactly its chunks in one batch (a larger kB computes phi of chunks
+// that are then not stored).
 template <int kB = 8>
 __device__ __forceinline__ void phi_tile_inplace(uint8_t* tile, int nbox, int n_valid, int d_real, int tid,
                                                  int nthreads) {

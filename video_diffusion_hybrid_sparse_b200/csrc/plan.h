@@ -27,7 +27,7 @@
 namespace vdn {
 
 constexpr int kMaxChunks = 256;     // chunk-order table carried in kernel parameters
-constexpr int kSliceTokens = 2048;  // tokens per state-build work item
+constexpr int kStateBuildCtas = 148;  // state-build ranges: one per SM of a B200
 constexpr int kBlockM = 128;        // query rows per tile
 constexpr int kBlockN = 128;        // keys per tile
 constexpr int kMaxSegs = kMaxChunks + 2;  // query segments (chunks, plus the anchor frames under GLOBAL)
@@ -39,10 +39,8 @@ struct Geom {
   long long N;              // F * P video tokens per batch
   int staged;               // inputs are converted/padded into the workspace first
   int fp32_io;              // q/k/v/text/gates/out are fp32
-  int n_slices;             // state-build slices per non-anchor frame
-  int n_video_parts;        // (F - |anchors|) * n_slices
-  int n_text_parts;         // ceil(T / kSliceTokens)
-  int n_parts;
+  int n_state_segs;         // state segments per (batch, head): chunks with a non-anchor frame, + text
+  long long n_part_slots;   // state-build partial slots: B * H * n_state_segs * cmax
   int rows_per_chunk;       // C * P query rows
   int n_pairs;              // work items of two 128-row query tiles per chunk
   int mt_rows;              // rows of one readout B-tile: Dp + 16 (values, z, zero padding)
@@ -50,7 +48,7 @@ struct Geom {
   float scale;              // softmax scale
   float eps;                // RMSNorm epsilon
   // workspace layout (byte offsets; each 1024-aligned)
-  size_t off_status, off_os, off_q, off_k, off_v, off_tk, off_tv, off_parts, off_mt, total;
+  size_t off_status, off_os, off_q, off_k, off_v, off_tk, off_tv, off_parts, off_segst, off_mt, total;
   int fp8;                  // softmax branch with e4m3 operands
   long long pitch_v8, pitch_t8;  // row pitches (bytes) of the transposed e4m3 v and text_v
   size_t off_q8, off_k8, off_vt8, off_tk8, off_tvt8, off_amax;
@@ -178,7 +176,100 @@ inline int query_segments(const Geom& g, QSeg* out) {
 VDN_HD int fwd_last_chunk(int c) { return c - 2; }
 VDN_HD int bwd_first_chunk(int c) { return c + 2; }
 
-// Frame of video state part p (parts ordered by non-anchor frame, then slice).
-VDN_HD int part_frame(int p, const Geom& g) { return 1 + p / g.n_slices; }
+// ---------------------------------------------------------------- state build plan
+//
+// The state build walks, for every (batch, head), the state segments in
+// order: one video segment per chunk that holds a non-anchor frame (its
+// non-anchor frames are consecutive token rows) and, when T > 0, the text.
+// A segment is cut into 128-token tiles; the tiles of all (batch, head)
+// pairs, (batch, head)-major, form one list that is split into `grid` equal
+// contiguous ranges, one per CTA (every CTA gets the same number of tiles,
+// +-1).  A CTA accumulates phi(K)^T [V | 1] over the run of its tiles that
+// falls in one segment and writes it as one partial; a segment gets one
+// partial from each CTA whose range meets it, in slots
+// seg_slot0(gseg) + 0, 1, ... (at most `cmax` per segment).
+
+constexpr int kMaxStateSegs = kMaxChunks + 1;  // video segments (one per chunk) + text
+
+struct StatePlan {
+  int n_segs;                         // segments per (batch, head)
+  int n_vsegs;                        // of which video (chunk) segments; the text segment is last
+  int seg_chunk[kMaxStateSegs];       // chunk of a video segment
+  int seg_row0[kMaxStateSegs];        // first token row within the batch (video rows, or text rows)
+  int seg_rows[kMaxStateSegs];        // token rows of the segment
+  int seg_tile0[kMaxStateSegs + 1];   // first tile of the segment within one (batch, head)
+  int tiles_per_bh;
+  int grid;                           // state-build CTAs (ranges)
+  int cmax;                           // partial slots per segment
+  long long total_tiles;              // B * H * tiles_per_bh
+};
+
+// CTA whose range holds global tile t: ranges start at floor(k * TT / G).
+VDN_HD int sb_cta_of(long long t, const StatePlan& sp) {
+  return (int)(((t + 1) * sp.grid - 1) / sp.total_tiles);
+}
+VDN_HD long long sb_range_start(int k, const StatePlan& sp) { return (long long)k * sp.total_tiles / sp.grid; }
+
+// Partial slot of contributor u (0, 1, ...) of segment s of (batch, head) bh.
+VDN_HD long long sb_slot(int bh, int s, int u, const StatePlan& sp) {
+  return ((long long)bh * sp.n_segs + s) * sp.cmax + u;
+}
+
+// Number of CTAs whose range meets segment s of bh (partials written for it).
+VDN_HD int sb_contributors(int bh, int s, const StatePlan& sp) {
+  const long long t0 = (long long)bh * sp.tiles_per_bh + sp.seg_tile0[s];
+  const long long t1 = (long long)bh * sp.tiles_per_bh + sp.seg_tile0[s + 1] - 1;
+  return sb_cta_of(t1, sp) - sb_cta_of(t0, sp) + 1;
+}
+
+// Host: the state-build plan of a problem (segments, tile ranges, slots).
+// Needs g.B, g.H, g.P, g.T, g.C, g.F, g.Nc.
+inline void build_state_plan(const Geom& g, StatePlan& sp) {
+  sp.n_segs = 0;
+  int tiles = 0;
+  for (int c = 0; c < g.Nc; ++c) {
+    // the chunk's frames [c*C, (c+1)*C) without the anchors 0 and F-1 are consecutive
+    const int f0 = c * g.C > 1 ? c * g.C : 1;
+    const int f1 = (c + 1) * g.C < g.F - 1 ? (c + 1) * g.C : g.F - 1;
+    if (f1 <= f0) continue;
+    const int n = sp.n_segs++;
+    sp.seg_chunk[n] = c;
+    sp.seg_row0[n] = f0 * g.P;
+    sp.seg_rows[n] = (f1 - f0) * g.P;
+    sp.seg_tile0[n] = tiles;
+    tiles += ceil_div(sp.seg_rows[n], 128);
+  }
+  sp.n_vsegs = sp.n_segs;
+  if (g.T > 0) {
+    const int n = sp.n_segs++;
+    sp.seg_chunk[n] = -1;
+    sp.seg_row0[n] = 0;
+    sp.seg_rows[n] = g.T;
+    sp.seg_tile0[n] = tiles;
+    tiles += ceil_div(g.T, 128);
+  }
+  sp.seg_tile0[sp.n_segs] = tiles;
+  sp.tiles_per_bh = tiles;
+  sp.total_tiles = (long long)g.B * g.H * tiles;
+  sp.grid = (int)(sp.total_tiles < kStateBuildCtas ? sp.total_tiles : kStateBuildCtas);
+  sp.cmax = 0;
+  if (sp.grid == 0) return;
+  for (int bh = 0; bh < g.B * g.H; ++bh)
+    for (int s = 0; s < sp.n_segs; ++s) {
+      const int n = sb_contributors(bh, s, sp);
+      if (n > sp.cmax) sp.cmax = n;
+    }
+}
+
+// Segment of local tile lt of a (batch, head) (binary search over seg_tile0).
+VDN_HD int sb_seg_of(int lt, const StatePlan& sp) {
+  int lo = 0, hi = sp.n_segs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (sp.seg_tile0[mid] <= lt) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
 
 }  // namespace vdn

@@ -93,6 +93,36 @@ __device__ __forceinline__ float exp2_fma(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+__device__ __forceinline__ uint64_t f32x2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^x of two values at once on the FMA pipe, packed f32x2 arithmetic: the
+// same reduction and polynomial as exp2_fma (x clamped at -126; n = round(x)
+// by the 1.5 * 2^23 addition, f = x - n in [-1/2, 1/2], 2^f by the fitted
+// cubic, 2^n added into the exponent field).  Ten instructions per pair;
+// valid for x <= 64.
+__device__ __forceinline__ uint64_t exp2x2_fma(uint64_t x) {
+  float x0, x1;
+  f32x2_unpack(x, x0, x1);
+  x = f32x2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t magic = f32x2_pack(12582912.0f, 12582912.0f);
+  const uint64_t t = f32x2_add(x, magic);   // n in the low mantissa bits
+  const uint64_t n = f32x2_sub(t, magic);   // round(x)
+  const uint64_t f = f32x2_sub(x, n);
+  uint64_t p = f32x2_fma(f32x2_pack(0.05517149344086647f, 0.05517149344086647f), f,
+                         f32x2_pack(0.24261093139648438f, 0.24261093139648438f));
+  p = f32x2_fma(p, f, f32x2_pack(0.6932609677314758f, 0.6932609677314758f));
+  p = f32x2_fma(p, f, f32x2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float p0, p1, t0, t1;
+  f32x2_unpack(p, p0, p1);
+  f32x2_unpack(t, t0, t1);
+  return f32x2_pack(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
+                    __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
+}
+
 // ------------------------------------------------------------------ abort / status
 
 // Status shared by the warps of one CTA.  A wait that runs out sets `abort`
@@ -166,6 +196,21 @@ static __device__ __noinline__ void record_timeout(const CtaAbort& ab, const voi
   r[kRecNs + 1] = (int)(ns >> 32);
   r[kRecSm] = sm_id();
   __threadfence();
+}
+
+// Named barrier `id` over `nthreads` threads (whole warps) that also ORs a
+// predicate: every participant leaves with the same answer.
+__device__ __forceinline__ bool bar_any(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 // ------------------------------------------------------------------ mbarrier
