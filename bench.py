@@ -64,8 +64,12 @@ def work(w):
     state = w.B * w.H * w.d * (w.d + 1) * 4
     k1 = 2 * (w.P * (w.F - anchors) + w.T) * w.B * w.H * w.d * e + (w.F - anchors + 1) * state
     k2 = (w.F - anchors + 1) * state + n_chunks * state
-    k4 = 5 * w.B * w.N * w.H * w.d * e + n_chunks * state
-    k3_bytes = (3 * w.B * w.N + 2 * w.B * w.T) * w.H * w.d * e + w.B * w.N * w.H * w.d * 2
+    # on the bf16 path with head_dim 64 or 128 the softmax kernel applies the
+    # softmax branch's gate: it reads g_s, and the readout reads q, the gated
+    # term and g_l and writes out (four tensors instead of five)
+    gated = w.dtype == "bf16" and w.d in (64, 128)
+    k4 = (4 if gated else 5) * w.B * w.N * w.H * w.d * e + n_chunks * state
+    k3_bytes = ((3 + (1 if gated else 0)) * w.B * w.N + 2 * w.B * w.T) * w.H * w.d * e + w.B * w.N * w.H * w.d * 2
     return dict(softmax_flops=softmax_flops, linear_flops=linear_flops, k1_bytes=k1, k2_bytes=k2, k4_bytes=k4,
                 k3_bytes=k3_bytes, linear_bytes=k1 + k2 + k4)
 

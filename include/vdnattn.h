@@ -171,8 +171,9 @@ VDN_API vdn_status vdn_plan_membership(const vdn_cfg* cfg, uint8_t* table);
 VDN_API vdn_status vdn_membership_device(const vdn_cfg* cfg, uint8_t* table_dev, void* stream);
 
 /* Whole call: staging (fp32 or head_dim 32 only), state build, sparse
- * softmax with the forward/backward scan in the same kernel, readout + merge,
- * all on stream.  out: [B, N, H, d] in dtype (and cfg->out_linear under
+ * softmax with the forward/backward scan (and, for bf16 with head_dim 64 or
+ * 128, the softmax branch's gate) in the same kernel, readout + merge, all on
+ * stream.  out: [B, N, H, d] in dtype (and cfg->out_linear under
  * VDN_OUTPUT_SPLIT). */
 VDN_API vdn_status vdn_hybrid_attn_fwd(const void* q, const void* k, const void* v,
                                const void* text_k, const void* text_v,
@@ -214,11 +215,17 @@ VDN_API vdn_status vdn_sparse_softmax(const void* q, const void* k, const void* 
                               const void* text_k, const void* text_v,
                               const vdn_cfg* cfg, void* stream);
 /* vdn_sparse_softmax and, in the same kernel, vdn_state_scan: must follow
- * vdn_state_build on the same workspace (stream order).  Errors as
+ * vdn_state_build on the same workspace (stream order).  gate_s (the
+ * softmax branch's gate logits, [B, N, H, d], or NULL): for bf16 tensors whose
+ * head_dim is 64 or 128, and without VDN_OUT_SOFTMAX_ONLY, the kernel stores
+ * sigmoid(gate_s) * o_s in place of o_s (the softmax branch's term of the
+ * gated merge; one rounding to bf16 either way) and notes so in the
+ * workspace, and vdn_readout_merge then takes that term as it is; otherwise
+ * o_s is stored and the readout applies the gate.  Errors as
  * vdn_sparse_softmax, plus VDN_ERR_INVALID_ARG for VDN_EXPORT_STATES without
- * export buffers. */
+ * export buffers and VDN_ERR_ALIGNMENT for a misaligned gate_s. */
 VDN_API vdn_status vdn_softmax_and_scan(const void* q, const void* k, const void* v,
-                                        const void* text_k, const void* text_v,
+                                        const void* text_k, const void* text_v, const void* gate_s,
                                         const vdn_cfg* cfg, void* stream);
 /* phi(Q) M_c readout, RMSNorm, gates and merge into out. */
 VDN_API vdn_status vdn_readout_merge(const void* q, const void* gate_s, const void* gate_l,

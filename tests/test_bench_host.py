@@ -27,7 +27,14 @@ def test_softmax_flops_match_oracle_pair_count(w):
 def test_768p_work_figures():
     wk = bench.work(BY_NAME["768p_bf16"])
     assert abs(wk["softmax_flops"] / 1e12 - 14.164) < 0.01
-    assert abs(wk["k4_bytes"] / 1e9 - 1.88) < 0.02
+    # the readout's bytes at 768p: q, sigmoid(g_s) * o_s (the softmax kernel
+    # applies that gate on the bf16 path), g_l read and out written (4 x 0.3716
+    # GB) plus the readout operands M_c (15 chunks x 24 heads x 128 x 129 fp32)
+    assert abs(wk["k4_bytes"] / 1e9 - (4 * 0.37159 + 0.02378)) < 0.002
+    # where the readout applies both gates (fp32 I/O): five tensors
+    tiny = bench.work(BY_NAME["tiny_fp32"])
+    w = BY_NAME["tiny_fp32"]
+    assert tiny["k4_bytes"] == 5 * w.N * w.H * w.d * 4 + w.F // w.C * w.H * w.d * (w.d + 1) * 4
 
 
 def _worker(rank, world, port, times, out):

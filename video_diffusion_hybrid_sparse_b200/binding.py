@@ -76,7 +76,7 @@ def library() -> ctypes.CDLL:
         lib.vdn_state_scan.argtypes = [C, P]
         lib.vdn_export_states.argtypes = [C, P, P, P]
         lib.vdn_sparse_softmax.argtypes = [P, P, P, P, P, C, P]
-        lib.vdn_softmax_and_scan.argtypes = [P, P, P, P, P, C, P]
+        lib.vdn_softmax_and_scan.argtypes = [P, P, P, P, P, P, C, P]
         lib.vdn_readout_merge.argtypes = [P, P, P, P, C, P]
         lib.vdn_hybrid_attn_fwd_static.argtypes = [P, P, P, P, P, P, P, P, C, P]
         lib.vdn_static_scratch_bytes.restype = ctypes.c_size_t
@@ -317,10 +317,14 @@ class Steps:
         _check(self.lib.vdn_sparse_softmax(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(tk), _ptr(tv),
                                            ctypes.byref(self.cfg), _stream(stream)), "vdn_sparse_softmax")
 
-    def softmax_and_scan(self, stream=None):
-        q, k, v, tk, tv = self.t[:5]
+    def softmax_and_scan(self, stream=None, gate=True):
+        """The softmax branch and the scan; with ``gate`` the kernel also
+        applies the softmax branch's gate (as the whole call does)."""
+        q, k, v, tk, tv, gs = self.t[:6]
         _check(self.lib.vdn_softmax_and_scan(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(tk), _ptr(tv),
-                                             ctypes.byref(self.cfg), _stream(stream)), "vdn_softmax_and_scan")
+                                             gs.data_ptr() if gate else None, ctypes.byref(self.cfg),
+                                             _stream(stream)),
+               "vdn_softmax_and_scan")
 
     def readout_merge(self, stream=None):
         q, gs, gl, out = self.t[0], self.t[5], self.t[6], self.t[7]

@@ -8,11 +8,23 @@
 #include <numeric>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "kernels.h"
 #include "vdnattn.h"
 
 namespace vdn {
 namespace {
+
+// NVTX range around the host-side launch of one step (the ranges a profiler
+// shows next to the kernels; without a profiler attached they cost a few
+// nanoseconds).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr int kMaxScanChunks = kMaxChunks;  // state segments carried in kernel parameters
 
@@ -225,6 +237,7 @@ vdn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? VDN_OK : VDN_E
 
 vdn_status step_stage(const vdn_cfg* cfg, const Geom& g, const void* q, const void* k, const void* v, const void* tk,
                       const void* tv, cudaStream_t st) {
+  NvtxRange nvtx("vdn:stage");
   if (!g.staged) return VDN_OK;
   const long long vrows = (long long)g.B * g.N, trows = (long long)g.B * g.T;
   cudaError_t e = launch_stage(q, g.fp32_io, reinterpret_cast<__nv_bfloat16*>(ws(cfg, g.off_q)), vrows, g.H, g.d, g.Dp, st);
@@ -243,7 +256,16 @@ unsigned long long* scan_counter_ptr(const vdn_cfg* cfg, const Geom& g) {
   return reinterpret_cast<unsigned long long*>(ws(cfg, g.off_status) + 128);
 }
 
+// Flag at byte 136 of the status slot, written by the softmax kernel: 1 when
+// o_s in the workspace holds sigmoid(g_s) * o_s.
+int* os_gated_ptr(const vdn_cfg* cfg, const Geom& g) { return reinterpret_cast<int*>(ws(cfg, g.off_status) + 136); }
+
+// The readout reads everything by TMA (bf16, head_dim without padding); only
+// then does the softmax kernel take the gate of its branch.
+bool tma_readout(const Geom& g) { return !g.fp32_io && g.d == g.Dp; }
+
 vdn_status step_state_build(const vdn_cfg* cfg, const Geom& g, const Srcs& s, cudaStream_t st) {
+  NvtxRange nvtx("vdn:state_build");
   K1Params p;
   p.g = g;
   build_state_plan(g, p.sp);
@@ -269,6 +291,7 @@ void make_scan_args(const vdn_cfg* cfg, const Geom& g, ScanArgs& sa) {
 }
 
 vdn_status step_state_scan(const vdn_cfg* cfg, const Geom& g, cudaStream_t st) {
+  NvtxRange nvtx("vdn:state_scan");
   ScanArgs sa;
   make_scan_args(cfg, g, sa);
   return cuda_status(launch_state_scan(sa, st));
@@ -301,9 +324,13 @@ void plan_items(const Geom& g, K3Params& p) {
   p.n_items = p.blk_item0[nb];
 }
 
-// The softmax branch; with do_scan, the kernel's otherwise idle warps also
-// run the forward/backward scan of the state partials in the workspace.
-vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s, cudaStream_t st, bool do_scan) {
+// The softmax branch; with do_scan, the kernel also runs the forward/backward
+// scan of the state partials in the workspace; with gate_s (bf16 tensors whose
+// head_dim needs no padding, not under VDN_OUT_SOFTMAX_ONLY), o_s is written
+// as sigmoid(gate_s) * o_s.
+vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s, cudaStream_t st, bool do_scan,
+                               const void* gate_s) {
+  NvtxRange nvtx("vdn:sparse_softmax");
   Maps m;
   if (!make_maps(m, g, s)) return VDN_ERR_CUDA;
   K3Params p;
@@ -341,6 +368,10 @@ vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s,
   plan_items(g, p);
   p.do_scan = do_scan ? 1 : 0;
   p.scan_counter = scan_counter_ptr(cfg, g);
+  p.os_gated = os_gated_ptr(cfg, g);
+  p.gate_s = (gate_s && tma_readout(g) && !g.fp8 && !(cfg->debug_flags & VDN_OUT_SOFTMAX_ONLY))
+                 ? static_cast<const __nv_bfloat16*>(gate_s)
+                 : nullptr;
   if (do_scan) make_scan_args(cfg, g, p.scan);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -351,6 +382,7 @@ vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s,
 
 vdn_status step_readout_merge(const vdn_cfg* cfg, const Geom& g, const Srcs& s, const void* gs, const void* gl,
                               void* out, cudaStream_t st) {
+  NvtxRange nvtx("vdn:readout_merge");
   Maps m;
   if (!make_maps(m, g, s)) return VDN_ERR_CUDA;
   K4Params p;
@@ -364,9 +396,10 @@ vdn_status step_readout_merge(const vdn_cfg* cfg, const Geom& g, const Srcs& s, 
   p.out_linear = cfg->output_mode == VDN_OUTPUT_SPLIT ? cfg->out_linear : nullptr;
   p.flags = cfg->debug_flags & (VDN_OUT_SOFTMAX_ONLY | VDN_OUT_LINEAR_ONLY | VDN_OUT_LINEAR_RAW);
   p.stall_ns = (cfg->debug_flags & VDN_STALL_READOUT_MMA) ? 50000 : 0;
+  p.os_gated = os_gated_ptr(cfg, g);
   p.status = status_ptr(cfg, g);
   p.record = record_ptr(cfg, g);
-  if (!g.fp32_io && g.d == g.Dp) {
+  if (tma_readout(g)) {
     // bf16 tensors without head_dim padding: every input tile by TMA
     MergeMaps mm;
     mm.q = m.q;
@@ -540,19 +573,20 @@ vdn_status vdn_sparse_softmax(const void* q, const void* k, const void* v, const
   s = check_inputs(cfg, g, {q, k, v}, {text_k, text_v});
   if (s != VDN_OK) return s;
   return step_sparse_softmax(cfg, g, kernel_srcs(cfg, g, q, k, v, text_k, text_v), static_cast<cudaStream_t>(stream),
-                             false);
+                             false, nullptr);
 }
 
 vdn_status vdn_softmax_and_scan(const void* q, const void* k, const void* v, const void* text_k, const void* text_v,
-                                const vdn_cfg* cfg, void* stream) {
+                                const void* gate_s, const vdn_cfg* cfg, void* stream) {
   Geom g;
   vdn_status s = make_geom(cfg, g);
   if (s != VDN_OK) return s;
   s = check_inputs(cfg, g, {q, k, v}, {text_k, text_v});
   if (s != VDN_OK) return s;
   if ((cfg->debug_flags & VDN_EXPORT_STATES) && (!cfg->export_fwd || !cfg->export_bwd)) return VDN_ERR_INVALID_ARG;
+  if (gate_s && (s = check_ptrs({gate_s})) != VDN_OK) return s;
   return step_sparse_softmax(cfg, g, kernel_srcs(cfg, g, q, k, v, text_k, text_v), static_cast<cudaStream_t>(stream),
-                             true);
+                             true, gate_s);
 }
 
 vdn_status vdn_readout_merge(const void* q, const void* gate_s, const void* gate_l, void* out, const vdn_cfg* cfg,
@@ -581,7 +615,7 @@ vdn_status vdn_hybrid_attn_fwd(const void* q, const void* k, const void* v, cons
   if (poison_ws(cfg, g, st) != cudaSuccess) return VDN_ERR_CUDA;
   if ((s = step_stage(cfg, g, q, k, v, text_k, text_v, st)) != VDN_OK) return s;
   if ((s = step_state_build(cfg, g, src, st)) != VDN_OK) return s;
-  if ((s = step_sparse_softmax(cfg, g, src, st, true)) != VDN_OK) return s;  // the scan runs inside
+  if ((s = step_sparse_softmax(cfg, g, src, st, true, gate_s)) != VDN_OK) return s;  // the scan runs inside
   return step_readout_merge(cfg, g, src, gate_s, gate_l, out, st);
 }
 
@@ -654,8 +688,10 @@ vdn_status vdn_hybrid_attn_fwd_host(const void* q, const void* k, const void* v,
     if ((s = step_stage(&c, g, dq, dk, dvv, dtk, dtv, st)) != VDN_OK) return finish(s);
   }
   if ((s = step_state_build(&c, g, src, st)) != VDN_OK) return finish(s);
+  // the softmax branch runs while the gates are still in flight, so here it
+  // leaves o_s ungated and the readout applies both gates
   if (cudaStreamWaitEvent(st, ev[2], 0) != cudaSuccess) return finish(VDN_ERR_CUDA);
-  if ((s = step_sparse_softmax(&c, g, src, st, true)) != VDN_OK) return finish(s);  // the scan runs inside
+  if ((s = step_sparse_softmax(&c, g, src, st, true, nullptr)) != VDN_OK) return finish(s);  // the scan runs inside
   if (cudaStreamWaitEvent(st, ev[3], 0) != cudaSuccess) return finish(VDN_ERR_CUDA);
   if ((s = step_readout_merge(&c, g, src, dv + h.gs, dv + h.gl, dv + h.out, st)) != VDN_OK) return finish(s);
   ce = cudaMemcpyAsync(out, dv + h.out, vid, cudaMemcpyDeviceToHost, st);

@@ -77,6 +77,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
 
+  if (threadIdx.x == 0 && blockIdx.x == 0 && p.os_gated) *p.os_gated = 0;  // o_s is left ungated
   if (threadIdx.x == 0) {
     mbar_init(&bars[kQFull], 1);
     mbar_init(&bars[kQEmpty], 1);

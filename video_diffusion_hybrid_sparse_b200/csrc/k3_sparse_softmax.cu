@@ -41,6 +41,8 @@
 // the tensor core works on one tile while the other tile's softmax runs.  A
 // commit after S_t(j+1) also covers PV_t(j), so when the softmax of tile t sees
 // S_t(j+1) its O_t is quiescent and may be rescaled.
+#include <type_traits>
+
 #include "k3_common.cuh"
 #include "kernels.h"
 #include "scan.cuh"
@@ -64,6 +66,9 @@ struct K3Layout {
 };
 
 constexpr int kThreads = 384;  // warp 0 loads, warp 1 MMA, warps 2-3 scan, warps 4-11 softmax
+constexpr uint32_t kLaunchRegs = 168;  // per thread at launch (65536 / 384, in steps of 8)
+constexpr uint32_t kLowRegs = 120;     // warpgroup 0
+constexpr uint32_t kHighRegs = 184;    // softmax warpgroups
 
 // Key pairs (bit e of each group of eight) exponentiated on the FMA pipe.
 constexpr uint32_t kEmuPairs = 0x0u;
@@ -149,13 +154,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const CtaAbort ab{abort_flag, p.status, p.record, 3};
+  // Register re-split between the warpgroups: the launch gives every thread
+  // kLaunchRegs; warpgroup 0 (loads, MMA issue, scan) hands registers to the
+  // two softmax warpgroups.  The re-split never asks for more than the launch
+  // holds (128 * kLowRegs + 256 * kHighRegs <= 384 * kLaunchRegs), or the
+  // increase would wait for registers that never come.
+  static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register re-split exceeds the launch");
 
   uint8_t* sQ = smem + L::kQ;
   uint8_t* sK = smem + L::kK;
   uint8_t* sV = smem + L::kV;
 
+  if (warp < 4) {
+  regs_dec<kLowRegs>();
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && blockIdx.x == 0 && p.os_gated) *p.os_gated = p.gate_s != nullptr;  // for the readout
     if (lane == 0) {
       uint32_t kv_cnt = 0, item_cnt = 0;
       bool ok = true;
@@ -276,10 +290,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&bars[kDone]);
       mbar_drain(&bars[kDone], 0);
     }
-  } else if (warp < 4) {
+  } else {
     // ------------------------------------------------------------ forward/backward scan
     if (p.do_scan) scan_dynamic(p, lane);
+  }
   } else {
+    regs_inc<kHighRegs>();
     // ------------------------------------------------------------ softmax warpgroups
     const int t = (warp - 4) >> 2;
     const uint32_t quarter = warp & 3;
@@ -298,6 +314,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Item it = decode_item(item, p);
         seg_c = it.c;
         ntiles = it.ntiles;
+        // the row's gate logits are read in the epilogue: bring them into L2 now
+        if (p.gate_s && t < ntiles && row < it.nrows - t * kBlockM) {
+          const __nv_bfloat16* gr =
+              p.gate_s + (((size_t)it.b * g.N + (size_t)(it.row0 + t * kBlockM + row)) * g.H + it.h) * D;
+#pragma unroll
+          for (int i = 0; i < D / 64; ++i) prefetch_l2(gr + 64 * i);
+        }
       }
       if (t >= ntiles) continue;
       float m_run = 0.f, l_run = 0.f;
@@ -315,50 +338,58 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++s_cnt;
         tc_fence_after();
         const uint32_t s_addr = tmem_addr(tmem, lane_base, t * 128);  // S_t, then P_t over its first half
-        uint32_t s[128];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) tmem_ld32(s_addr + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * i]));
-        tmem_wait_ld();
-        if (n_valid < kBlockN) {
-#pragma unroll
-          for (int i = 0; i < 128; ++i)
-            if (i >= n_valid) s[i] = __float_as_uint(-INFINITY);
-        }
-        // row max: four independent fmax3 chains
-        float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < 128; i += 8) {
-          a0 = fmax3(a0, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
-          a1 = fmax3(a1, __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
-          a2 = fmax3(a2, __uint_as_float(s[i + 4]), __uint_as_float(s[i + 5]));
-          a3 = fmax3(a3, __uint_as_float(s[i + 6]), __uint_as_float(s[i + 7]));
-        }
-        const float mxs = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * sl2;
-        // lazy rescale: move the running max only when this tile's max is
-        // more than 2^8 above it (O is rescaled below, once P is stored)
         float alpha = 1.0f;
         bool rescale = false;
-        if (j == 0) {
-          m_run = mxs;
-        } else {
-          const bool need = mxs > m_run + 8.0f;
-          rescale = __any_sync(0xffffffffu, need);
-          if (need) {
-            alpha = ex2_approx(m_run - mxs);
-            m_run = mxs;
-          }
-        }
-        // p = 2^(s * scale * log2(e) - m); P goes to TMEM 8 columns (16 keys)
-        // at a time, which keeps the live registers within the 168 of a
-        // 384-thread CTA
         uint64_t l0 = f32x2_pack(0.f, 0.f), l1 = l0;
-        const uint64_t negm = f32x2_pack(-m_run, -m_run);
+        // One KV tile: the row max over all 128 scores, then the exponentials.
+        // kMasked: the last tile of a key range, whose keys past n_valid get
+        // s = -inf (a weight of 0 from the SFU, below 2^-126 from the FMA-pipe
+        // form); the full tiles run a copy of the code without the masking.
+        auto tile = [&](auto masked_tag) {
+          constexpr bool kMasked = decltype(masked_tag)::value;
+          uint32_t s[128];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          uint32_t pk[8];
-          exp_group(&s[16 * i], sl2x2, negm, pk, l0, l1);
-          tmem_st8(s_addr + 8 * i, pk);
-        }
+          for (int i = 0; i < 4; ++i) tmem_ld32(s_addr + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * i]));
+          tmem_wait_ld();
+          if (kMasked) {
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+              if (i >= n_valid) s[i] = __float_as_uint(-INFINITY);
+          }
+          // row max: four independent fmax3 chains
+          float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < 128; i += 8) {
+            a0 = fmax3(a0, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
+            a1 = fmax3(a1, __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
+            a2 = fmax3(a2, __uint_as_float(s[i + 4]), __uint_as_float(s[i + 5]));
+            a3 = fmax3(a3, __uint_as_float(s[i + 6]), __uint_as_float(s[i + 7]));
+          }
+          const float mxs = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * sl2;
+          // lazy rescale: move the running max only when this tile's max is
+          // more than 2^8 above it (O is rescaled below, once P is stored)
+          if (j == 0) {
+            m_run = mxs;
+          } else {
+            const bool need = mxs > m_run + 8.0f;
+            rescale = __any_sync(0xffffffffu, need);
+            if (need) {
+              alpha = ex2_approx(m_run - mxs);
+              m_run = mxs;
+            }
+          }
+          // p = 2^(s * scale * log2(e) - m); P goes to TMEM 8 columns (16
+          // keys) at a time
+          const uint64_t negm = f32x2_pack(-m_run, -m_run);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            uint32_t pk[8];
+            exp_group(&s[16 * i], sl2x2, negm, pk, l0, l1);
+            tmem_st8(s_addr + 8 * i, pk);
+          }
+        };
+        if (n_valid < kBlockN) tile(std::true_type());
+        else tile(std::false_type());
         if (rescale) {
           // O_t is quiescent here: S_t(j) completing implies PV_t(j-1)
           // completed, and PV_t(j) starts only after P_t(j) is handed over.
@@ -383,29 +414,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue: o_s = O / l
+      // (times sigmoid(g_s) when the gate is given: the softmax branch's term
+      // of the gated merge; the gate logits were brought into L2 at the start
+      // of the item).
       const bool got = mbar_wait(&bars[kOFull + t], o_cnt & 1, ab);
       if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
       ++o_cnt;
       tc_fence_after();
-      const float inv_l = 1.0f / l_run;
       const Item it = decode_item(item, p);
       const int nrows = min(kBlockM, it.nrows - t * kBlockM);  // valid rows of this tile
-      __nv_bfloat16* dst = p.o_s + (((size_t)it.b * g.N + (size_t)(it.row0 + t * kBlockM + row)) * g.H + it.h) * D;
+      const size_t row_el = (((size_t)it.b * g.N + (size_t)(it.row0 + t * kBlockM + row)) * g.H + it.h) * D;
+      const bool gated = p.gate_s != nullptr;
+      const float inv_l = 1.0f / l_run;
+      __nv_bfloat16* dst = p.o_s + row_el;
 #pragma unroll
       for (int i = 0; i < D / 32; ++i) {
         uint32_t o[32];
+        uint4 gv[4];
+        if (gated && row < nrows) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) gv[v4] = __ldg(reinterpret_cast<const uint4*>(p.gate_s + row_el) + 4 * i + v4);
+        }
         tmem_ld32(tmem_addr(tmem, lane_base, 256 + t * D + 32 * i), o);
         tmem_wait_ld();
         if (row < nrows) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * i);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(o[8 * v4 + 0]) * inv_l, __uint_as_float(o[8 * v4 + 1]) * inv_l);
-            w.y = pack_bf16x2(__uint_as_float(o[8 * v4 + 2]) * inv_l, __uint_as_float(o[8 * v4 + 3]) * inv_l);
-            w.z = pack_bf16x2(__uint_as_float(o[8 * v4 + 4]) * inv_l, __uint_as_float(o[8 * v4 + 5]) * inv_l);
-            w.w = pack_bf16x2(__uint_as_float(o[8 * v4 + 6]) * inv_l, __uint_as_float(o[8 * v4 + 7]) * inv_l);
-            d4[v4] = w;
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(o[8 * v4 + e]) * inv_l;
+            if (gated) {
+              const uint4 gq = gv[v4];
+              const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                x[2 * e] *= sigmoid_tanh(bf16_lo(gw[e]));
+                x[2 * e + 1] *= sigmoid_tanh(bf16_hi(gw[e]));
+              }
+            }
+            d4[v4] = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                                pack_bf16x2(x[6], x[7]));
           }
         }
       }

@@ -10,12 +10,7 @@
 namespace vdn {
 namespace k4 {
 
-// sigmoid(x) = (1 + tanh(x / 2)) / 2 with the hardware tanh (one special-function op)
-__device__ __forceinline__ float sigmoid_f(float x) {
-  float t;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
-  return fmaf(0.5f, t, 0.5f);
-}
+__device__ __forceinline__ float sigmoid_f(float x) { return sigmoid_tanh(x); }
 
 template <bool FP32>
 __device__ __forceinline__ void store8(void* base, size_t idx, const float (&x)[8]) {

@@ -7,7 +7,9 @@
 // Same persistent walk as k4_readout_merge (CTA k keeps head k % H and takes
 // the 128-row tiles s, s + S, ... of stream s = k / H).  Per tile:
 //   * warp 0 (one thread) TMA-loads the q tile, and, one tile later, the
-//     tile's o_s, gate_s and gate_l tiles (128 rows x head_dim each); it
+//     tile's o_s and gate_l tiles (128 rows x head_dim each), and gate_s only
+//     when the softmax kernel left o_s ungated (o_s then holds
+//     sigmoid(g_s) * o_s when it was given the gate); it
 //     bulk-copies M_c (bf16 hi/lo readout operand) when the chunk changes and
 //     prefetches the next tiles into L2;
 //   * warp 1 (one thread): D = phi(Q) M_hi^T + phi(Q) M_lo^T (M = 128,
@@ -126,6 +128,9 @@ __global__ void __launch_bounds__(kTThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const CtaAbort ab{abort_flag, p.status, p.record, 4};
   auto row0_of = [&](const Item4& it) { return it.b * (int)g.N + it.c * g.rows_per_chunk + it.tile * 128; };
+  // o_s already holds sigmoid(g_s) * o_s (the softmax kernel was given the
+  // gate): g_s is then neither loaded nor applied
+  const bool gated = p.os_gated != nullptr && __ldg(p.os_gated) != 0;
 
   if (warp == 0) {
     // ------------------------------------------------------------ loads
@@ -157,18 +162,19 @@ __global__ void __launch_bounds__(kTThreads, 1)
           }
           for (int bx = 0; bx < D / 64; ++bx) {
             tma_prefetch_2d(&tm_os, it.h * D + bx * 64, row0_of(it));
-            tma_prefetch_2d(&tm_gs, it.h * D + bx * 64, row0_of(it));
+            if (!gated) tma_prefetch_2d(&tm_gs, it.h * D + bx * 64, row0_of(it));
             tma_prefetch_2d(&tm_gl, it.h * D + bx * 64, row0_of(it));
           }
         }
         if (i >= 1) {
           const Item4 it = decode4(i - 1, head, stream, n_streams, g, tiles);
           if (!mbar_wait(&bars[kTGEmpty], ((i - 1) & 1) ^ 1, ab)) { ok = false; break; }
-          mbar_expect_tx(&bars[kTGFull], (uint32_t)(3 * L::kTile));
+          mbar_expect_tx(&bars[kTGFull], (uint32_t)((gated ? 2 : 3) * L::kTile));
           for (int bx = 0; bx < D / 64; ++bx) {
             tma_load_2d(smem + L::kG + bx * 16384, &tm_os, &bars[kTGFull], it.h * D + bx * 64, row0_of(it));
-            tma_load_2d(smem + L::kG + L::kTile + bx * 16384, &tm_gs, &bars[kTGFull], it.h * D + bx * 64,
-                        row0_of(it));
+            if (!gated)
+              tma_load_2d(smem + L::kG + L::kTile + bx * 16384, &tm_gs, &bars[kTGFull], it.h * D + bx * 64,
+                          row0_of(it));
             tma_load_2d(smem + L::kG + 2 * L::kTile + bx * 16384, &tm_gl, &bars[kTGFull], it.h * D + bx * 64,
                         row0_of(it));
           }
@@ -267,16 +273,28 @@ __global__ void __launch_bounds__(kTThreads, 1)
 #pragma unroll
       for (int c8 = 0; c8 < D / 16; ++c8) {
         const int col = col0 + 8 * c8;
-        const uint4 vo = tile_piece(t_os, row, col), vs = tile_piece(t_gs, row, col), vl = tile_piece(t_gl, row, col);
+        const uint4 vo = tile_piece(t_os, row, col), vl = tile_piece(t_gl, row, col);
         const uint32_t ow[4] = {vo.x, vo.y, vo.z, vo.w};
-        const uint32_t sw[4] = {vs.x, vs.y, vs.z, vs.w};
         const uint32_t lw[4] = {vl.x, vl.y, vl.z, vl.w};
-        float os[8], gs[8], gl[8], rr[8];
+        float os[8], gl[8], rr[8];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           os[2 * k] = bf16_lo(ow[k]); os[2 * k + 1] = bf16_hi(ow[k]);
-          gs[2 * k] = bf16_lo(sw[k]); gs[2 * k + 1] = bf16_hi(sw[k]);
           gl[2 * k] = bf16_lo(lw[k]); gl[2 * k + 1] = bf16_hi(lw[k]);
+        }
+        // the softmax branch's gated term sigmoid(g_s) * o_s
+        float sterm[8];
+        if (gated) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) sterm[k] = os[k];
+        } else {
+          const uint4 vs = tile_piece(t_gs, row, col);
+          const uint32_t sw[4] = {vs.x, vs.y, vs.z, vs.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            sterm[2 * k] = sigmoid_f(bf16_lo(sw[k])) * os[2 * k];
+            sterm[2 * k + 1] = sigmoid_f(bf16_hi(sw[k])) * os[2 * k + 1];
+          }
         }
 #pragma unroll
         for (int k = 0; k < 8; ++k) rr[k] = r[8 * c8 + k] * inv_rms;
@@ -291,14 +309,14 @@ __global__ void __launch_bounds__(kTThreads, 1)
           float ol[8];
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            o[k] = sigmoid_f(gs[k]) * os[k];
+            o[k] = sterm[k];
             ol[k] = sigmoid_f(gl[k]) * rr[k];
           }
           if (row < nrows) store8<false>(p.out_linear, row_h * d + col, ol);
         } else {
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            const float merged = sigmoid_f(gs[k]) * os[k] + sigmoid_f(gl[k]) * rr[k];
+            const float merged = sterm[k] + sigmoid_f(gl[k]) * rr[k];
             o[k] = mode == 0 ? merged : (mode == 1 ? os[k] : rr[k]);
           }
         }

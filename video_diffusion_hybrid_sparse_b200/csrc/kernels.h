@@ -39,6 +39,8 @@ struct K3Params {
   int blk_item0[kMaxSegs + 1];
   QSeg segs[kMaxSegs];
   int seg_pair0[kMaxSegs + 1];
+  const __nv_bfloat16* gate_s;  // [B, N, H, Dp] or null: o_s is written as sigmoid(gate_s) * o_s
+  int* os_gated;           // workspace flag: 1 when o_s holds the gated term (read by the readout)
   int do_scan;             // the kernel also runs the forward/backward scan (scan below)
   unsigned long long* scan_counter;  // next scan unit to take (workspace; zeroed by the state build)
   ScanArgs scan;
@@ -65,6 +67,7 @@ struct K4Params {
   void* out_linear;        // SPLIT output: sigmoid(g_l) * r goes here, out gets sigmoid(g_s) * o_s
   int flags;
   int stall_ns;            // > 0: the MMA thread sleeps this long at each readout-operand change
+  const int* os_gated;     // workspace flag written by the softmax kernel: o_s already holds sigmoid(g_s) * o_s
   int* status;
   int* record;             // timeout record (workspace), may be null
 };

@@ -123,6 +123,13 @@ __device__ __forceinline__ uint64_t exp2x2_fma(uint64_t x) {
                     __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
 }
 
+// sigmoid(x) = (1 + tanh(x / 2)) / 2 with the hardware tanh (one special-function op)
+__device__ __forceinline__ float sigmoid_tanh(float x) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+  return fmaf(0.5f, t, 0.5f);
+}
+
 // ------------------------------------------------------------------ abort / status
 
 // Status shared by the warps of one CTA.  A wait that runs out sets `abort`
