@@ -476,6 +476,12 @@ def test_state_build_protocol(pieces):
     assert check(k1_roles(pieces)) > 0
 
 
+@pytest.mark.parametrize("pieces,stages", [([7], 6), ([2, 3, 2], 6), ([4, 5], 8)])
+def test_state_build_protocol_deep_pipeline(pieces, stages):
+    # the protocol does not depend on the number of stages
+    assert check(k1_roles(pieces, stages=stages)) > 0
+
+
 K3_SCHEDULES = [[(2, 1)], [(2, 3)], [(2, 4)], [(1, 2)], [(2, 2), (2, 1)], [(2, 1), (1, 2)], [(1, 1), (2, 2), (1, 1)],
                 [(2, 3), (1, 2), (2, 1)], [(2, 2), (2, 2), (2, 2)]]
 

@@ -175,15 +175,15 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 view [rows, H*Dp] (row pitch H*Dp*2 bytes), box 128 rows x 64
-// columns, 128-byte swizzle, zero fill out of bounds.
-bool make_map(CUtensorMap* m, const void* base, long long rows, int H, int Dp) {
+// 2-D bf16 view [rows, H*Dp] (row pitch H*Dp*2 bytes), box box_rows rows x
+// 64 columns, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, long long rows, int H, int Dp, int box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   if (rows < 1) rows = 1;
   const cuuint64_t dims[2] = {(cuuint64_t)H * Dp, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)H * Dp * 2};
-  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -217,13 +217,13 @@ Srcs kernel_srcs(const vdn_cfg* cfg, const Geom& g, const void* q, const void* k
   return Srcs{ws(cfg, g.off_q), ws(cfg, g.off_k), ws(cfg, g.off_v), ws(cfg, g.off_tk), ws(cfg, g.off_tv)};
 }
 
-bool make_maps(Maps& m, const Geom& g, const Srcs& s) {
+bool make_maps(Maps& m, const Geom& g, const Srcs& s, int box_rows = 128) {
   const long long vrows = (long long)g.B * g.N;
   const long long trows = (long long)g.B * g.T;
-  bool ok = make_map(&m.q, s.q, vrows, g.H, g.Dp) && make_map(&m.k, s.k, vrows, g.H, g.Dp) &&
-            make_map(&m.v, s.v, vrows, g.H, g.Dp);
+  bool ok = make_map(&m.q, s.q, vrows, g.H, g.Dp, box_rows) && make_map(&m.k, s.k, vrows, g.H, g.Dp, box_rows) &&
+            make_map(&m.v, s.v, vrows, g.H, g.Dp, box_rows);
   if (g.T > 0) {
-    ok = ok && make_map(&m.tk, s.tk, trows, g.H, g.Dp) && make_map(&m.tv, s.tv, trows, g.H, g.Dp);
+    ok = ok && make_map(&m.tk, s.tk, trows, g.H, g.Dp, box_rows) && make_map(&m.tv, s.tv, trows, g.H, g.Dp, box_rows);
   } else {  // never read; any valid descriptor
     m.tk = m.q;
     m.tv = m.q;

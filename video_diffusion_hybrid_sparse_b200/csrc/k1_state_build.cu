@@ -21,7 +21,7 @@
 //
 // Roles (22 warps):
 //   * warp 0 (one thread): TMA loads of the K and V tiles (128-byte swizzle),
-//     three stages, with L2 prefetches of the tiles after them;
+//     three stages;
 //   * warps 2-17: phi in place on the K tile (rows past the segment and padded
 //     head_dim columns zeroed), fenced to the async proxy;
 //   * warp 1 (one thread): D[:, 0:Dp] += phi(K)^T V and D[:, Dp:Dp+16] +=
@@ -53,7 +53,6 @@ struct K1Layout {
 };
 
 enum { kFull = 0, kPhi = 3, kEmpty = 6, kAccFull = 9, kAccEmpty = 11, kDone = 13, kNumBars1 = 14 };
-constexpr int kPrefetch = 4;         // tiles prefetched into L2 beyond the stages
 constexpr int kPhiWarps = 16;        // warps 2..17
 constexpr int kPhiThreads = 32 * kPhiWarps;
 constexpr int kEpiWarp0 = 2 + kPhiWarps;  // warps 18..21
@@ -145,26 +144,11 @@ __global__ void __launch_bounds__(kK1Threads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ loads
     if (lane == 0) {
-      // L2 prefetch kPrefetch tiles ahead of the loads: the shared-memory
-      // stages alone hold too few bytes to cover DRAM latency at full rate
-      auto prefetch = [&](int i) {
-        if (i >= ntiles) return;
-        const SbTile tl = sb_tile(t_begin + i, g, sp);
-        const int h = tl.bh % g.H;
-        const CUtensorMap* mk = tl.text ? &tm_tk : &tm_k;
-        const CUtensorMap* mv = tl.text ? &tm_tv : &tm_v;
-        for (int bx = 0; bx < D / 64; ++bx) {
-          tma_prefetch_2d(mk, h * D + bx * 64, tl.row);
-          tma_prefetch_2d(mv, h * D + bx * 64, tl.row);
-        }
-      };
-      for (int i = L::kStages; i < L::kStages + kPrefetch; ++i) prefetch(i);
       int i = 0;
       bool ok = true;
       for (; i < ntiles; ++i) {
         const int st = i % L::kStages;
         const uint32_t ph = (i / L::kStages) & 1;
-        prefetch(i + L::kStages + kPrefetch);
         if (!mbar_wait(&bars[kEmpty + st], ph ^ 1, ab)) { ok = false; break; }
         const SbTile tl = sb_tile(t_begin + i, g, sp);
         const int h = tl.bh % g.H;

@@ -356,16 +356,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 128; ++i)
               if (i >= n_valid) s[i] = __float_as_uint(-INFINITY);
           }
-          // row max: four independent fmax3 chains
-          float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+          // row max: eight independent fmax3 chains of eight (the max's
+          // latency, not its instruction count, is on the critical path)
+          float mc[8];
 #pragma unroll
-          for (int i = 0; i < 128; i += 8) {
-            a0 = fmax3(a0, __uint_as_float(s[i]), __uint_as_float(s[i + 1]));
-            a1 = fmax3(a1, __uint_as_float(s[i + 2]), __uint_as_float(s[i + 3]));
-            a2 = fmax3(a2, __uint_as_float(s[i + 4]), __uint_as_float(s[i + 5]));
-            a3 = fmax3(a3, __uint_as_float(s[i + 6]), __uint_as_float(s[i + 7]));
-          }
-          const float mxs = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * sl2;
+          for (int c = 0; c < 8; ++c) mc[c] = fmaxf(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1]));
+#pragma unroll
+          for (int i = 16; i < 128; i += 16)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) mc[c] = fmax3(mc[c], __uint_as_float(s[i + 2 * c]), __uint_as_float(s[i + 2 * c + 1]));
+          const float mxs =
+              fmaxf(fmaxf(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5])), fmaxf(mc[6], mc[7])) * sl2;
           // lazy rescale: move the running max only when this tile's max is
           // more than 2^8 above it (O is rescaled below, once P is stored)
           if (j == 0) {
