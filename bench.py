@@ -54,8 +54,9 @@ def softmax_key_frames(c, F, C):
     return win | {0, F - 1}
 
 
-def work(w):
-    """Algorithmic FLOPs and bytes per call (counts only what the method must do)."""
+def work(w, fp8: bool = False):
+    """Algorithmic FLOPs and bytes per call (counts only what the method must do);
+    fp8: the e4m3 softmax path (its softmax kernel does not apply the gate)."""
     e = 2 if w.dtype == "bf16" else 4
     n_chunks, anchors = w.F // w.C, len({0, w.F - 1})
     pairs = sum(w.C * w.P * (w.P * len(softmax_key_frames(c, w.F, w.C)) + w.T) for c in range(n_chunks))
@@ -67,7 +68,7 @@ def work(w):
     # on the bf16 path with head_dim 64 or 128 the softmax kernel applies the
     # softmax branch's gate: it reads g_s, and the readout reads q, the gated
     # term and g_l and writes out (four tensors instead of five)
-    gated = w.dtype == "bf16" and w.d in (64, 128)
+    gated = w.dtype == "bf16" and w.d in (64, 128) and not fp8
     k4 = (4 if gated else 5) * w.B * w.N * w.H * w.d * e + n_chunks * state
     k3_bytes = ((3 + (1 if gated else 0)) * w.B * w.N + 2 * w.B * w.T) * w.H * w.d * e + w.B * w.N * w.H * w.d * 2
     return dict(softmax_flops=softmax_flops, linear_flops=linear_flops, k1_bytes=k1, k2_bytes=k2, k4_bytes=k4,
@@ -188,7 +189,10 @@ def gpu_id_for(local_rank: int) -> str:
 
 def kernel_source_hash(name: str) -> str:
     """sha1 of the kernel's source file and of the headers it is compiled with."""
-    files = {"sparse_softmax": ["k3_sparse_softmax.cu", "sm100.cuh", "plan.h", "kernels.h"]}
+    files = {"sparse_softmax": ["k3_sparse_softmax.cu", "k3_common.cuh", "scan.cuh", "sm100.cuh", "plan.h",
+                                "kernels.h"],
+             "state_build": ["k1_state_build.cu", "phi.cuh", "sm100.cuh", "plan.h", "kernels.h"],
+             "readout_merge": ["k4_merge_tma.cu", "k4_common.cuh", "phi.cuh", "sm100.cuh", "plan.h", "kernels.h"]}
     h = hashlib.sha1()
     for f in files[name]:
         with open(os.path.join(ROOT, "video_diffusion_hybrid_sparse_b200", "csrc", f), "rb") as fh:
@@ -373,7 +377,7 @@ def run_ours(args, w, world, rank, local):
     steps = vb.Steps(dev["q"], dev["k"], dev["v"], dev["text_k"], dev["text_v"], dev["gate_s"], dev["gate_l"], out,
                      frames=w.F, chunk_frames=w.C, softmax_precision=prec)
     stream = torch.cuda.current_stream()
-    wk = work(w)
+    wk = work(w, fp8)
     staged = w.dtype == "fp32" or w.d == 32
     launches_per_step = 3 + (5 if staged else 0) + (4 if fp8 and w.T > 0 else 3 if fp8 else 0)
 
@@ -438,7 +442,8 @@ def run_ours(args, w, world, rank, local):
         t = per_kernel[n] * 1e-3
         if bound == "hbm":
             a = amount / t / 1e9 if t > 0 else None
-            kern[n] = {"ms": per_kernel[n], "bound": "hbm", "achieved_gbs": a, "frac": a / hbm if a else None}
+            kern[n] = {"ms": per_kernel[n], "bound": "hbm", "achieved_gbs": a, "frac": a / hbm if a else None,
+                       "bytes": amount, "traffic": None if fp8 else recorded_traffic(n, w.name)}
         else:
             a = amount / t / 1e12
             kern[n] = {"ms": per_kernel[n], "bound": "tensor", "achieved_tflops": a, "frac": a / tc_peak}

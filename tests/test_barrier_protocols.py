@@ -359,15 +359,16 @@ def k1_roles(pieces, stages=3):
 
 # ------------------------------------------------------------------ k3_sparse_softmax / k3_fp8
 # items: (query tiles of the item, KV tiles of its key set) in the CTA's order.
-# P is handed to the MMA thread in one piece per tile.  The fp8
-# kernel performs the same barrier operations (checked below on the sources).
-# Buffers: Q (the item's query tiles), K0/K1 and V0/V1 (the stages), SP0/SP1
-# (TMEM of S, with P written over it, per query tile), O0/O1 (TMEM output
-# accumulators; the softmax warps may rescale them in place before handing
-# over P, modelled at every step).
+# The bf16 kernel hands P to the MMA thread in two halves per tile (keys
+# 0-63 on PFull, keys 64-127 on PFull2); the fp8 kernel in one piece
+# (halves=1).  Buffers: Q (the item's query tiles), K0/K1 and V0/V1 (the
+# stages), SPa/SPb per query tile (the two halves of the TMEM columns of S,
+# with P written over them), O0/O1 (TMEM output accumulators; the softmax
+# warps may rescale them in place before handing over the first half of P,
+# modelled at every step).
 
 
-def k3_roles(items, stages=2):
+def k3_roles(items, stages=2, halves=2):
     loads, kv = [], 0
     for n_item, (_, nkv) in enumerate(items):
         if n_item > 0:
@@ -381,8 +382,11 @@ def k3_roles(items, stages=2):
 
     mma_, kv, p_cnt, s_idx = [], 0, [0, 0], [0, 0]
 
+    parts = ["a", "b"][:halves]
+
     def issue_s(t, n_item, st, kv_):
-        mma_.append(mma(reads=[("Q", n_item), (f"K{st}", kv_)], writes=[(f"SP{t}", ("S", s_idx[t]))]))
+        mma_.append(mma(reads=[("Q", n_item), (f"K{st}", kv_)],
+                        writes=[(f"SP{h}{t}", ("S", s_idx[t])) for h in parts]))
         s_idx[t] += 1
 
     for n_item, (nt, nkv) in enumerate(items):
@@ -397,9 +401,10 @@ def k3_roles(items, stages=2):
             st, nst, has_next = kv % stages, (kv + 1) % stages, j + 1 < nkv
             mma_.append(wait(f"VFull{st}", kv // stages))
             for t in range(nt):
-                mma_.append(wait(f"PFull{t}", p_cnt[t]))
-                mma_.append(mma(reads=[(f"SP{t}", ("P", p_cnt[t])), (f"V{st}", kv)],
-                                writes=[(f"O{t}", ("O", n_item, j))]))
+                for h in parts:
+                    mma_.append(wait(f"PFull{'2' if h == 'b' else ''}{t}", p_cnt[t]))
+                    mma_.append(mma(reads=[(f"SP{h}{t}", ("P", p_cnt[t])), (f"V{st}", kv)],
+                                    writes=[(f"O{t}", ("O", n_item, j))]))
                 p_cnt[t] += 1
                 if not has_next:
                     mma_.append(commit(f"OFull{t}"))
@@ -422,9 +427,12 @@ def k3_roles(items, stages=2):
             if t >= nt:
                 continue
             for j in range(nkv):
-                sm += [wait(f"SFull{t}", s_cnt), beg(reads=[(f"SP{t}", ("S", s_cnt))]), end(f"SP{t}"),
-                       beg(writes=[(f"O{t}", ("scaled", n_item, j))]), end(f"O{t}"),
-                       beg(writes=[(f"SP{t}", ("P", s_cnt))]), end(f"SP{t}"), arrive(f"PFull{t}")]
+                sm += [wait(f"SFull{t}", s_cnt)]
+                sm += [x for h in parts for x in (beg(reads=[(f"SP{h}{t}", ("S", s_cnt))]), end(f"SP{h}{t}"))]
+                sm += [beg(writes=[("SPa" + str(t), ("P", s_cnt))]), end(f"SPa{t}"),
+                       beg(writes=[(f"O{t}", ("scaled", n_item, j))]), end(f"O{t}"), arrive(f"PFull{t}")]
+                if halves == 2:
+                    sm += [beg(writes=[(f"SPb{t}", ("P", s_cnt))]), end(f"SPb{t}"), arrive(f"PFull2{t}")]
                 s_cnt += 1
             sm += [wait(f"OFull{t}", o_cnt), beg(reads=[(f"O{t}", ("O", n_item, nkv - 1))]), end(f"O{t}")]
             o_cnt += 1
@@ -491,18 +499,10 @@ def test_sparse_softmax_protocol(items):
     assert check(k3_roles(items)) > 0
 
 
-def test_fp8_softmax_has_the_bf16_barrier_operations():
-    import os
-    import re
-    csrc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
-                        "video_diffusion_hybrid_sparse_b200", "csrc")
-    pat = re.compile(r"mbar_wait\(&bars\[[^]]*\][^;]*|mma_commit\(&bars\[[^]]*\]\)|"
-                     r"mbar_arrive\(&bars\[[^]]*\]\)|mbar_expect_tx\(&bars\[[^]]*\]")
-
-    def ops(f):
-        return pat.findall(open(os.path.join(csrc, f)).read())
-
-    assert ops("k3_sparse_softmax.cu") == ops("k3_fp8.cu") and len(ops("k3_fp8.cu")) > 10
+@pytest.mark.parametrize("items", K3_SCHEDULES[:5], ids=[str(s) for s in K3_SCHEDULES[:5]])
+def test_fp8_softmax_protocol(items):
+    # one P handoff per tile
+    assert check(k3_roles(items, halves=1)) > 0
 
 
 def _drop(roles, role, pred):
@@ -532,16 +532,19 @@ def _move_before(roles, role, pred_move, pred_anchor):
 
 def _move_o_rescale_before_s_wait(roles):
     ops = list(roles["softmax0"])
-    out, i = [], 0
-    while i < len(ops):
-        op = ops[i]
+    out, pending = [], None
+    for i, op in enumerate(ops):
+        if op is None:
+            continue
+        if op.kind == "beg" and op.writes and op.writes[0][1][0] == "scaled":
+            # the rescale (this op and its end) goes before the preceding S wait
+            ops[i + 1] = None
+            out.insert(pending, op)
+            out.insert(pending + 1, end(op.writes[0][0]))
+            continue
         if op.kind == "wait" and op.bar == "SFull0":
-            # ops i+1..i+2 read S; ops i+3..i+4 rescale O: put the rescale first
-            out += ops[i + 3:i + 5] + [op] + ops[i + 1:i + 3]
-            i += 5
-        else:
-            out.append(op)
-            i += 1
+            pending = len(out)
+        out.append(op)
     roles = dict(roles)
     roles["softmax0"] = out
     return roles
@@ -577,6 +580,14 @@ PLANTED = {
     # the softmax MMA thread does not wait for P
     "softmax_mma_skips_p": lambda: _drop(k3_roles([(2, 2)]), "mma",
                                          lambda op: op.kind == "wait" and op.bar.startswith("PFull")),
+    # the MMA thread starts the P.V of the second half of the keys when only
+    # the first half of P is stored
+    "softmax_mma_skips_second_half": lambda: _drop(k3_roles([(2, 2)]), "mma",
+                                                   lambda op: op.kind == "wait" and op.bar.startswith("PFull2")),
+    # the softmax warps hand over the first half of P before rescaling O
+    "softmax_first_half_before_rescale": lambda: _move_before(
+        k3_roles([(1, 3)]), "softmax0", lambda op: op.kind == "arrive" and op.bar == "PFull0",
+        lambda op: op.kind == "beg" and op.writes and op.writes[0][0] == "O0"),
     # the loader refills a K stage before the S MMAs that read it completed
     "softmax_loader_skips_k_release": lambda: _drop(k3_roles([(1, 3)]), "loads",
                                                     lambda op: op.kind == "wait" and op.bar.startswith("KEmpty")),
@@ -610,10 +621,16 @@ SOURCE_BARRIER_OPS = {
                          "wait:kAccFull+buf arrive:kAccEmpty+buf",
     "k3_sparse_softmax.cu": "wait:kQEmpty expect_tx:kQFull wait:kKEmpty+st expect_tx:kKFull+st wait:kVEmpty+st "
                             "expect_tx:kVFull+st wait:kQFull wait:kKFull+st mma_commit:kSFull+t "
-                            "mma_commit:kKEmpty+st wait:kVFull+st wait:kPFull+t mma_commit:kOFull+t "
-                            "wait:kKFull+nst mma_commit:kSFull+t mma_commit:kVEmpty+st mma_commit:kKEmpty+nst "
-                            "mma_commit:kQEmpty mma_commit:kDone wait:kSFull+t arrive:kPFull+t "
-                            "wait:kOFull+t",
+                            "mma_commit:kKEmpty+st wait:kVFull+st wait:kPFull+t wait:kPFull2+t "
+                            "mma_commit:kOFull+t wait:kKFull+nst mma_commit:kSFull+t mma_commit:kVEmpty+st "
+                            "mma_commit:kKEmpty+nst mma_commit:kQEmpty mma_commit:kDone wait:kSFull+t "
+                            "arrive:kPFull+t arrive:kPFull2+t wait:kOFull+t",
+    "k3_fp8.cu": "wait:kQEmpty expect_tx:kQFull wait:kKEmpty+st expect_tx:kKFull+st wait:kVEmpty+st "
+                 "expect_tx:kVFull+st wait:kQFull wait:kKFull+st mma_commit:kSFull+t "
+                 "mma_commit:kKEmpty+st wait:kVFull+st wait:kPFull+t mma_commit:kOFull+t "
+                 "wait:kKFull+nst mma_commit:kSFull+t mma_commit:kVEmpty+st mma_commit:kKEmpty+nst "
+                 "mma_commit:kQEmpty mma_commit:kDone wait:kSFull+t arrive:kPFull+t "
+                 "wait:kOFull+t",
     "k4_merge_tma.cu": "wait:kTBEmpty expect_tx:kTBFull wait:kTAEmpty expect_tx:kTAFull wait:kTGEmpty "
                        "expect_tx:kTGFull wait:kTBFull wait:kTAReady+s wait:kTAccEmpty+s mma_commit:kTAccFull+s "
                        "mma_commit:kTBEmpty mma_commit:kTDone wait:kTAccFull+s arrive:kTAccEmpty+s wait:kTGFull "

@@ -38,9 +38,13 @@
 // a weight of 0 from the SFU, below 2^-126 from the FMA-pipe form.
 //
 // The MMA issue order per KV tile j is PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), so
-// the tensor core works on one tile while the other tile's softmax runs.  A
-// commit after S_t(j+1) also covers PV_t(j), so when the softmax of tile t sees
-// S_t(j+1) its O_t is quiescent and may be rescaled.
+// the tensor core works on one tile while the other tile's softmax runs.  P is
+// handed over in two halves (keys 0-63, then 64-127): the P.V of the first
+// half runs while the second half is exponentiated, which takes its time off
+// the tile's critical chain (S -> softmax -> P.V -> next S).  A commit after
+// S_t(j+1) also covers PV_t(j), so when the softmax of tile t sees S_t(j+1)
+// its O_t is quiescent and may be rescaled (before the first half is handed
+// over).
 #include <type_traits>
 
 #include "k3_common.cuh"
@@ -139,6 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars[kSFull + t], 1);
       mbar_init(&bars[kPFull + t], kBlockM);
+      mbar_init(&bars[kPFull2 + t], kBlockM);
       mbar_init(&bars[kOFull + t], 1);
     }
     mbar_init(&bars[kDone], 1);
@@ -234,14 +239,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(d_tmem, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
-      // O_t += P_t·V over the 128 keys of the tile
-      auto issue_pv = [&](int t, int st, bool acc) {
+      // O_t += P_t·V over keys 64*part .. 64*part + 63 of the tile
+      auto issue_pv = [&](int t, int st, int part, bool acc) {
         const uint32_t d_tmem = tmem + 256 + t * D;
         const uint64_t vd = v_desc0 + (uint64_t)((st * L::kTile) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk)
+        for (int k = 0; k < 4; ++k) {
+          const int kk = 4 * part + k;
           mma_ts(d_tmem, tmem + t * 128 + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
                  (acc || kk > 0) ? 1u : 0u);
+        }
       };
 
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++item_cnt) {
@@ -266,7 +273,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int t = 0; t < it.ntiles; ++t) {
             if (!mbar_wait(&bars[kPFull + t], p_cnt[t] & 1, ab)) { ok = false; break; }
             tc_fence_after();
-            issue_pv(t, st, j > 0);
+            issue_pv(t, st, 0, j > 0);
+            if (!mbar_wait(&bars[kPFull2 + t], p_cnt[t] & 1, ab)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(t, st, 1, true);
             ++p_cnt[t];
             if (!has_next) mma_commit(&bars[kOFull + t]);
             if (has_next) {
@@ -387,27 +397,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk[8];
             exp_group(&s[16 * i], sl2x2, negm, pk, l0, l1);
             tmem_st8(s_addr + 8 * i, pk);
+            if (i == 3) {
+              if (rescale) {
+#pragma unroll 1
+                for (int c = 0; c < D / 16; ++c) {
+                  uint32_t o[16];
+                  const uint32_t ta = tmem_addr(tmem, lane_base, 256 + t * D + 16 * c);
+                  tmem_ld16(ta, o);
+                  tmem_wait_ld();
+#pragma unroll
+                  for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                  tmem_st16(ta, o);
+                }
+              }
+              tmem_wait_st();
+              tc_fence_before();
+              mbar_arrive(&bars[kPFull + t]);  // keys 0-63: the P.V of the first half may start
+            }
           }
         };
         if (n_valid < kBlockN) tile(std::true_type());
         else tile(std::false_type());
-        if (rescale) {
-          // O_t is quiescent here: S_t(j) completing implies PV_t(j-1)
-          // completed, and PV_t(j) starts only after P_t(j) is handed over.
-#pragma unroll 1
-          for (int c = 0; c < D / 16; ++c) {
-            uint32_t o[16];
-            const uint32_t ta = tmem_addr(tmem, lane_base, 256 + t * D + 16 * c);
-            tmem_ld16(ta, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st16(ta, o);
-          }
-        }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars[kPFull + t]);
+        mbar_arrive(&bars[kPFull2 + t]);
         float c0, c1, c2, c3;
         f32x2_unpack(l0, c0, c1);
         f32x2_unpack(l1, c2, c3);
