@@ -225,7 +225,10 @@ def _fmt(trace, names, bars):
 # accumulator slots).
 
 
-def k4_tma_roles(keys, per_slot_ready=True):
+def k4_tma_roles(keys, per_slot_ready=True, tma_store=True):
+    """tma_store: the workers merge each tile into the o_s buffer (G) and the
+    loader stores it by TMA (reading G until the store's wait_group.read)
+    before reloading G."""
     n = len(keys)
     ready = (lambda i: f"AReady{i & 1}") if per_slot_ready else (lambda i: "AReady")
     ready_phase = (lambda i: i >> 1) if per_slot_ready else (lambda i: i)
@@ -243,7 +246,11 @@ def k4_tma_roles(keys, per_slot_ready=True):
             loads.append(tma("AFull", ("Q", i)))
         if i >= 1:
             loads.append(wait("GEmpty", i - 2))  # parity ((i - 1) & 1) ^ 1
+            if tma_store and i >= 2:
+                loads += [beg(reads=[("G", ("out", i - 2))]), end("G")]
             loads.append(tma("GFull", ("G", i - 1)))
+    if tma_store and n > 0:
+        loads += [wait("GEmpty", n - 1), beg(reads=[("G", ("out", n - 1))]), end("G")]
 
     mma_, prev, b_loads = [], None, 0
     for i in range(n):
@@ -265,8 +272,10 @@ def k4_tma_roles(keys, per_slot_ready=True):
     def finish(j):
         s = j & 1
         workers.extend([wait(f"AccFull{s}", j >> 1), beg(reads=[(f"Acc{s}", j)]), end(f"Acc{s}"),
-                        arrive(f"AccEmpty{s}"), wait("GFull", j), beg(reads=[("G", j)]), end("G"),
-                        arrive("GEmpty")])
+                        arrive(f"AccEmpty{s}"), wait("GFull", j), beg(reads=[("G", j)]), end("G")])
+        if tma_store:
+            workers.extend([beg(writes=[("G", ("out", j))]), end("G")])
+        workers.append(arrive("GEmpty"))
 
     for i in range(n):
         s = i & 1
@@ -511,6 +520,14 @@ def _drop(roles, role, pred):
     return out
 
 
+def _drop_last(roles, role, pred):
+    ops = list(roles[role])
+    i = max(k for k, op in enumerate(ops) if pred(op))
+    out = dict(roles)
+    out[role] = ops[:i] + ops[i + 1:]
+    return out
+
+
 def _move_before(roles, role, pred_move, pred_anchor):
     """Move every op matching pred_move to just before the preceding op that
     matches pred_anchor."""
@@ -558,6 +575,9 @@ PLANTED = {
     "readout_release_before_read": lambda: _move_before(
         k4_tma_roles([0, 0, 1, 1]), "workers", lambda op: op.kind == "arrive" and op.bar == "AEmpty",
         lambda op: op.kind == "beg" and op.reads and op.reads[0][0] == "Q"),
+    # the loader stores the last output tile without waiting for the merge to finish
+    "readout_store_before_merge": lambda: _drop_last(k4_tma_roles([0, 0, 1]), "loads",
+                                                     lambda op: op.kind == "wait" and op.bar == "GEmpty"),
     # the loader reloads o_s and the gates without waiting for the merge to finish
     "readout_loader_skips_g_release": lambda: _drop(k4_tma_roles([0, 0, 1, 1]), "loads",
                                                     lambda op: op.kind == "wait" and op.bar == "GEmpty"),
@@ -632,7 +652,7 @@ SOURCE_BARRIER_OPS = {
                  "mma_commit:kQEmpty mma_commit:kDone wait:kSFull+t arrive:kPFull+t "
                  "wait:kOFull+t",
     "k4_merge_tma.cu": "wait:kTBEmpty expect_tx:kTBFull wait:kTAEmpty expect_tx:kTAFull wait:kTGEmpty "
-                       "expect_tx:kTGFull wait:kTBFull wait:kTAReady+s wait:kTAccEmpty+s mma_commit:kTAccFull+s "
+                       "expect_tx:kTGFull wait:kTGEmpty wait:kTBFull wait:kTAReady+s wait:kTAccEmpty+s mma_commit:kTAccFull+s "
                        "mma_commit:kTBEmpty mma_commit:kTDone wait:kTAccFull+s arrive:kTAccEmpty+s wait:kTGFull "
                        "arrive:kTGEmpty wait:kTAFull arrive:kTAEmpty arrive:kTAReady+(i&1)",
     "k4_readout_merge.cu": "wait:kBEmpty expect_tx:kBFull wait:kAEmpty+s expect_tx:kAFull+s wait:kBFull "

@@ -405,7 +405,7 @@ vdn_status step_readout_merge(const vdn_cfg* cfg, const Geom& g, const Srcs& s, 
     mm.q = m.q;
     const long long vrows = (long long)g.B * g.N;
     if (!make_map(&mm.os, ws(cfg, g.off_os), vrows, g.H, g.Dp) || !make_map(&mm.gs, gs, vrows, g.H, g.Dp) ||
-        !make_map(&mm.gl, gl, vrows, g.H, g.Dp))
+        !make_map(&mm.gl, gl, vrows, g.H, g.Dp) || !make_map(&mm.out, out, vrows, g.H, g.Dp))
       return VDN_ERR_CUDA;
     return cuda_status(launch_readout_merge_tma(mm, p, st));
   }

@@ -91,7 +91,7 @@ cudaError_t launch_readout_merge(const Maps& m, const K4Params& p, cudaStream_t 
 // Maps of the TMA-fed readout/merge (bf16, head_dim == Dp): q, o_s and the
 // two gates as 2-D [rows, H*Dp] views like Maps.
 struct MergeMaps {
-  CUtensorMap q, os, gs, gl;
+  CUtensorMap q, os, gs, gl, out;  // out: the output tensor, same geometry (TMA stores of full tiles)
 };
 cudaError_t launch_readout_merge_tma(const MergeMaps& m, const K4Params& p, cudaStream_t st);
 cudaError_t launch_membership(const Geom& g, uint8_t* table, cudaStream_t st);
