@@ -58,33 +58,38 @@ constexpr int kPhiThreads = 32 * kPhiWarps;
 constexpr int kEpiWarp0 = 2 + kPhiWarps;  // warps 18..21
 constexpr int kK1Threads = 32 * (kEpiWarp0 + 4);
 
-// Tile `t` of this CTA's range, decoded.
-struct SbTile {
-  int bh, seg, row, n_valid;
-  bool text;
+// Walk over the tiles of this CTA's range: (batch, head), tile within the
+// (batch, head) and its segment, advanced one tile at a time (one division
+// at the start of the range, none per tile).
+struct SbCursor {
+  int bh, lt, seg;
+
+  __device__ __forceinline__ SbCursor(long long t, const StatePlan& sp) {
+    bh = (int)(t / sp.tiles_per_bh);
+    lt = (int)(t - (long long)bh * sp.tiles_per_bh);
+    seg = sb_seg_of(lt, sp);
+  }
+  // The tile is the last of its segment (the next one starts another piece).
+  __device__ __forceinline__ bool seg_ends(const StatePlan& sp) const { return lt + 1 == sp.seg_tile0[seg + 1]; }
+  __device__ __forceinline__ void next(const StatePlan& sp) {
+    if (++lt == sp.tiles_per_bh) {
+      lt = 0;
+      seg = 0;
+      ++bh;
+    } else if (lt == sp.seg_tile0[seg + 1]) {
+      ++seg;
+    }
+  }
+  __device__ __forceinline__ bool text(const StatePlan& sp) const { return seg >= sp.n_vsegs; }
+  // first token row of the tile in the [B * N] video or [B * T] text rows
+  __device__ __forceinline__ int row(const Geom& g, const StatePlan& sp) const {
+    const int b = bh / g.H;
+    return (text(sp) ? b * g.T : b * (int)g.N) + sp.seg_row0[seg] + (lt - sp.seg_tile0[seg]) * 128;
+  }
+  __device__ __forceinline__ int n_valid(const StatePlan& sp) const {
+    return min(128, sp.seg_rows[seg] - (lt - sp.seg_tile0[seg]) * 128);
+  }
 };
-
-__device__ __forceinline__ SbTile sb_tile(long long t, const Geom& g, const StatePlan& sp) {
-  SbTile r;
-  r.bh = (int)(t / sp.tiles_per_bh);
-  const int lt = (int)(t - (long long)r.bh * sp.tiles_per_bh);
-  r.seg = sb_seg_of(lt, sp);
-  const int tis = lt - sp.seg_tile0[r.seg];
-  r.text = r.seg >= sp.n_vsegs;
-  const int b = r.bh / g.H;
-  r.row = (r.text ? b * g.T : b * (int)g.N) + sp.seg_row0[r.seg] + tis * 128;
-  r.n_valid = min(128, sp.seg_rows[r.seg] - tis * 128);
-  return r;
-}
-
-// The CTA's tile t ends its piece (the next tile is in another segment, or the range ends).
-__device__ __forceinline__ bool piece_ends(long long t, long long t_end, const StatePlan& sp) {
-  if (t + 1 >= t_end) return true;
-  const int bh = (int)(t / sp.tiles_per_bh), bh1 = (int)((t + 1) / sp.tiles_per_bh);
-  if (bh != bh1) return true;
-  const int lt1 = (int)(t + 1 - (long long)bh * sp.tiles_per_bh);
-  return sb_seg_of(lt1, sp) != sb_seg_of(lt1 - 1, sp);
-}
 
 }  // namespace
 
@@ -146,20 +151,20 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     if (lane == 0) {
       int i = 0;
       bool ok = true;
-      for (; i < ntiles; ++i) {
+      SbCursor cur(t_begin, sp);
+      for (; i < ntiles; ++i, cur.next(sp)) {
         const int st = i % L::kStages;
         const uint32_t ph = (i / L::kStages) & 1;
         if (!mbar_wait(&bars[kEmpty + st], ph ^ 1, ab)) { ok = false; break; }
-        const SbTile tl = sb_tile(t_begin + i, g, sp);
-        const int h = tl.bh % g.H;
-        const CUtensorMap* mk = tl.text ? &tm_tk : &tm_k;
-        const CUtensorMap* mv = tl.text ? &tm_tv : &tm_v;
+        const int h = cur.bh % g.H, row = cur.row(g, sp);
+        const CUtensorMap* mk = cur.text(sp) ? &tm_tk : &tm_k;
+        const CUtensorMap* mv = cur.text(sp) ? &tm_tv : &tm_v;
         mbar_expect_tx(&bars[kFull + st], (D / 64) * 16384 * 2);
         uint8_t* sa = smem + st * L::kStage;
         uint8_t* sb = sa + L::kATile;
         for (int bx = 0; bx < D / 64; ++bx) {
-          tma_load_2d(sa + bx * 16384, mk, &bars[kFull + st], h * D + bx * 64, tl.row);
-          tma_load_2d(sb + bx * 16384, mv, &bars[kFull + st], h * D + bx * 64, tl.row);
+          tma_load_2d(sa + bx * 16384, mk, &bars[kFull + st], h * D + bx * 64, row);
+          tma_load_2d(sb + bx * 16384, mv, &bars[kFull + st], h * D + bx * 64, row);
         }
       }
       if (!ok)
@@ -178,7 +183,8 @@ __global__ void __launch_bounds__(kK1Threads, 1)
       const bool injected = p.inject_timeout && blockIdx.x == 0 && !mbar_wait(&bars[kAccFull], 0, ab, 10000000ll);
       int piece = 0;
       bool first = true;  // first tile of the current piece
-      for (int i = 0; i < ntiles && !injected; ++i) {
+      SbCursor cur(t_begin, sp);
+      for (int i = 0; i < ntiles && !injected; ++i, cur.next(sp)) {
         const int st = i % L::kStages;
         const int a = piece & 1;
         if (first && !mbar_wait(&bars[kAccEmpty + a], ((piece >> 1) & 1) ^ 1, ab)) break;
@@ -197,7 +203,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
           mma_ss(acc + D, da, b1, idesc_1, accum);
         }
         mma_commit(&bars[kEmpty + st]);
-        first = piece_ends(t_begin + i, t_end, sp);
+        first = i + 1 == ntiles || cur.seg_ends(sp);  // this tile ends its piece
         if (first) {
           mma_commit(&bars[kAccFull + a]);
           ++piece;
@@ -209,12 +215,13 @@ __global__ void __launch_bounds__(kK1Threads, 1)
   } else if (warp < kEpiWarp0) {
     // ------------------------------------------------------------ phi workers
     const int tid = threadIdx.x - 64;
-    for (int i = 0; i < ntiles; ++i) {
+    SbCursor cur(t_begin, sp);
+    for (int i = 0; i < ntiles; ++i, cur.next(sp)) {
       const int st = i % L::kStages;
       const bool got = mbar_wait(&bars[kFull + st], (i / L::kStages) & 1, ab);
       if (__any_sync(0xffffffffu, !got)) break;
-      const SbTile tl = sb_tile(t_begin + i, g, sp);
-      phi_tile_inplace<D / 64 * 1024 / kPhiThreads>(smem + st * L::kStage, D / 64, tl.n_valid, g.d, tid, kPhiThreads);
+      phi_tile_inplace<D / 64 * 1024 / kPhiThreads>(smem + st * L::kStage, D / 64, cur.n_valid(sp), g.d, tid,
+                                                     kPhiThreads);
       fence_proxy_async_smem();
       mbar_arrive(&bars[kPhi + st]);
     }
@@ -223,17 +230,17 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     const uint32_t quarter = warp & 3;
     const int a = quarter * 32 + lane;  // TMEM lane = head_dim slot of phi(k)
     int piece = 0;
-    for (int i = 0; i < ntiles; ++i) {
-      if (!piece_ends(t_begin + i, t_end, sp)) continue;
+    SbCursor cur(t_begin, sp);
+    for (int i = 0; i < ntiles; ++i, cur.next(sp)) {
+      if (!(i + 1 == ntiles || cur.seg_ends(sp))) continue;  // not the last tile of a piece
       const int buf = piece & 1;
       const bool got = mbar_wait(&bars[kAccFull + buf], (piece >> 1) & 1, ab);
       if (__any_sync(0xffffffffu, !got)) break;
       tc_fence_after();
-      const SbTile tl = sb_tile(t_begin + i, g, sp);
       // this CTA's contributor index within the segment
-      const long long seg_first = (long long)tl.bh * sp.tiles_per_bh + sp.seg_tile0[tl.seg];
+      const long long seg_first = (long long)cur.bh * sp.tiles_per_bh + sp.seg_tile0[cur.seg];
       const int u = (int)blockIdx.x - sb_cta_of(seg_first, sp);
-      float* dst = p.parts + sb_slot(tl.bh, tl.seg, u, sp) * (long long)(D + 1) * D;
+      float* dst = p.parts + sb_slot(cur.bh, cur.seg, u, sp) * (long long)(D + 1) * D;
       const uint32_t acc = tmem + buf * L::kAccCols;
 #pragma unroll
       for (int c = 0; c < L::kCols / 16; ++c) {

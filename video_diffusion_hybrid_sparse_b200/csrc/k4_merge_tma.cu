@@ -427,7 +427,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
           const uint4 v = *reinterpret_cast<const uint4*>(smem + L::kA + piece_off(row, col0 + 8 * c8));
           const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) pk[4 * c8 + e] = pack_bf16x2(phi_f(bf16_lo(w[e])), phi_f(bf16_hi(w[e])));
+          for (int e = 0; e < 4; ++e) pk[4 * c8 + e] = phi_bf16x2(w[e]);
         }
         mbar_arrive(&bars[kTAEmpty]);  // q tile read: the next one may be loaded
         const uint32_t base = tmem_addr(tmem + (i & 1) * L::kAccCols, quarter * 32, L::kPhiCol + col0 / 2);

@@ -64,6 +64,8 @@ WORKLOADS = [
     Workload("768p_long_bf16", 1, 60, 4032, 24, 128, 512, 5, "bf16", "rms", 4),
     # profiling shape: the 768p latent with 4 of its 24 heads (inputs still larger than L2)
     Workload("768p_h4_bf16", 1, 15, 4032, 4, 128, 512, 1, "bf16", "rms", 5),
+    # profiling shape: half the heads (every SM gets half the steady-state work of the full launch)
+    Workload("768p_h12_bf16", 1, 15, 4032, 12, 128, 512, 1, "bf16", "rms", 6),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
 
