@@ -122,6 +122,18 @@ __device__ __forceinline__ Item4 decode_pos(int pos, const Geom& g, int tiles) {
   return it;
 }
 
+// Item4 of consecutive positions, advanced without divisions.
+__device__ __forceinline__ void next_pos(Item4& it, const Geom& g, int tiles) {
+  if (++it.tile < tiles) return;
+  it.tile = 0;
+  ++it.key;
+  if (++it.c < g.Nc) return;
+  it.c = 0;
+  if (++it.b < g.B) return;
+  it.b = 0;
+  ++it.h;
+}
+
 }  // namespace
 
 // kGeneral: the debug outputs or the SPLIT output (flags & 7 or out_linear set)
@@ -188,8 +200,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
       bool ok = true;
       // the output tile of tile j (merged in the o_s buffer) goes out before
       // that buffer is reloaded
-      auto store_out = [&](int j) {
-        const Item4 it = item(j);
+      auto store_out = [&](const Item4& it) {
         if (!tma_out(it)) return;
         for (int bx = 0; bx < D / 64; ++bx) tma_store_2d(&tm_out, smem + L::kG + bx * 16384, it.h * D + bx * 64, row0_of(it));
         bulk_commit();
@@ -197,9 +208,15 @@ __global__ void __launch_bounds__(kTThreads, 1)
       };
       // step i: q of tile i, then o_s and the gates of tile i - 1 (they are
       // needed one tile later, once the merge of tile i - 2 has freed the buffer)
+      // items i + 1, i, i - 1 and i - 2 of the step
+      Item4 nx = item(0), cur = nx, prev1 = nx, prev2 = nx;
       for (int i = 0; i <= n && ok; ++i) {
+        prev2 = prev1;
+        prev1 = cur;
+        cur = nx;
+        next_pos(nx, g, tiles);
         if (i < n) {
-          const Item4 it = item(i);
+          const Item4& it = cur;
           if (it.key != prev_key) {
             if (b_loads > 0 && !mbar_wait(&bars[kTBEmpty], (b_loads - 1) & 1, ab)) { ok = false; break; }
             mbar_expect_tx(&bars[kTBFull], (uint32_t)(2 * L::kBTile));
@@ -214,10 +231,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
             tma_load_2d(smem + L::kA + bx * 16384, &tm_q, &bars[kTAFull], it.h * D + bx * 64, row0_of(it));
           ++a_issued;
           // warm L2 for what the next steps load
-          if (i + 1 < n) {
-            const Item4 nx = item(i + 1);
+          if (i + 1 < n)
             for (int bx = 0; bx < D / 64; ++bx) tma_prefetch_2d(&tm_q, nx.h * D + bx * 64, row0_of(nx));
-          }
           for (int bx = 0; bx < D / 64; ++bx) {
             tma_prefetch_2d(&tm_os, it.h * D + bx * 64, row0_of(it));
             if (!gated) tma_prefetch_2d(&tm_gs, it.h * D + bx * 64, row0_of(it));
@@ -225,9 +240,9 @@ __global__ void __launch_bounds__(kTThreads, 1)
           }
         }
         if (i >= 1) {
-          const Item4 it = item(i - 1);
+          const Item4& it = prev1;
           if (!mbar_wait(&bars[kTGEmpty], ((i - 1) & 1) ^ 1, ab)) { ok = false; break; }
-          if (i >= 2) store_out(i - 2);
+          if (i >= 2) store_out(prev2);
           mbar_expect_tx(&bars[kTGFull], (uint32_t)((gated ? 2 : 3) * L::kTile));
           for (int bx = 0; bx < D / 64; ++bx) {
             tma_load_2d(smem + L::kG + bx * 16384, &tm_os, &bars[kTGFull], it.h * D + bx * 64, row0_of(it));
@@ -241,7 +256,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
         }
       }
       // the last tile's output
-      if (ok && n > 0 && mbar_wait(&bars[kTGEmpty], (n - 1) & 1, ab)) store_out(n - 1);
+      // (the loop ended after step n: prev1 is item n - 1)
+      if (ok && n > 0 && mbar_wait(&bars[kTGEmpty], (n - 1) & 1, ab)) store_out(prev1);
       if (!ok) {  // let loads in flight land before the CTA exits
         if (a_issued > 0) mbar_drain(&bars[kTAFull], (a_issued - 1) & 1);
         if (g_issued > 0) mbar_drain(&bars[kTGFull], (g_issued - 1) & 1);
@@ -255,8 +271,9 @@ __global__ void __launch_bounds__(kTThreads, 1)
       constexpr uint32_t idesc = idesc_bf16_f32(128, kCols, 0, 0);
       const uint64_t b_desc0 = smem_desc(smem_u32(smem + L::kB), 16, 1024, kLayoutSw128);
       int prev_key = -1, b_loads = 0;
-      for (int i = 0; i < n; ++i) {
-        const Item4 it = item(i);
+      Item4 it = item(0), nx = it;
+      next_pos(nx, g, tiles);
+      for (int i = 0; i < n; ++i, it = nx, next_pos(nx, g, tiles)) {
         const int s = i & 1;
         if (it.key != prev_key) {
           if (p.stall_ns > 0 && i > 0) sleep_ns(p.stall_ns);  // debug: let the other warps run ahead
@@ -277,7 +294,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
                    (hl | kk) ? 1u : 0u);
           }
         mma_commit(&bars[kTAccFull + s]);
-        const bool key_ends = i + 1 >= n || item(i + 1).key != it.key;
+        const bool key_ends = i + 1 >= n || nx.key != it.key;
         if (key_ends) mma_commit(&bars[kTBEmpty]);
       }
       mma_commit(&bars[kTDone]);
@@ -297,9 +314,10 @@ __global__ void __launch_bounds__(kTThreads, 1)
     // gated o_s, plain merge; 1: ungated o_s, plain merge; 2: the general
     // merge (debug outputs, SPLIT).  Returns false on a timeout (the four
     // warps of a row quarter agree).
+    Item4 wit = item(0);  // the item of the next finish (tiles are finished in order)
     auto finish = [&](int j, auto variant) -> bool {
       constexpr int V = decltype(variant)::value;
-      const Item4 it = item(j);
+      const Item4 it = wit;
       const int s = j & 1;
       const bool got = mbar_wait(&bars[kTAccFull + s], (j >> 1) & 1, ab);
       if (quad_any(quarter, !got)) return false;
@@ -336,43 +354,84 @@ __global__ void __launch_bounds__(kTThreads, 1)
       uint8_t* t_os = smem + L::kG;
       const uint8_t* t_gs = smem + L::kG + L::kTile;
       const uint8_t* t_gl = smem + L::kG + 2 * L::kTile;
+      if constexpr (V != 2) {
+        // plain merge, two columns per packed f32x2 operation
+        const uint64_t scale2 = f32x2_pack(scale, scale);
 #pragma unroll
-      for (int c8 = 0; c8 < kQC / 8; ++c8) {
-        const int col = col0 + 8 * c8;
-        const int off = piece_off(row, col);
-        const uint4 vo = *reinterpret_cast<const uint4*>(t_os + off);
-        const uint4 vl = *reinterpret_cast<const uint4*>(t_gl + off);
-        const uint32_t ow[4] = {vo.x, vo.y, vo.z, vo.w};
-        const uint32_t lw[4] = {vl.x, vl.y, vl.z, vl.w};
-        float os[8], gl[8], rr[8], sterm[8];
+        for (int c8 = 0; c8 < kQC / 8; ++c8) {
+          const int col = col0 + 8 * c8;
+          const int off = piece_off(row, col);
+          const uint4 vo = *reinterpret_cast<const uint4*>(t_os + off);
+          const uint4 vl = *reinterpret_cast<const uint4*>(t_gl + off);
+          const uint32_t ow[4] = {vo.x, vo.y, vo.z, vo.w};
+          const uint32_t lw[4] = {vl.x, vl.y, vl.z, vl.w};
+          uint32_t sw[4] = {0u, 0u, 0u, 0u};
+          if constexpr (V == 1) {
+            const uint4 vs = *reinterpret_cast<const uint4*>(t_gs + off);
+            sw[0] = vs.x; sw[1] = vs.y; sw[2] = vs.z; sw[3] = vs.w;
+          }
+          const float2* gam = reinterpret_cast<const float2*>(p.gamma + it.h * d + col);
+          float o[8];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          os[2 * k] = bf16_lo(ow[k]); os[2 * k + 1] = bf16_hi(ow[k]);
-          gl[2 * k] = bf16_lo(lw[k]); gl[2 * k + 1] = bf16_hi(lw[k]);
-        }
-        // the softmax branch's gated term sigmoid(g_s) * o_s
-        if (V == 0 || (V == 2 && gated)) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) sterm[k] = os[k];
-        } else {
-          const uint4 vs = *reinterpret_cast<const uint4*>(t_gs + off);
-          const uint32_t sw[4] = {vs.x, vs.y, vs.z, vs.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            sterm[2 * k] = sigmoid_f(bf16_lo(sw[k])) * os[2 * k];
-            sterm[2 * k + 1] = sigmoid_f(bf16_hi(sw[k])) * os[2 * k + 1];
+          for (int e = 0; e < 4; ++e) {
+            // the softmax branch's gated term sigmoid(g_s) * o_s
+            uint64_t st2 = f32x2_pack(bf16_lo(ow[e]), bf16_hi(ow[e]));
+            if constexpr (V == 1) st2 = f32x2_mul(sigmoid2_tanh(f32x2_pack(bf16_lo(sw[e]), bf16_hi(sw[e]))), st2);
+            uint64_t rr2 = f32x2_mul(f32x2_pack(__uint_as_float(v[8 * c8 + 2 * e]), __uint_as_float(v[8 * c8 + 2 * e + 1])),
+                                     scale2);
+            if (use_gamma) {
+              const float2 g2 = __ldg(gam + e);
+              rr2 = f32x2_mul(rr2, f32x2_pack(g2.x, g2.y));
+            }
+            const uint64_t o2 = f32x2_fma(sigmoid2_tanh(f32x2_pack(bf16_lo(lw[e]), bf16_hi(lw[e]))), rr2, st2);
+            f32x2_unpack(o2, o[2 * e], o[2 * e + 1]);
+          }
+          if (via_tma) {
+            // in place of this thread's own o_s piece, for the TMA store
+            *reinterpret_cast<uint4*>(t_os + off) = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                                                               pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+          } else if (row < nrows) {
+            store8<false>(p.out, row_h * d + col, o);
           }
         }
+      } else {
+        // general merge: debug outputs, SPLIT (16-byte stores)
 #pragma unroll
-        for (int k = 0; k < 8; ++k) rr[k] = __uint_as_float(v[8 * c8 + k]) * scale;
-        if (use_gamma) {
-          const float4 ga = __ldg(reinterpret_cast<const float4*>(p.gamma + it.h * d + col));
-          const float4 gb = __ldg(reinterpret_cast<const float4*>(p.gamma + it.h * d + col) + 1);
-          rr[0] *= ga.x; rr[1] *= ga.y; rr[2] *= ga.z; rr[3] *= ga.w;
-          rr[4] *= gb.x; rr[5] *= gb.y; rr[6] *= gb.z; rr[7] *= gb.w;
-        }
-        float o[8];
-        if constexpr (V == 2) {
+        for (int c8 = 0; c8 < kQC / 8; ++c8) {
+          const int col = col0 + 8 * c8;
+          const int off = piece_off(row, col);
+          const uint4 vo = *reinterpret_cast<const uint4*>(t_os + off);
+          const uint4 vl = *reinterpret_cast<const uint4*>(t_gl + off);
+          const uint32_t ow[4] = {vo.x, vo.y, vo.z, vo.w};
+          const uint32_t lw[4] = {vl.x, vl.y, vl.z, vl.w};
+          float os[8], gl[8], rr[8], sterm[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            os[2 * k] = bf16_lo(ow[k]); os[2 * k + 1] = bf16_hi(ow[k]);
+            gl[2 * k] = bf16_lo(lw[k]); gl[2 * k + 1] = bf16_hi(lw[k]);
+          }
+          // the softmax branch's gated term sigmoid(g_s) * o_s
+          if (gated) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) sterm[k] = os[k];
+          } else {
+            const uint4 vs = *reinterpret_cast<const uint4*>(t_gs + off);
+            const uint32_t sw[4] = {vs.x, vs.y, vs.z, vs.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              sterm[2 * k] = sigmoid_f(bf16_lo(sw[k])) * os[2 * k];
+              sterm[2 * k + 1] = sigmoid_f(bf16_hi(sw[k])) * os[2 * k + 1];
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) rr[k] = __uint_as_float(v[8 * c8 + k]) * scale;
+          if (use_gamma) {
+            const float4 ga = __ldg(reinterpret_cast<const float4*>(p.gamma + it.h * d + col));
+            const float4 gb = __ldg(reinterpret_cast<const float4*>(p.gamma + it.h * d + col) + 1);
+            rr[0] *= ga.x; rr[1] *= ga.y; rr[2] *= ga.z; rr[3] *= ga.w;
+            rr[4] *= gb.x; rr[5] *= gb.y; rr[6] *= gb.z; rr[7] *= gb.w;
+          }
+          float o[8];
           if (split) {
             float ol[8];
 #pragma unroll
@@ -389,20 +448,11 @@ __global__ void __launch_bounds__(kTThreads, 1)
             }
           }
           if (row < nrows) store8<false>(p.out, row_h * d + col, o);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) o[k] = sterm[k] + sigmoid_f(gl[k]) * rr[k];
-          if (via_tma) {
-            // in place of this thread's own o_s piece, for the TMA store
-            *reinterpret_cast<uint4*>(t_os + off) = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
-                                                               pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
-          } else if (row < nrows) {
-            store8<false>(p.out, row_h * d + col, o);
-          }
         }
       }
       if (via_tma) fence_proxy_async_smem();  // the output tile is read by the async proxy
       mbar_arrive(&bars[kTGEmpty]);           // the shared tiles may be reloaded (after the store)
+      next_pos(wit, g, tiles);
       return true;
     };
     auto fin = [&](int j) -> bool {

@@ -136,6 +136,17 @@ __device__ __forceinline__ float sigmoid_tanh(float x) {
   return fmaf(0.5f, t, 0.5f);
 }
 
+// sigmoid of two packed fp32 values: the arithmetic of sigmoid_tanh on each,
+// the multiply and the fma packed
+__device__ __forceinline__ uint64_t sigmoid2_tanh(uint64_t x) {
+  const uint64_t half = f32x2_pack(0.5f, 0.5f);
+  float h0, h1, t0, t1;
+  f32x2_unpack(f32x2_mul(x, half), h0, h1);
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t0) : "f"(h0));
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t1) : "f"(h1));
+  return f32x2_fma(half, f32x2_pack(t0, t1), half);
+}
+
 // ------------------------------------------------------------------ abort / status
 
 // Status shared by the warps of one CTA.  A wait that runs out sets `abort`
