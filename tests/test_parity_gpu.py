@@ -39,8 +39,11 @@ def assert_close(got, ref, what, abs_tol=TOL_ABS, rel_tol=TOL_REL):
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
     err = np.abs(got - ref)
     i = np.unravel_index(np.argmax(err), err.shape)
-    assert err[i] <= abs_tol, f"{what}: max-abs {err[i]:.3e} at {i} (got {got[i]}, ref {ref[i]})"
     r = rel_l2(got, ref)
+    # one line per comparison (shown with pytest -s): the accuracy record
+    print(f"ACCURACY {what}: max-abs {err[i]:.2e} at {tuple(int(x) for x in i)}, rel-L2 {r:.2e}, "
+          f"max|ref| {np.abs(ref).max():.3g}")
+    assert err[i] <= abs_tol, f"{what}: max-abs {err[i]:.3e} at {i} (got {got[i]}, ref {ref[i]})"
     assert r <= rel_tol, f"{what}: rel-L2 {r:.3e}"
 
 
