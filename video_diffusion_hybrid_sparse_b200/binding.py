@@ -170,6 +170,11 @@ def workspace_bytes(s: Shape, softmax_precision: int = PREC_BF16) -> int:
 _WS: dict = {}
 
 
+def new_workspace(s: Shape, device, softmax_precision: int = PREC_BF16) -> torch.Tensor:
+    """A fresh device workspace for shape s (one per call in flight)."""
+    return torch.empty(workspace_bytes(s, softmax_precision), dtype=torch.uint8, device=torch.device(device))
+
+
 def workspace_for(s: Shape, device, softmax_precision: int = PREC_BF16) -> torch.Tensor:
     """A cached device workspace large enough for shape s."""
     n = workspace_bytes(s, softmax_precision)
@@ -242,14 +247,25 @@ def clear_timeout_record(workspace: torch.Tensor) -> None:
     workspace[64:128].zero_()
 
 
-def staging_for(s: Shape, device, split: bool = False) -> torch.Tensor:
-    """A cached device staging buffer for :func:`hybrid_attn_fwd_host`."""
+def staging_bytes(s: Shape, split: bool = False) -> int:
+    """Bytes of the device staging buffer :func:`hybrid_attn_fwd_host` needs."""
     cfg = make_cfg(s)
     if split:
         cfg.output_mode = OUTPUT_SPLIT
     n = library().vdn_host_staging_bytes(ctypes.byref(cfg))
     if n == 0:
         _check(library().vdn_validate(ctypes.byref(cfg)), "vdn_host_staging_bytes")
+    return n
+
+
+def new_staging(s: Shape, device, split: bool = False) -> torch.Tensor:
+    """A fresh device staging buffer (one per host call in flight)."""
+    return torch.empty(staging_bytes(s, split), dtype=torch.uint8, device=torch.device(device))
+
+
+def staging_for(s: Shape, device, split: bool = False) -> torch.Tensor:
+    """A cached device staging buffer for :func:`hybrid_attn_fwd_host`."""
+    n = staging_bytes(s, split)
     dev = torch.device(device)
     key = (dev.index if dev.index is not None else torch.cuda.current_device())
     buf = _STAGING.get(key)
