@@ -90,6 +90,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars[kSFull + t], 1);
       mbar_init(&bars[kPFull + t], kBlockM);
+      mbar_init(&bars[kPFull2 + t], kBlockM);
       mbar_init(&bars[kOFull + t], 1);
     }
     mbar_init(&bars[kDone], 1);
@@ -172,13 +173,15 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk) mma_ss_f8(d_tmem, qd + 2 * kk, kd + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
       };
-      // O_t += P_t·V over the 128 keys of the tile
-      auto issue_pv = [&](int t, int st, bool acc) {
+      // O_t += P_t·V over keys 64*part .. 64*part + 63 of the tile
+      auto issue_pv = [&](int t, int st, int part, bool acc) {
         const uint32_t d_tmem = tmem + 256 + t * D;
         const uint64_t vd = v_desc0 + (uint64_t)((st * L::kTile) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kBlockN / 32; ++kk)  // 32 keys: 8 TMEM columns of P, 32 bytes of a V^T row
+        for (int k = 0; k < 2; ++k) {  // 32 keys: 8 TMEM columns of P, 32 bytes of a V^T row
+          const int kk = 2 * part + k;
           mma_ts_f8(d_tmem, tmem + t * 128 + kk * 8, vd + 2 * kk, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
       };
 
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++item_cnt) {
@@ -203,7 +206,10 @@ __global__ void __launch_bounds__(384, 1)
           for (int t = 0; t < it.ntiles; ++t) {
             if (!mbar_wait(&bars[kPFull + t], p_cnt[t] & 1, ab)) { ok = false; break; }
             tc_fence_after();
-            issue_pv(t, st, j > 0);
+            issue_pv(t, st, 0, j > 0);
+            if (!mbar_wait(&bars[kPFull2 + t], p_cnt[t] & 1, ab)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(t, st, 1, true);
             ++p_cnt[t];
             if (!has_next) mma_commit(&bars[kOFull + t]);
             if (has_next) {
@@ -336,24 +342,29 @@ __global__ void __launch_bounds__(384, 1)
               else pk[e >> 1] = pr;
             }
             tmem_st4(tmem_addr(tmem, lane_base, t * 128 + 4 * i), pk);
-          }
-          if (rescale) {
-            // O_t is quiescent here: S_t(j) completing implies PV_t(j-1)
-            // completed, and PV_t(j) starts only after P_t(j) is handed over.
+            if (i == 3) {
+              if (rescale) {
+                // O_t is quiescent here: S_t(j) completing implies PV_t(j-1)
+                // completed, and PV_t(j) starts only after P_t(j) is handed over.
 #pragma unroll 1
-            for (int c = 0; c < D / 16; ++c) {
-              uint32_t o[16];
-              const uint32_t ta = tmem_addr(tmem, lane_base, 256 + t * D + 16 * c);
-              tmem_ld16(ta, o);
-              tmem_wait_ld();
+                for (int c = 0; c < D / 16; ++c) {
+                  uint32_t o[16];
+                  const uint32_t ta = tmem_addr(tmem, lane_base, 256 + t * D + 16 * c);
+                  tmem_ld16(ta, o);
+                  tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st16(ta, o);
+                  for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                  tmem_st16(ta, o);
+                }
+              }
+              tmem_wait_st();
+              tc_fence_before();
+              mbar_arrive(&bars[kPFull + t]);  // keys 0-63: the P.V of the first half may start
             }
           }
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(&bars[kPFull + t]);
+          mbar_arrive(&bars[kPFull2 + t]);
           {
             float l0, l1, l2, l3;
             f32x2_unpack(lsum0, l0, l1);
