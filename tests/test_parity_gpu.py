@@ -196,12 +196,14 @@ def test_host_tensor_call_matches_device_call_and_oracle(w, mode, split):
         assert torch.equal(out_lin, ref_lin.cpu())
 
 
-# Exported forward/backward states against the oracle's: relative L2 4e-3.
+# Exported forward/backward states against the oracle's: relative L2 2e-3.
 # The states are fp32 sums of phi(k) v^T with phi(k) rounded to bf16 for the
 # tensor cores (relative rounding <= 2^-9, about 1.1e-3 RMS per term,
-# unbiased), so the relative error of a state is about 1e-3; fp32 inputs add
-# their own rounding to bf16 before phi.
-STATE_TOL = 4e-3
+# unbiased, independent across terms), so the relative error of a state
+# whose terms have random signs is about 1.1e-3 (measured: 1.7e-4 to 1.4e-3
+# on these four shapes, the largest on the fp32 one, whose inputs are first
+# rounded to bf16).
+STATE_TOL = 2e-3
 
 
 @pytest.mark.parametrize("w", [SMALL[0], SMALL[2], SMALL[3], SMALL[1]], ids=["tiny", "ragged", "c5_ragged", "small"])
