@@ -196,6 +196,37 @@ def test_host_tensor_call_matches_device_call_and_oracle(w, mode, split):
         assert torch.equal(out_lin, ref_lin.cpu())
 
 
+def test_host_calls_in_flight_on_two_streams():
+    """Host-tensor calls with two in flight, as bench.py's end-to-end number
+    runs them: call i on stream i % 2 with its own staging buffer, workspace
+    and host output, all enqueued before any synchronisation.  Each call's
+    output must equal the same call made alone, bit for bit, whatever the
+    overlap of one call's copies and kernels with the other's."""
+    calls = [BY_NAME["small_bf16"], SMALL[2], BY_NAME["small_bf16"], SMALL[2]]
+    hosts, alone = [], []
+    for w in calls:
+        inputs = make_inputs(w)
+        host = {k: t.pin_memory() for k, t in inputs.items()}
+        hosts.append(host)
+        ref = vb.hybrid_attn_fwd_host(host["q"], host["k"], host["v"], host["text_k"], host["text_v"],
+                                      host["gate_s"], host["gate_l"], frames=w.F, chunk_frames=w.C)
+        torch.cuda.synchronize()
+        alone.append(ref.clone())
+    streams = [torch.cuda.current_stream(), torch.cuda.Stream()]
+    outs = []
+    for i, (w, host) in enumerate(zip(calls, hosts)):
+        s = vb.shape_of(host["q"], host["text_k"], w.F, w.C)
+        stg, ws = vb.new_staging(s, "cuda"), vb.new_workspace(s, "cuda")
+        out = torch.empty(host["q"].shape, dtype=host["q"].dtype, pin_memory=True)
+        vb.hybrid_attn_fwd_host(host["q"], host["k"], host["v"], host["text_k"], host["text_v"], host["gate_s"],
+                                host["gate_l"], frames=w.F, chunk_frames=w.C, out=out, workspace=ws, staging=stg,
+                                stream=streams[i % 2])
+        outs.append((out, stg, ws))
+    torch.cuda.synchronize()
+    for i, (out, _, _) in enumerate(outs):
+        assert torch.equal(out, alone[i]), f"call {i}"
+
+
 # Exported forward/backward states against the oracle's: relative L2 2e-3.
 # The states are fp32 sums of phi(k) v^T with phi(k) rounded to bf16 for the
 # tensor cores (relative rounding <= 2^-9, about 1.1e-3 RMS per term,
