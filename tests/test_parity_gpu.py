@@ -227,14 +227,16 @@ def test_host_calls_in_flight_on_two_streams():
         assert torch.equal(out, alone[i]), f"call {i}"
 
 
-# Exported forward/backward states against the oracle's: relative L2 2e-3.
-# The states are fp32 sums of phi(k) v^T with phi(k) rounded to bf16 for the
+# Exported forward/backward states against the oracle's, relative L2.  The
+# states are fp32 sums of phi(k) v^T with phi(k) rounded to bf16 for the
 # tensor cores (relative rounding <= 2^-9, about 1.1e-3 RMS per term,
 # unbiased, independent across terms), so the relative error of a state
-# whose terms have random signs is about 1.1e-3 (measured: 1.7e-4 to 1.4e-3
-# on these four shapes, the largest on the fp32 one, whose inputs are first
-# rounded to bf16).
+# whose terms have random signs is about 1.1e-3: bound 2e-3.  fp32 inputs
+# are first rounded to bf16 themselves (k and v), three roundings per term,
+# about 1.9e-3 RMS: bound 4e-3.  Measured: 1.7e-4 to 1.3e-3 (bf16 shapes),
+# 2.6e-3 (the fp32 shape's 8-token text state).
 STATE_TOL = 2e-3
+STATE_TOL_FP32 = 4e-3
 
 
 @pytest.mark.parametrize("w", [SMALL[0], SMALL[2], SMALL[3], SMALL[1]], ids=["tiny", "ragged", "c5_ragged", "small"])
@@ -247,6 +249,7 @@ def test_exported_states_match_oracle(w):
     bwd = torch.zeros_like(fwd)
     run(w, dev, debug_flags=vb.EXPORT_STATES, export=(fwd, bwd))
     fwd, bwd = fwd.cpu().numpy(), bwd.cpu().numpy()
+    tol = STATE_TOL_FP32 if w.dtype == "fp32" else STATE_TOL
     worst = 0.0
     for b in range(w.B):
         for h in range(w.H):
@@ -256,9 +259,11 @@ def test_exported_states_match_oracle(w):
             ref_b = np.concatenate([st["SB"].transpose(0, 2, 1), st["zB"][:, None, :]], axis=1)
             ef, eb = rel_l2(fwd[b, :, h], ref_f), rel_l2(bwd[b, :, h], ref_b)
             worst = max(worst, ef, eb)
-            assert ef <= STATE_TOL and eb <= STATE_TOL, (b, h, ef, eb)
+            assert ef <= tol and eb <= tol, (b, h, ef, eb)
             if w.T > 0:  # chunk 0's forward state holds nothing but half of the text state
-                assert rel_l2(fwd[b, 0, h, :w.d, :], 0.5 * st["S_t"].T) <= STATE_TOL
+                et = rel_l2(fwd[b, 0, h, :w.d, :], 0.5 * st["S_t"].T)
+                worst = max(worst, et)
+                assert et <= tol, (b, h, et)
             # the states that hold no video frame are the same half text state, bit for bit:
             # forward of chunks 0 and 1, backward of the last two chunks
             half_t = fwd[b, 0, h]
