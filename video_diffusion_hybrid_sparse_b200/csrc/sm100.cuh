@@ -2,8 +2,8 @@
 // use: mbarriers (with bounded waits), TMA tile loads, bulk copies, and the
 // 5th-generation tensor core (tcgen05: TMEM allocation, MMA, commit, TMEM
 // loads/stores, fences) plus the UMMA shared-memory and instruction
-// descriptors.  Written from the PTX ISA; no multicast forms are used
-// anywhere.
+// descriptors.  Written from the PTX ISA; every TMA and bulk load writes
+// the shared memory of the issuing CTA only.
 #pragma once
 
 #include <cstdint>
@@ -319,7 +319,7 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
 
 // ------------------------------------------------------------------ TMA / bulk copies
 
-// 2-D tiled TMA load (no multicast) of the box at element coordinates
+// 2-D tiled TMA load, into this CTA's shared memory, of the box at element coordinates
 // (x = innermost, y) into shared memory; completes `bytes` on bar.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
   asm volatile(
