@@ -24,6 +24,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -187,16 +188,25 @@ def gpu_id_for(local_rank: int) -> str:
 # ---------------------------------------------------------------- ncu traffic record
 
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source without comments and blank space (what the compiler
+    sees; a comment edit does not change the kernel)."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash(name: str) -> str:
-    """sha1 of the kernel's source file and of the headers it is compiled with."""
+    """sha1 of the code (comments and blank space removed) of the kernel's
+    source file and of the headers it is compiled with."""
     files = {"sparse_softmax": ["k3_sparse_softmax.cu", "k3_common.cuh", "scan.cuh", "sm100.cuh", "plan.h",
                                 "kernels.h"],
              "state_build": ["k1_state_build.cu", "phi.cuh", "sm100.cuh", "plan.h", "kernels.h"],
              "readout_merge": ["k4_merge_tma.cu", "k4_common.cuh", "phi.cuh", "sm100.cuh", "plan.h", "kernels.h"]}
     h = hashlib.sha1()
     for f in files[name]:
-        with open(os.path.join(ROOT, "video_diffusion_hybrid_sparse_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "video_diffusion_hybrid_sparse_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:12]
 
 
