@@ -53,8 +53,7 @@ __device__ __forceinline__ Item decode_item(int item, const K3Params& p) {
 }
 
 // Barrier slots.  kPFull + t: the first half of P_t (keys 0-63) is in TMEM;
-// kPFull2 + t: the second half (the bf16 softmax kernel; the e4m3 one hands P
-// over whole on kPFull).
+// kPFull2 + t: the second half (both softmax kernels hand P over in halves).
 enum {
   kQFull = 0, kQEmpty = 1, kKFull = 2, kKEmpty = 4, kVFull = 6, kVEmpty = 8,
   kSFull = 10, kPFull = 12, kOFull = 14, kDone = 16, kPFull2 = 17, kNumBars = 19
