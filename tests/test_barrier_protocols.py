@@ -225,10 +225,11 @@ def _fmt(trace, names, bars):
 # accumulator slots).
 
 
-def k4_tma_roles(keys, per_slot_ready=True, tma_store=True):
+def k4_tma_roles(keys, per_slot_ready=True, tma_store=True, nq=2):
     """tma_store: the workers merge each tile into the o_s buffer (G) and the
     loader stores it by TMA (reading G until the store's wait_group.read)
-    before reloading G."""
+    before reloading G.  nq: q tiles in flight (2 when the softmax kernel
+    applied the gate and its slot holds a second q tile)."""
     n = len(keys)
     ready = (lambda i: f"AReady{i & 1}") if per_slot_ready else (lambda i: "AReady")
     ready_phase = (lambda i: i >> 1) if per_slot_ready else (lambda i: i)
@@ -242,8 +243,8 @@ def k4_tma_roles(keys, per_slot_ready=True, tma_store=True):
                 loads.append(tma("BFull", ("B", keys[i])))
                 b_loads += 1
                 prev = keys[i]
-            loads.append(wait("AEmpty", i - 1))  # parity (i & 1) ^ 1
-            loads.append(tma("AFull", ("Q", i)))
+            loads.append(wait(f"AEmpty{i % nq}", i // nq - 1))  # parity ((i / nq) & 1) ^ 1
+            loads.append(tma(f"AFull{i % nq}", (f"Q{i % nq}", i)))
         if i >= 1:
             loads.append(wait("GEmpty", i - 2))  # parity ((i - 1) & 1) ^ 1
             if tma_store and i >= 2:
@@ -279,7 +280,8 @@ def k4_tma_roles(keys, per_slot_ready=True, tma_store=True):
 
     for i in range(n):
         s = i & 1
-        workers += [wait("AFull", i), beg(reads=[("Q", i)]), end("Q"), arrive("AEmpty"),
+        workers += [wait(f"AFull{i % nq}", i // nq), beg(reads=[(f"Q{i % nq}", i)]), end(f"Q{i % nq}"),
+                    arrive(f"AEmpty{i % nq}"),
                     beg(writes=[(f"Phi{s}", i)]), end(f"Phi{s}"), arrive(ready(i))]
         if i > 0:
             finish(i - 1)
@@ -469,8 +471,9 @@ READOUT_KEYS = [[0, 0, 0, 0], [0, 0, 1, 1], [0, 1, 1, 2], [0, 1, 2, 3], [0, 0, 0
 
 
 @pytest.mark.parametrize("keys", READOUT_KEYS, ids=["".join(map(str, k)) for k in READOUT_KEYS])
-def test_tma_readout_protocol(keys):
-    assert check(k4_tma_roles(keys)) > 0
+@pytest.mark.parametrize("nq", [2, 1], ids=["two_q", "one_q"])
+def test_tma_readout_protocol(keys, nq):
+    assert check(k4_tma_roles(keys, nq=nq)) > 0
 
 
 def test_tma_readout_single_ready_barrier_fails():
@@ -573,12 +576,14 @@ def _move_o_rescale_before_s_wait(roles):
 
 PLANTED = {
     # the loader refills the q tile without waiting for the workers to release it
-    "readout_loader_skips_q_release": lambda: _drop(k4_tma_roles([0, 0, 1, 1]), "loads",
-                                                    lambda op: op.kind == "wait" and op.bar == "AEmpty"),
-    # the workers release the q tile before reading it
+    # (with one q slot; with two, the wait for the o_s / gate release orders
+    # the refill after the read anyway)
+    "readout_loader_skips_q_release": lambda: _drop(k4_tma_roles([0, 0, 1, 1, 1], nq=1), "loads",
+                                                    lambda op: op.kind == "wait" and op.bar.startswith("AEmpty")),
+    # the workers release the q tile before reading it (one q slot)
     "readout_release_before_read": lambda: _move_before(
-        k4_tma_roles([0, 0, 1, 1]), "workers", lambda op: op.kind == "arrive" and op.bar == "AEmpty",
-        lambda op: op.kind == "beg" and op.reads and op.reads[0][0] == "Q"),
+        k4_tma_roles([0, 0, 1, 1, 1], nq=1), "workers", lambda op: op.kind == "arrive" and op.bar.startswith("AEmpty"),
+        lambda op: op.kind == "beg" and op.reads and op.reads[0][0].startswith("Q")),
     # the loader stores the last output tile without waiting for the merge to finish
     "readout_store_before_merge": lambda: _drop_last(k4_tma_roles([0, 0, 1]), "loads",
                                                      lambda op: op.kind == "wait" and op.bar == "GEmpty"),
@@ -655,10 +660,10 @@ SOURCE_BARRIER_OPS = {
                  "mma_commit:kOFull+t wait:kKFull+nst mma_commit:kSFull+t mma_commit:kVEmpty+st "
                  "mma_commit:kKEmpty+nst mma_commit:kQEmpty mma_commit:kDone wait:kSFull+t "
                  "arrive:kPFull+t arrive:kPFull2+t wait:kOFull+t",
-    "k4_merge_tma.cu": "wait:kTBEmpty expect_tx:kTBFull wait:kTAEmpty expect_tx:kTAFull wait:kTGEmpty "
+    "k4_merge_tma.cu": "wait:kTBEmpty expect_tx:kTBFull wait:kTAEmpty+qs expect_tx:kTAFull+qs wait:kTGEmpty "
                        "expect_tx:kTGFull wait:kTGEmpty wait:kTBFull wait:kTAReady+s wait:kTAccEmpty+s mma_commit:kTAccFull+s "
                        "mma_commit:kTBEmpty mma_commit:kTDone wait:kTAccFull+s arrive:kTAccEmpty+s wait:kTGFull "
-                       "arrive:kTGEmpty wait:kTAFull arrive:kTAEmpty arrive:kTAReady+(i&1)",
+                       "arrive:kTGEmpty wait:kTAFull+i%nq arrive:kTAEmpty+i%nq arrive:kTAReady+(i&1)",
     "k4_readout_merge.cu": "wait:kBEmpty expect_tx:kBFull wait:kAEmpty+s expect_tx:kAFull+s wait:kBFull "
                            "wait:kAReady+s wait:kAccEmpty+s mma_commit:kAccFull+s mma_commit:kAEmpty+s "
                            "mma_commit:kBEmpty mma_commit:kDone4 wait:kAccFull+s arrive:kAccEmpty+s wait:kAFull+s "

@@ -66,9 +66,12 @@ struct K4TLayout {
 };
 
 enum {
-  kTAFull = 0, kTAReady = 1, kTAEmpty = 3, kTAccFull = 4, kTAccEmpty = 6, kTBFull = 8, kTBEmpty = 9,
-  kTGFull = 10, kTGEmpty = 11, kTDone = 12, kTNumBars = 13
+  kTAFull = 0, kTAReady = 2, kTAEmpty = 4, kTAccFull = 6, kTAccEmpty = 8, kTBFull = 10, kTBEmpty = 11,
+  kTGFull = 12, kTGEmpty = 13, kTDone = 14, kTNumBars = 15
 };
+// kTAFull + q / kTAEmpty + q: q tile slot q (the slot of tile i is i % nq;
+// nq = 2 when the softmax kernel applied the gate, whose g_s slot in the G
+// region then holds the second q tile, else 1).
 // kTAReady + s: phi(Q) of a tile of accumulator slot s is in TMEM (workers);
 // kTAEmpty: the workers have read the q tile out of shared memory (the
 // producer may load the next one); kTGEmpty: the workers are done with the
@@ -160,8 +163,10 @@ __global__ void __launch_bounds__(kTThreads, 1)
   const uint32_t warp = warp_id(), lane = lane_id();
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars[kTAFull], 1);
-    mbar_init(&bars[kTAEmpty], kTWorkers);
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&bars[kTAFull + q], 1);
+      mbar_init(&bars[kTAEmpty + q], kTWorkers);
+    }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[kTAReady + s], kTWorkers);
       mbar_init(&bars[kTAccFull + s], 1);
@@ -189,6 +194,9 @@ __global__ void __launch_bounds__(kTThreads, 1)
   // o_s already holds sigmoid(g_s) * o_s (the softmax kernel was given the
   // gate): g_s is then neither loaded nor applied
   const bool gated = p.os_gated != nullptr && __ldg(p.os_gated) != 0;
+  // q tiles in flight: the g_s slot is free for a second one when o_s comes gated
+  const int nq = gated ? 2 : 1;
+  auto q_slot = [&](int i) { return i % nq == 0 ? smem + L::kA : smem + L::kG + L::kTile; };
   // a full tile of the plain merge leaves by one TMA store from the o_s buffer
   // (the debug outputs and the SPLIT output take 16-byte stores)
   auto tma_out = [&](const Item4& it) { return !kGeneral && g.rows_per_chunk - it.tile * 128 >= 128; };
@@ -225,10 +233,11 @@ __global__ void __launch_bounds__(kTThreads, 1)
             ++b_loads;
             prev_key = it.key;
           }
-          if (!mbar_wait(&bars[kTAEmpty], (i & 1) ^ 1, ab)) { ok = false; break; }
-          mbar_expect_tx(&bars[kTAFull], (uint32_t)L::kTile);
+          const int qs = i % nq;
+          if (!mbar_wait(&bars[kTAEmpty + qs], ((i / nq) & 1) ^ 1, ab)) { ok = false; break; }
+          mbar_expect_tx(&bars[kTAFull + qs], (uint32_t)L::kTile);
           for (int bx = 0; bx < D / 64; ++bx)
-            tma_load_2d(smem + L::kA + bx * 16384, &tm_q, &bars[kTAFull], it.h * D + bx * 64, row0_of(it));
+            tma_load_2d(q_slot(i) + bx * 16384, &tm_q, &bars[kTAFull + qs], it.h * D + bx * 64, row0_of(it));
           ++a_issued;
           // warm L2 for what the next steps load
           if (i + 1 < n)
@@ -259,7 +268,8 @@ __global__ void __launch_bounds__(kTThreads, 1)
       // (the loop ended after step n: prev1 is item n - 1)
       if (ok && n > 0 && mbar_wait(&bars[kTGEmpty], (n - 1) & 1, ab)) store_out(prev1);
       if (!ok) {  // let loads in flight land before the CTA exits
-        if (a_issued > 0) mbar_drain(&bars[kTAFull], (a_issued - 1) & 1);
+        for (int i = (a_issued > nq ? a_issued - nq : 0); i < a_issued; ++i)
+          mbar_drain(&bars[kTAFull + i % nq], (i / nq) & 1);
         if (g_issued > 0) mbar_drain(&bars[kTGFull], (g_issued - 1) & 1);
         if (b_loads > 0) mbar_drain(&bars[kTBFull], (b_loads - 1) & 1);
       }
@@ -465,7 +475,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
 
     bool ok = true;
     for (int i = 0; i < n && ok; ++i) {
-      const bool got = mbar_wait(&bars[kTAFull], i & 1, ab);
+      const bool got = mbar_wait(&bars[kTAFull + i % nq], (i / nq) & 1, ab);
       if (all_workers_any(!got)) { ok = false; break; }
       // phi of this thread's quarter row, bf16 pairs into the free columns of
       // accumulator slot i % 2 (the MMA of tile i - 2, which read that slot's
@@ -474,12 +484,12 @@ __global__ void __launch_bounds__(kTThreads, 1)
         uint32_t pk[kQC / 2];
 #pragma unroll
         for (int c8 = 0; c8 < kQC / 8; ++c8) {
-          const uint4 v = *reinterpret_cast<const uint4*>(smem + L::kA + piece_off(row, col0 + 8 * c8));
+          const uint4 v = *reinterpret_cast<const uint4*>(q_slot(i) + piece_off(row, col0 + 8 * c8));
           const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) pk[4 * c8 + e] = phi_bf16x2(w[e]);
         }
-        mbar_arrive(&bars[kTAEmpty]);  // q tile read: the next one may be loaded
+        mbar_arrive(&bars[kTAEmpty + i % nq]);  // q tile read: its slot may be reloaded
         const uint32_t base = tmem_addr(tmem + (i & 1) * L::kAccCols, quarter * 32, L::kPhiCol + col0 / 2);
         if constexpr (kQC == 32) {
           tmem_st16(base, pk);
