@@ -389,15 +389,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               m_run = mxs;
             }
           }
-          // p = 2^(s * scale * log2(e) - m); P goes to TMEM 8 columns (16
+          // p = 2^(s * scale * log2(e) - m); P goes to TMEM 16 columns (32
           // keys) at a time
           const uint64_t negm = f32x2_pack(-m_run, -m_run);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            uint32_t pk[8];
-            exp_group(&s[16 * i], sl2x2, negm, pk, l0, l1);
-            tmem_st8(s_addr + 8 * i, pk);
-            if (i == 3) {
+          for (int i = 0; i < 8; i += 2) {
+            uint32_t pk[16];
+            exp_group(&s[16 * i], sl2x2, negm, *reinterpret_cast<uint32_t(*)[8]>(&pk[0]), l0, l1);
+            exp_group(&s[16 * i + 16], sl2x2, negm, *reinterpret_cast<uint32_t(*)[8]>(&pk[8]), l0, l1);
+            tmem_st16(s_addr + 8 * i, pk);
+            if (i == 2) {
               if (rescale) {
 #pragma unroll 1
                 for (int c = 0; c < D / 16; ++c) {
