@@ -12,7 +12,8 @@
 //   * warp 0 (one thread) TMA-loads the q tile, and, one tile later, the
 //     tile's o_s and gate_l tiles (128 rows x head_dim each), and gate_s only
 //     when the softmax kernel left o_s ungated (o_s holds sigmoid(g_s) * o_s
-//     when it was given the gate); it bulk-copies M_c (bf16 hi/lo readout
+//     when it was given the gate, and the gate_s slot then holds a second q
+//     tile, so two q tiles are in flight); it bulk-copies M_c (bf16 hi/lo readout
 //     operand) when the chunk changes, prefetches the next tiles into L2 and,
 //     once the workers have merged a full tile into the o_s buffer, TMA-stores
 //     it to out before that buffer is reloaded;
@@ -24,7 +25,7 @@
 //   * warps 2-17 (512 threads): warp w holds TMEM lanes 32 (w % 4) .. + 31
 //     (the tile's rows) and a quarter of the columns, (w - 2) / 4.  Each
 //     thread applies phi to its quarter row of the q tile and stores it to
-//     TMEM as bf16 (the q buffer is free for the next tile's load right
+//     TMEM as bf16 (its q slot is free for a later tile's load right
 //     after), then finishes the previous tile: o_l = num / den (0 for an empty
 //     state or a GLOBAL anchor query row), the row's sum of squares from the
 //     four quarter rows, and the merge out = sigmoid(g_s) o_s +
