@@ -41,9 +41,15 @@ from video_diffusion_hybrid_sparse_b200.workloads import BY_NAME, make_inputs  #
 METRIC = "hybrid-attn ms/call & TFLOP/s at 768p-shaped latent, 1×B200, % of roofline"
 SPEC_TFLOPS, SPEC_GBS = 2250.0, 8000.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# Steps timed separately (CUDA events between them); the forward/backward scan
-# runs inside the softmax kernel (its otherwise idle warps).
-KERNELS = ["stage", "state_build", "sparse_softmax", "readout_merge"]
+# Steps timed separately (CUDA events between them), with the Steps method
+# that runs each.  Separate readout (the default): the forward/backward scan
+# runs inside the softmax kernel (its otherwise idle warps), the readout and
+# merge in a kernel of their own.  Fused readout: the scan is a kernel of its
+# own and the softmax kernel's epilogue does the readout and merge.
+KERNELS = [("stage", "stage"), ("state_build", "state_build"), ("sparse_softmax", "softmax_and_scan"),
+           ("readout_merge", "readout_merge")]
+KERNELS_FUSED = [("stage", "stage"), ("state_build", "state_build"), ("state_scan", "state_scan"),
+                 ("sparse_softmax", "softmax_merge")]
 
 
 # ---------------------------------------------------------------- algorithmic work
@@ -55,9 +61,10 @@ def softmax_key_frames(c, F, C):
     return win | {0, F - 1}
 
 
-def work(w, fp8: bool = False):
+def work(w, fp8: bool = False, fused: bool = False):
     """Algorithmic FLOPs and bytes per call (counts only what the method must do);
-    fp8: the e4m3 softmax path (its softmax kernel does not apply the gate)."""
+    fp8: the e4m3 softmax path (its softmax kernel does not apply the gate);
+    fused: the readout and merge run in the softmax kernel (k3f_bytes)."""
     e = 2 if w.dtype == "bf16" else 4
     n_chunks, anchors = w.F // w.C, len({0, w.F - 1})
     pairs = sum(w.C * w.P * (w.P * len(softmax_key_frames(c, w.F, w.C)) + w.T) for c in range(n_chunks))
@@ -72,6 +79,12 @@ def work(w, fp8: bool = False):
     gated = w.dtype == "bf16" and w.d in (64, 128) and not fp8
     k4 = (4 if gated else 5) * w.B * w.N * w.H * w.d * e + n_chunks * state
     k3_bytes = ((3 + (1 if gated else 0)) * w.B * w.N + 2 * w.B * w.T) * w.H * w.d * e + w.B * w.N * w.H * w.d * 2
+    # fused: q, k, v, text, g_s and g_l read, M_c read once per item pair of
+    # tiles (counted once per (batch, chunk, head)), out written
+    k3f_bytes = ((5 * w.B * w.N + 2 * w.B * w.T) * w.H * w.d + w.B * w.N * w.H * w.d) * e + n_chunks * state
+    if fused:
+        return dict(softmax_flops=softmax_flops, linear_flops=linear_flops, k1_bytes=k1, k2_bytes=k2, k4_bytes=0,
+                    k3_bytes=k3f_bytes, linear_bytes=k1 + k2 + (k3f_bytes - k3_bytes))
     return dict(softmax_flops=softmax_flops, linear_flops=linear_flops, k1_bytes=k1, k2_bytes=k2, k4_bytes=k4,
                 k3_bytes=k3_bytes, linear_bytes=k1 + k2 + k4)
 
@@ -199,8 +212,9 @@ def _code_only(text: str) -> str:
 def kernel_source_hash(name: str) -> str:
     """sha1 of the code (comments and blank space removed) of the kernel's
     source file and of the headers it is compiled with."""
-    files = {"sparse_softmax": ["k3_sparse_softmax.cu", "k3_common.cuh", "scan.cuh", "sm100.cuh", "plan.h",
-                                "kernels.h"],
+    k3 = ["k3_sparse_softmax.cu", "k3_common.cuh", "phi.cuh", "scan.cuh", "sm100.cuh", "plan.h", "kernels.h"]
+    files = {"sparse_softmax": k3, "sparse_softmax_fused": k3,
+             "state_scan": ["k2_state_scan.cu", "scan.cuh", "sm100.cuh", "plan.h", "kernels.h"],
              "state_build": ["k1_state_build.cu", "phi.cuh", "sm100.cuh", "plan.h", "kernels.h"],
              "readout_merge": ["k4_merge_tma.cu", "k4_common.cuh", "phi.cuh", "sm100.cuh", "plan.h", "kernels.h"]}
     h = hashlib.sha1()
@@ -376,6 +390,65 @@ def config_of(w, world, precision="bf16"):
     return c
 
 
+def bench_line(args, w, world, wk, per_kernel, ms, e2e_ms, h2d, d2h, launches_per_step, clocks):
+    """The JSON line of our arm from the measured times (ms per call, per
+    kernel, end to end)."""
+    fp8 = args.precision == "fp8"
+    fused = args.readout == "fused"
+    flops_call = wk["softmax_flops"] + wk["linear_flops"]
+    value = flops_call * world / (ms * 1e-3) / 1e12
+    pk, src = peaks()
+    # an e4m3 contraction takes the bf16 measured peak x the nominal fp8 / bf16 ratio (4.5 / 2.25)
+    ratio = 2.0 if fp8 else 1.0
+    tc_peak, hbm = pk["bf16_tflops"] * ratio, pk["hbm_gbs"]
+    k3_ms = per_kernel["sparse_softmax"]
+    achieved = wk["softmax_flops"] / (k3_ms * 1e-3) / 1e12
+    k3_key = "sparse_softmax_fused" if fused else "sparse_softmax"
+    traffic = recorded_traffic(k3_key, w.name)
+    kern = {}
+    hbm_steps = (("state_build", wk["k1_bytes"], "hbm"), ("state_scan", wk["k2_bytes"], "hbm")) if fused else \
+        (("state_build", wk["k1_bytes"], "hbm"), ("readout_merge", wk["k4_bytes"], "hbm"))
+    for n, amount, bound in hbm_steps + (("sparse_softmax", wk["softmax_flops"], "tensor"),):
+        t = per_kernel[n] * 1e-3
+        if bound == "hbm":
+            a = amount / t / 1e9 if t > 0 else None
+            kern[n] = {"ms": per_kernel[n], "bound": "hbm", "achieved_gbs": a, "frac": a / hbm if a else None,
+                       "bytes": amount, "traffic": None if fp8 else recorded_traffic(n, w.name)}
+        else:
+            a = amount / t / 1e12
+            kern[n] = {"ms": per_kernel[n], "bound": "tensor", "achieved_tflops": a, "frac": a / tc_peak}
+    kern["stage"] = {"ms": per_kernel["stage"]}
+    if fused:
+        kern["sparse_softmax"]["includes"] = "readout, RMSNorm and gated merge (fused epilogue)"
+        kern["sparse_softmax"]["bytes"] = wk["k3_bytes"]
+    else:
+        kern["state_scan"] = {"ms": None, "in": "sparse_softmax (warps 2-3)", "bytes": wk["k2_bytes"]}
+    roof_s = wk["softmax_flops"] / (tc_peak * 1e12) + wk["linear_bytes"] / (hbm * 1e9)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8 (e4m3 softmax operands)" if fp8 else "bf16", "data": "synthetic",
+        "config": config_of(w, world, args.precision),
+        "readout": args.readout,
+        "roofline": {"bound": "tensor", "kernel": "sparse_softmax" + (" (incl. e4m3 quantisation)" if fp8 else "")
+                     + (" (readout and merge fused)" if fused else ""),
+                     "achieved": achieved, "peak": tc_peak,
+                     "unit": "TFLOP/s", "frac": achieved / tc_peak, "traffic": None if fp8 else traffic,
+                     "peak_source": (f"{src} bf16 burst (MEASURED_PEAKS.json)" if src == "measured" else "fallback")
+                     + (" x 2 (nominal fp8 / bf16)" if fp8 else ""),
+                     "frac_of_sustained": achieved / (pk.get("bf16_tflops_sustained", tc_peak) * ratio),
+                     "frac_of_spec": achieved / (SPEC_TFLOPS * ratio)},
+        "call_roofline": {"roofline_ms": roof_s * 1e3, "frac": roof_s * 1e3 / ms},
+        "kernels": kern,
+        "e2e": {"value": flops_call * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "calls_in_flight": 2,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    return line
+
+
 def run_ours(args, w, world, rank, local):
     from video_diffusion_hybrid_sparse_b200 import binding as vb
 
@@ -383,35 +456,44 @@ def run_ours(args, w, world, rank, local):
     dev = {k: t.cuda() for k, t in dev_t.items()}
     out = torch.empty_like(dev["q"])
     fp8 = args.precision == "fp8"
+    if args.readout == "fused" and (fp8 or w.dtype != "bf16" or w.d != 128):
+        args.readout = "separate"  # the fused readout is built for bf16, head_dim 128
+    fused = args.readout == "fused"
     prec = vb.PREC_FP8 if fp8 else vb.PREC_BF16
+    mode = vb.READOUT_FUSED if fused else vb.READOUT_SEPARATE
     steps = vb.Steps(dev["q"], dev["k"], dev["v"], dev["text_k"], dev["text_v"], dev["gate_s"], dev["gate_l"], out,
-                     frames=w.F, chunk_frames=w.C, softmax_precision=prec)
+                     frames=w.F, chunk_frames=w.C, softmax_precision=prec, readout_mode=mode)
     stream = torch.cuda.current_stream()
-    wk = work(w, fp8)
+    wk = work(w, fp8, fused)
     staged = w.dtype == "fp32" or w.d == 32
     launches_per_step = 3 + (5 if staged else 0) + (4 if fp8 and w.T > 0 else 3 if fp8 else 0)
+    seq = KERNELS_FUSED if fused else KERNELS
+
+    def one_call():
+        for _, method in seq:
+            getattr(steps, method)()
 
     for _ in range(args.warmup):
-        steps.all()
+        one_call()
     torch.cuda.synchronize()
 
     # ------------------------------------------------ device-resident timing
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(KERNELS) + 1)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(seq) + 1)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(gpu_id_for(local)) as clk:
         for s in range(args.steps):
             ev[s][0].record(stream)
-            for i, name in enumerate(KERNELS):
-                getattr(steps, "softmax_and_scan" if name == "sparse_softmax" else name)()
+            for i, (_, method) in enumerate(seq):
+                getattr(steps, method)()
                 ev[s][i + 1].record(stream)
         torch.cuda.synchronize()
     barrier(world)
-    per_kernel = {n: 0.0 for n in KERNELS}
+    per_kernel = {n: 0.0 for n, _ in seq}
     total_ms = 0.0
     for s in range(args.steps):
         total_ms += ev[s][0].elapsed_time(ev[s][-1])
-        for i, n in enumerate(KERNELS):
+        for i, (n, _) in enumerate(seq):
             per_kernel[n] += ev[s][i].elapsed_time(ev[s][i + 1]) / args.steps
     total_ms = max_over_ranks(total_ms, world)
     ms = total_ms / args.steps
@@ -442,7 +524,7 @@ def run_ours(args, w, world, rank, local):
         k = i % 2
         vb.hybrid_attn_fwd_host(host["q"], host["k"], host["v"], host["text_k"], host["text_v"], host["gate_s"],
                                 host["gate_l"], frames=w.F, chunk_frames=w.C, out=host_outs[k], workspace=wss[k],
-                                staging=stagings[k], stream=streams[k], softmax_precision=prec)
+                                staging=stagings[k], stream=streams[k], softmax_precision=prec, readout_mode=mode)
     joined = torch.cuda.Event()
     joined.record(streams[1])
     stream.wait_event(joined)
@@ -451,49 +533,7 @@ def run_ours(args, w, world, rank, local):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / n_e2e
     del stagings, wss
 
-    flops_call = wk["softmax_flops"] + wk["linear_flops"]
-    value = flops_call * world / (ms * 1e-3) / 1e12
-    pk, src = peaks()
-    # an e4m3 contraction takes the bf16 measured peak x the nominal fp8 / bf16 ratio (4.5 / 2.25)
-    ratio = 2.0 if fp8 else 1.0
-    tc_peak, hbm = pk["bf16_tflops"] * ratio, pk["hbm_gbs"]
-    k3_ms = per_kernel["sparse_softmax"]
-    achieved = wk["softmax_flops"] / (k3_ms * 1e-3) / 1e12
-    traffic = recorded_traffic("sparse_softmax", w.name)
-    kern = {}
-    for n, amount, bound in (("state_build", wk["k1_bytes"], "hbm"), ("readout_merge", wk["k4_bytes"], "hbm"),
-                             ("sparse_softmax", wk["softmax_flops"], "tensor")):
-        t = per_kernel[n] * 1e-3
-        if bound == "hbm":
-            a = amount / t / 1e9 if t > 0 else None
-            kern[n] = {"ms": per_kernel[n], "bound": "hbm", "achieved_gbs": a, "frac": a / hbm if a else None,
-                       "bytes": amount, "traffic": None if fp8 else recorded_traffic(n, w.name)}
-        else:
-            a = amount / t / 1e12
-            kern[n] = {"ms": per_kernel[n], "bound": "tensor", "achieved_tflops": a, "frac": a / tc_peak}
-    kern["stage"] = {"ms": per_kernel["stage"]}
-    kern["state_scan"] = {"ms": None, "in": "sparse_softmax (warps 2-3)", "bytes": wk["k2_bytes"]}
-    roof_s = wk["softmax_flops"] / (tc_peak * 1e12) + wk["linear_bytes"] / (hbm * 1e9)
-    line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "fp8 (e4m3 softmax operands)" if fp8 else "bf16", "data": "synthetic",
-        "config": config_of(w, world, args.precision),
-        "roofline": {"bound": "tensor", "kernel": "sparse_softmax" + (" (incl. e4m3 quantisation)" if fp8 else ""),
-                     "achieved": achieved, "peak": tc_peak,
-                     "unit": "TFLOP/s", "frac": achieved / tc_peak, "traffic": None if fp8 else traffic,
-                     "peak_source": (f"{src} bf16 burst (MEASURED_PEAKS.json)" if src == "measured" else "fallback")
-                     + (" x 2 (nominal fp8 / bf16)" if fp8 else ""),
-                     "frac_of_sustained": achieved / (pk.get("bf16_tflops_sustained", tc_peak) * ratio),
-                     "frac_of_spec": achieved / (SPEC_TFLOPS * ratio)},
-        "call_roofline": {"roofline_ms": roof_s * 1e3, "frac": roof_s * 1e3 / ms},
-        "kernels": kern,
-        "e2e": {"value": flops_call * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
-                "calls_in_flight": 2,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
-    }
+    line = bench_line(args, w, world, wk, per_kernel, ms, e2e_ms, h2d, d2h, launches_per_step, clk.summary())
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = OracleSample(w, dev_t)
         rec = cb.record(min(cb.run() for _ in range(3 if cb.full else 1)))
@@ -511,6 +551,9 @@ def main():
     ap.add_argument("--workload", default="768p_bf16", choices=sorted(BY_NAME))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--readout", default="fused", choices=["fused", "separate"],
+                    help="readout and merge in the softmax kernel's epilogue (bf16, head_dim 128; the faster "
+                         "path, falls back to separate elsewhere), or in a kernel of their own")
     ap.add_argument("--precision", default="bf16", choices=["bf16", "fp8"],
                     help="operand precision of the softmax branch (bf16 is the headline)")
     args = ap.parse_args()

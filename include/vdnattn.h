@@ -35,6 +35,19 @@
  *     (section 自适应门控融合双分支输出: one output per branch), for callers
  *     that project each branch before summing.
  *
+ * Where the linear read and the merge run is selectable too (same result up
+ * to rounding):
+ *   readout_mode = VDN_READOUT_SEPARATE (default): the softmax kernel stores
+ *     sigmoid(gate_s) * o_s (bf16) and a readout kernel of its own reads it
+ *     back with q, M_c and gate_l and writes out;
+ *     VDN_READOUT_FUSED: the readout, the RMSNorm and the merge run in the
+ *     softmax kernel's epilogue (the frame-7 paragraph combines the linear read
+ *     with the local branch at the query's position): o_s stays in TMEM in
+ *     fp32, q is read once, and the forward/backward scan runs as a kernel of
+ *     its own before the softmax kernel.  Needs bf16 tensors, head_dim 128,
+ *     the BF16 softmax precision and VDN_OUTPUT_MERGED without the VDN_OUT_*
+ *     debug outputs (VDN_ERR_UNSUPPORTED otherwise).
+ *
  * Layouts (row-major, no padding between rows):
  *   q, k, v, gate_s, gate_l, out : [batch, frames*tokens_per_frame, heads, head_dim]
  *   text_k, text_v               : [batch, text_tokens, heads, head_dim]
@@ -91,6 +104,7 @@ typedef enum { VDN_BF16 = 0, VDN_FP32 = 1 } vdn_dtype;
 
 typedef enum { VDN_ANCHOR_LOCAL = 0, VDN_ANCHOR_GLOBAL = 1 } vdn_anchor_query_mode;
 typedef enum { VDN_OUTPUT_MERGED = 0, VDN_OUTPUT_SPLIT = 1 } vdn_output_mode;
+typedef enum { VDN_READOUT_SEPARATE = 0, VDN_READOUT_FUSED = 1 } vdn_readout_mode;
 
 /* Operand precision of the softmax branch's two contractions.  BF16 (default):
  * bf16 operands, fp32 accumulation.  FP8: q, k, v, text_k, text_v quantised
@@ -145,6 +159,7 @@ typedef struct {
   int32_t output_mode;      /* vdn_output_mode; 0 = MERGED.  SPLIT excludes the VDN_OUT_* debug flags */
   int32_t softmax_precision; /* vdn_softmax_precision; 0 = BF16 */
   void* out_linear;         /* SPLIT only: device [B, N, H, d] in dtype, 16-byte aligned; else ignored */
+  int32_t readout_mode;     /* vdn_readout_mode; 0 = SEPARATE */
 } vdn_cfg;
 
 /* Library version, (major << 16) | minor. */
@@ -173,7 +188,8 @@ VDN_API vdn_status vdn_membership_device(const vdn_cfg* cfg, uint8_t* table_dev,
 /* Whole call: staging (fp32 or head_dim 32 only), state build, sparse
  * softmax with the forward/backward scan (and, for bf16 with head_dim 64 or
  * 128, the softmax branch's gate) in the same kernel, readout + merge, all on
- * stream.  out: [B, N, H, d] in dtype (and cfg->out_linear under
+ * stream; under VDN_READOUT_FUSED: state build, scan, then the softmax kernel
+ * with the readout and merge in its epilogue.  out: [B, N, H, d] in dtype (and cfg->out_linear under
  * VDN_OUTPUT_SPLIT). */
 VDN_API vdn_status vdn_hybrid_attn_fwd(const void* q, const void* k, const void* v,
                                const void* text_k, const void* text_v,
@@ -230,6 +246,16 @@ VDN_API vdn_status vdn_softmax_and_scan(const void* q, const void* k, const void
 /* phi(Q) M_c readout, RMSNorm, gates and merge into out. */
 VDN_API vdn_status vdn_readout_merge(const void* q, const void* gate_s, const void* gate_l,
                              void* out, const vdn_cfg* cfg, void* stream);
+/* The steps of a VDN_READOUT_FUSED call: vdn_state_build -> vdn_state_scan ->
+ * vdn_sparse_softmax_merge, which runs the softmax branch and, in the same
+ * kernel's epilogue, the readout, RMSNorm, gates and merge into out (the scan's
+ * readout operands M_c must be in the workspace).  Requirements of
+ * VDN_READOUT_FUSED apply whatever cfg->readout_mode says (VDN_ERR_UNSUPPORTED
+ * otherwise); VDN_ERR_ALIGNMENT for a misaligned pointer. */
+VDN_API vdn_status vdn_sparse_softmax_merge(const void* q, const void* k, const void* v,
+                                            const void* text_k, const void* text_v,
+                                            const void* gate_s, const void* gate_l, void* out,
+                                            const vdn_cfg* cfg, void* stream);
 
 /* For callers that cannot allocate device memory (code running inside another
  * runtime's plugin/operator interface that hands over tensors but no

@@ -9,6 +9,7 @@
 import ctypes
 import os
 import re
+import subprocess
 
 import numpy as np
 import pytest
@@ -102,15 +103,46 @@ def test_validate_rejects_unknown_dtype_and_flags():
     assert lib.vdn_validate(None) == 1
 
 
-def test_cfg_struct_layout_matches_header():
-    """Offsets of the fields that follow the pointers (the ctypes mirror of
-    vdn_cfg must match the C layout on LP64)."""
-    assert vb.VdnCfg.anchor_query_mode.offset == 52
-    assert vb.VdnCfg.workspace.offset == 56
-    assert vb.VdnCfg.export_bwd.offset == 88
-    assert vb.VdnCfg.output_mode.offset == 96
-    assert vb.VdnCfg.out_linear.offset == 104
-    assert ctypes.sizeof(vb.VdnCfg) == 112
+def test_cfg_struct_layout_matches_header(tmp_path):
+    """The ctypes mirror of vdn_cfg has the C layout: every field's offset
+    and the size, as a C compiler lays out the header's struct."""
+    fields = [f[0] for f in vb.VdnCfg._fields_]
+    src = tmp_path / "layout.c"
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "vdnattn.h"', "int main(void) {"]
+    lines += [f'  printf("%zu\\n", offsetof(vdn_cfg, {f}));' for f in fields]
+    lines += ['  printf("%zu\\n", sizeof(vdn_cfg));', "  return 0;", "}"]
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    assert got[:-1] == [getattr(vb.VdnCfg, f).offset for f in fields]
+    assert got[-1] == ctypes.sizeof(vb.VdnCfg)
+
+
+def test_readout_mode_validation():
+    """VDN_READOUT_FUSED: bf16, head_dim 128, bf16 softmax operands and the
+    merged output without debug outputs; anything else is unsupported, and an
+    unknown mode is an invalid argument."""
+    lib = vb.library()
+    ok = vb.Shape(1, 15, 256, 2, 128, 64, 1)
+    assert lib.vdn_validate(ctypes.byref(vb.make_cfg(ok, readout_mode=vb.READOUT_FUSED))) == 0
+    assert lib.vdn_validate(ctypes.byref(vb.make_cfg(ok, readout_mode=vb.READOUT_FUSED,
+                                                      anchor_query_mode=vb.ANCHOR_GLOBAL))) == 0
+    assert lib.vdn_validate(ctypes.byref(vb.make_cfg(ok, readout_mode=2))) == 1
+    unsupported = [
+        vb.make_cfg(vb.Shape(1, 15, 256, 2, 64, 64, 1), readout_mode=vb.READOUT_FUSED),
+        vb.make_cfg(vb.Shape(1, 15, 256, 2, 128, 64, 1, fp32=True), readout_mode=vb.READOUT_FUSED),
+        vb.make_cfg(ok, readout_mode=vb.READOUT_FUSED, softmax_precision=vb.PREC_FP8),
+        vb.make_cfg(ok, readout_mode=vb.READOUT_FUSED, debug_flags=vb.OUT_LINEAR_RAW),
+    ]
+    split = vb.make_cfg(ok, readout_mode=vb.READOUT_FUSED)
+    split.output_mode = vb.OUTPUT_SPLIT
+    unsupported.append(split)
+    for cfg in unsupported:
+        assert lib.vdn_validate(ctypes.byref(cfg)) == 2
+    # the fused step itself checks the requirements whatever the mode says
+    cfg = vb.make_cfg(vb.Shape(1, 15, 256, 2, 64, 64, 1))
+    assert lib.vdn_sparse_softmax_merge(*([None] * 8), ctypes.byref(cfg), None) == 2
 
 
 def test_workspace_bytes():

@@ -379,25 +379,34 @@ def k1_roles(pieces, stages=3):
 # modelled at every step).
 
 
-def k3_roles(items, stages=2, halves=2):
+def k3_roles(items, stages=2, halves=2, fused=False):
+    """Roles of k3_sparse_softmax.cu for items [(query tiles, KV tiles), ...].
+    Buffers: Q0/Q1 (the two query tiles of the Q slot), K/V stages, SPa/SPb
+    (the two halves of a tile's S columns: S, then P over them; under the
+    fused readout also num), O0/O1.  fused: the readout operand M_c travels
+    as one more K/V stage, the softmax warps write phi(Q_t) over Q_t, the MMA
+    thread writes num_t over S_t's columns, the epilogue reads it and
+    releases the columns (RDone)."""
     loads, kv = [], 0
-    for n_item, (_, nkv) in enumerate(items):
+    for n_item, (nt, nkv) in enumerate(items):
         if n_item > 0:
             loads.append(wait("QEmpty", n_item - 1))
-        loads.append(tma("QFull", ("Q", n_item)))
-        for _ in range(nkv):
+        loads.append(tma("QFull", *[(f"Q{t}", ("Q", n_item)) for t in range(nt)]))
+        for _ in range(nkv + (1 if fused else 0)):
             st, r = kv % stages, kv // stages
             loads += [wait(f"KEmpty{st}", r - 1), tma(f"KFull{st}", (f"K{st}", kv)), wait(f"VEmpty{st}", r - 1),
                       tma(f"VFull{st}", (f"V{st}", kv))]
             kv += 1
 
     mma_, kv, p_cnt, s_idx = [], 0, [0, 0], [0, 0]
+    phi_cnt, rd_cnt, rd_pend = [0, 0], [0, 0], [False, False]
 
     parts = ["a", "b"][:halves]
+    regions = ["a", "b"]  # the S columns of a tile, whatever the P handoff
 
     def issue_s(t, n_item, st, kv_):
-        mma_.append(mma(reads=[("Q", n_item), (f"K{st}", kv_)],
-                        writes=[(f"SP{h}{t}", ("S", s_idx[t])) for h in parts]))
+        mma_.append(mma(reads=[(f"Q{t}", ("Q", n_item)), (f"K{st}", kv_)],
+                        writes=[(f"SP{h}{t}", ("S", s_idx[t])) for h in regions]))
         s_idx[t] += 1
 
     for n_item, (nt, nkv) in enumerate(items):
@@ -405,6 +414,10 @@ def k3_roles(items, stages=2, halves=2):
         st = kv % stages
         mma_.append(wait(f"KFull{st}", kv // stages))
         for t in range(nt):
+            if fused and rd_pend[t]:
+                mma_.append(wait(f"RDone{t}", rd_cnt[t]))
+                rd_cnt[t] += 1
+                rd_pend[t] = False
             issue_s(t, n_item, st, kv)
             mma_.append(commit(f"SFull{t}"))
         mma_.append(commit(f"KEmpty{st}"))
@@ -413,8 +426,10 @@ def k3_roles(items, stages=2, halves=2):
             mma_.append(wait(f"VFull{st}", kv // stages))
             for t in range(nt):
                 for h in parts:
+                    # one handoff: P.V reads P over both halves of the columns
+                    held = [h] if halves == 2 else regions
                     mma_.append(wait(f"PFull{'2' if h == 'b' else ''}{t}", p_cnt[t]))
-                    mma_.append(mma(reads=[(f"SP{h}{t}", ("P", p_cnt[t])), (f"V{st}", kv)],
+                    mma_.append(mma(reads=[(f"SP{x}{t}", ("P", p_cnt[t])) for x in held] + [(f"V{st}", kv)],
                                     writes=[(f"O{t}", ("O", n_item, j))]))
                 p_cnt[t] += 1
                 if not has_next:
@@ -428,6 +443,18 @@ def k3_roles(items, stages=2, halves=2):
             if has_next:
                 mma_.append(commit(f"KEmpty{nst}"))
             kv += 1
+        if fused:
+            st = kv % stages
+            mma_ += [wait(f"KFull{st}", kv // stages), wait(f"VFull{st}", kv // stages)]
+            for t in range(nt):
+                mma_.append(wait(f"PhiFull{t}", phi_cnt[t]))
+                phi_cnt[t] += 1
+                mma_.append(mma(reads=[(f"Q{t}", ("phi", n_item)), (f"K{st}", kv), (f"V{st}", kv)],
+                                writes=[(f"SP{h}{t}", ("num", n_item)) for h in regions]))
+                mma_.append(commit(f"RFull{t}"))
+                rd_pend[t] = True
+            mma_ += [commit(f"KEmpty{st}"), commit(f"VEmpty{st}")]
+            kv += 1
         mma_.append(commit("QEmpty"))
     mma_ += [commit("Done"), wait("Done", 0)]
 
@@ -439,13 +466,22 @@ def k3_roles(items, stages=2, halves=2):
                 continue
             for j in range(nkv):
                 sm += [wait(f"SFull{t}", s_cnt)]
-                sm += [x for h in parts for x in (beg(reads=[(f"SP{h}{t}", ("S", s_cnt))]), end(f"SP{h}{t}"))]
-                sm += [beg(writes=[("SPa" + str(t), ("P", s_cnt))]), end(f"SPa{t}"),
-                       beg(writes=[(f"O{t}", ("scaled", n_item, j))]), end(f"O{t}"), arrive(f"PFull{t}")]
+                sm += [x for h in regions for x in (beg(reads=[(f"SP{h}{t}", ("S", s_cnt))]), end(f"SP{h}{t}"))]
+                sm += [beg(writes=[("SPa" + str(t), ("P", s_cnt))]), end(f"SPa{t}")]
+                if halves == 1:
+                    sm += [beg(writes=[("SPb" + str(t), ("P", s_cnt))]), end(f"SPb{t}")]
+                sm += [beg(writes=[(f"O{t}", ("scaled", n_item, j))]), end(f"O{t}"), arrive(f"PFull{t}")]
                 if halves == 2:
                     sm += [beg(writes=[(f"SPb{t}", ("P", s_cnt))]), end(f"SPb{t}"), arrive(f"PFull2{t}")]
                 s_cnt += 1
-            sm += [wait(f"OFull{t}", o_cnt), beg(reads=[(f"O{t}", ("O", n_item, nkv - 1))]), end(f"O{t}")]
+            if fused:
+                sm += [beg(writes=[(f"Q{t}", ("phi", n_item))]), end(f"Q{t}"), arrive(f"PhiFull{t}"),
+                       wait(f"OFull{t}", o_cnt), wait(f"RFull{t}", o_cnt),
+                       beg(reads=[(f"O{t}", ("O", n_item, nkv - 1))] + [(f"SP{h}{t}", ("num", n_item))
+                                                                        for h in regions]),
+                       end(f"O{t}", f"SPa{t}", f"SPb{t}"), arrive(f"RDone{t}")]
+            else:
+                sm += [wait(f"OFull{t}", o_cnt), beg(reads=[(f"O{t}", ("O", n_item, nkv - 1))]), end(f"O{t}")]
             o_cnt += 1
         roles[f"softmax{t}"] = sm
     return roles
@@ -511,8 +547,19 @@ def test_sparse_softmax_protocol(items):
     assert check(k3_roles(items)) > 0
 
 
+K3_FUSED_SCHEDULES = [[(2, 1)], [(2, 2)], [(1, 2)], [(2, 1), (2, 1)], [(2, 2), (1, 1)], [(1, 1), (2, 2)],
+                      [(2, 1), (1, 1), (2, 1)]]
+
+
+@pytest.mark.parametrize("items", K3_FUSED_SCHEDULES, ids=[str(s) for s in K3_FUSED_SCHEDULES])
+def test_fused_readout_protocol(items):
+    assert check(k3_roles(items, fused=True)) > 0
+
+
 def test_fp8_softmax_has_the_bf16_barrier_operations():
-    assert SOURCE_BARRIER_OPS["k3_fp8.cu"] == SOURCE_BARRIER_OPS["k3_sparse_softmax.cu"]
+    """The e4m3 kernel's barrier operations are the bf16 kernel's without
+    the fused readout."""
+    assert SOURCE_BARRIER_OPS["k3_fp8.cu"] == K3_OPS
 
 
 @pytest.mark.parametrize("items", K3_SCHEDULES[:3], ids=[str(s) for s in K3_SCHEDULES[:3]])
@@ -623,6 +670,23 @@ PLANTED = {
     # the softmax warps rescale O before the commit after S (which also
     # covers the previous P.V into O) landed
     "softmax_rescale_before_s": lambda: _move_o_rescale_before_s_wait(k3_roles([(1, 3)])),
+    # fused readout: the next item's first S overwrites num while the epilogue reads it
+    "fused_mma_skips_readout_release": lambda: _drop(k3_roles([(2, 1), (2, 1)], fused=True), "mma",
+                                                     lambda op: op.kind == "wait" and op.bar.startswith("RDone")),
+    # fused readout: the MMA thread reads Q before phi(Q) is written over it
+    "fused_mma_skips_phi": lambda: _drop(k3_roles([(2, 1)], fused=True), "mma",
+                                         lambda op: op.kind == "wait" and op.bar.startswith("PhiFull")),
+    # fused readout: Q released for the next item before the readout MMAs read phi(Q)
+    "fused_q_release_before_readout": lambda: _move_before(
+        k3_roles([(1, 1), (1, 1)], fused=True), "mma", lambda op: op.kind == "commit" and op.bar == "QEmpty",
+        lambda op: op.kind == "wait" and op.bar.startswith("PhiFull")),
+    # fused readout: the epilogue reads num before the readout MMAs completed
+    "fused_epilogue_skips_num": lambda: _drop(k3_roles([(1, 2)], fused=True), "softmax0",
+                                              lambda op: op.kind == "wait" and op.bar == "RFull0"),
+    # fused readout: the softmax warps write phi over Q before the item's last S landed
+    "fused_phi_before_last_s": lambda: _move_before(
+        k3_roles([(1, 2)], fused=True), "softmax0", lambda op: op.kind == "beg" and op.writes
+        and op.writes[0][0] == "Q0", lambda op: op.kind == "wait" and op.bar == "SFull0"),
 }
 
 
@@ -644,22 +708,30 @@ def test_readout_acc_release_wait_is_implied():
 # The barrier operations of each kernel source, in source order, as the role
 # programs above model them.  A change to a kernel's barrier use fails here
 # until the model (and this list) is brought up to date.
+K3_OPS = ("wait:kQEmpty expect_tx:kQFull wait:kKEmpty+st expect_tx:kKFull+st wait:kVEmpty+st "
+          "expect_tx:kVFull+st wait:kQFull wait:kKFull+st mma_commit:kSFull+t "
+          "mma_commit:kKEmpty+st wait:kVFull+st wait:kPFull+t wait:kPFull2+t "
+          "mma_commit:kOFull+t wait:kKFull+nst mma_commit:kSFull+t mma_commit:kVEmpty+st "
+          "mma_commit:kKEmpty+nst mma_commit:kQEmpty mma_commit:kDone wait:kSFull+t "
+          "arrive:kPFull+t arrive:kPFull2+t wait:kOFull+t")
+# the bf16 kernel: the same, with the fused readout's operations in their
+# places (the epilogue of a fused tile is a function ahead of the kernel)
+K3_FUSED_OPS = ("arrive:kPhiFull+t wait:kOFull+t wait:kRFull+t arrive:kRDone+t " + K3_OPS
+                .replace("expect_tx:kVFull+st wait:kQFull",
+                         "expect_tx:kVFull+st wait:kKEmpty+st expect_tx:kKFull+st wait:kVEmpty+st "
+                         "expect_tx:kVFull+st wait:kQFull")
+                .replace("wait:kKFull+st mma_commit:kSFull+t", "wait:kKFull+st wait:kRDone+t mma_commit:kSFull+t")
+                .replace("mma_commit:kKEmpty+nst mma_commit:kQEmpty",
+                         "mma_commit:kKEmpty+nst wait:kKFull+st wait:kVFull+st wait:kPhiFull+t mma_commit:kRFull+t "
+                         "mma_commit:kKEmpty+st mma_commit:kVEmpty+st mma_commit:kQEmpty")
+)
+
 SOURCE_BARRIER_OPS = {
     "k1_state_build.cu": "wait:kEmpty+st expect_tx:kFull+st wait:kAccFull wait:kAccEmpty+a wait:kPhi+st "
                          "mma_commit:kEmpty+st mma_commit:kAccFull+a mma_commit:kDone wait:kFull+st arrive:kPhi+st "
                          "wait:kAccFull+buf arrive:kAccEmpty+buf",
-    "k3_sparse_softmax.cu": "wait:kQEmpty expect_tx:kQFull wait:kKEmpty+st expect_tx:kKFull+st wait:kVEmpty+st "
-                            "expect_tx:kVFull+st wait:kQFull wait:kKFull+st mma_commit:kSFull+t "
-                            "mma_commit:kKEmpty+st wait:kVFull+st wait:kPFull+t wait:kPFull2+t "
-                            "mma_commit:kOFull+t wait:kKFull+nst mma_commit:kSFull+t mma_commit:kVEmpty+st "
-                            "mma_commit:kKEmpty+nst mma_commit:kQEmpty mma_commit:kDone wait:kSFull+t "
-                            "arrive:kPFull+t arrive:kPFull2+t wait:kOFull+t",
-    "k3_fp8.cu": "wait:kQEmpty expect_tx:kQFull wait:kKEmpty+st expect_tx:kKFull+st wait:kVEmpty+st "
-                 "expect_tx:kVFull+st wait:kQFull wait:kKFull+st mma_commit:kSFull+t "
-                 "mma_commit:kKEmpty+st wait:kVFull+st wait:kPFull+t wait:kPFull2+t "
-                 "mma_commit:kOFull+t wait:kKFull+nst mma_commit:kSFull+t mma_commit:kVEmpty+st "
-                 "mma_commit:kKEmpty+nst mma_commit:kQEmpty mma_commit:kDone wait:kSFull+t "
-                 "arrive:kPFull+t arrive:kPFull2+t wait:kOFull+t",
+    "k3_sparse_softmax.cu": K3_FUSED_OPS,
+    "k3_fp8.cu": K3_OPS,
     "k4_merge_tma.cu": "wait:kTBEmpty expect_tx:kTBFull wait:kTAEmpty+qs expect_tx:kTAFull+qs wait:kTGEmpty "
                        "expect_tx:kTGFull wait:kTGEmpty wait:kTBFull wait:kTAReady+s wait:kTAccEmpty+s mma_commit:kTAccFull+s "
                        "mma_commit:kTBEmpty mma_commit:kTDone wait:kTAccFull+s arrive:kTAccEmpty+s wait:kTGFull "

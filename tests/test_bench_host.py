@@ -37,6 +37,54 @@ def test_768p_work_figures():
     assert tiny["k4_bytes"] == 5 * w.N * w.H * w.d * 4 + w.F // w.C * w.H * w.d * (w.d + 1) * 4
 
 
+def test_fused_work_figures():
+    """With the readout fused into the softmax kernel there is no readout
+    kernel: the softmax kernel reads q, k, v, text, both gates and M_c and
+    writes out (five video tensors read, one written)."""
+    w = BY_NAME["768p_bf16"]
+    sep, fus = bench.work(w), bench.work(w, fused=True)
+    assert fus["k4_bytes"] == 0 and fus["softmax_flops"] == sep["softmax_flops"]
+    video = w.N * w.H * w.d * 2
+    assert fus["k3_bytes"] == 6 * video + 2 * w.T * w.H * w.d * 2 + 15 * w.H * w.d * (w.d + 1) * 4
+
+
+@pytest.mark.parametrize("name", sorted({n for n, _ in bench.KERNELS + bench.KERNELS_FUSED} - {"stage"}
+                                        | {"sparse_softmax_fused"}))
+def test_every_timed_kernel_has_a_source_hash(name):
+    """bench.py looks up a DRAM-traffic record for every timed kernel by the
+    hash of its sources; each step name must map to its files, and each
+    Steps method named in the sequences must exist."""
+    assert len(bench.kernel_source_hash(name)) == 12
+    bench.recorded_traffic(name, "768p_bf16")
+    from video_diffusion_hybrid_sparse_b200 import binding as vb
+    for _, method in bench.KERNELS + bench.KERNELS_FUSED:
+        assert callable(getattr(vb.Steps, method))
+
+
+@pytest.mark.parametrize("readout,precision", [("separate", "bf16"), ("fused", "bf16"), ("separate", "fp8")])
+def test_bench_line_from_fake_times(readout, precision):
+    """The JSON line our arm prints, built from made-up kernel times: the
+    contract keys, per-kernel entries of the sequence that ran, and the
+    roofline of the softmax kernel (no GPU needed)."""
+    import argparse
+    args = argparse.Namespace(steps=20, warmup=5, precision=precision, readout=readout)
+    w = BY_NAME["768p_bf16"]
+    fused = readout == "fused"
+    seq = bench.KERNELS_FUSED if fused else bench.KERNELS
+    per_kernel = {n: {"stage": 0.005, "state_build": 0.13, "state_scan": 0.03, "sparse_softmax": 13.0,
+                      "readout_merge": 0.31}[n] for n, _ in seq}
+    ms = sum(per_kernel.values())
+    wk = bench.work(w, precision == "fp8", fused)
+    line = bench.bench_line(args, w, 1, wk, per_kernel, ms, 35.0, 10, 2, 3, {"sm_mhz": 1700.0})
+    json.dumps(line)
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert key in line
+    assert set(line["kernels"]) >= {n for n, _ in seq}
+    assert abs(line["roofline"]["achieved"] - 14.164e12 / 13e-3 / 1e12) < 1.0
+    assert line["readout"] == readout and "readout" not in line["config"]
+
+
 def _worker(rank, world, port, times, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
     dist.init_process_group("gloo", rank=rank, world_size=world)

@@ -26,6 +26,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "po
 EXPORTED = ["vdn_version", "vdn_status_string", "vdn_validate", "vdn_workspace_bytes", "vdn_plan_membership",
             "vdn_membership_device", "vdn_hybrid_attn_fwd", "vdn_stage_inputs", "vdn_state_build",
             "vdn_state_scan", "vdn_sparse_softmax", "vdn_softmax_and_scan", "vdn_readout_merge",
+            "vdn_sparse_softmax_merge",
             "vdn_hybrid_attn_fwd_static",
             "vdn_static_scratch_bytes", "vdn_host_staging_bytes", "vdn_hybrid_attn_fwd_host", "vdn_export_states"]
 
@@ -48,7 +49,7 @@ class VdnCfg(ctypes.Structure):
         ("status_word", ctypes.c_void_p),
         ("export_fwd", ctypes.c_void_p), ("export_bwd", ctypes.c_void_p),
         ("output_mode", ctypes.c_int32), ("softmax_precision", ctypes.c_int32),
-        ("out_linear", ctypes.c_void_p),
+        ("out_linear", ctypes.c_void_p), ("readout_mode", ctypes.c_int32),
     ]
 
 
@@ -78,6 +79,7 @@ def library() -> ctypes.CDLL:
         lib.vdn_sparse_softmax.argtypes = [P, P, P, P, P, C, P]
         lib.vdn_softmax_and_scan.argtypes = [P, P, P, P, P, P, C, P]
         lib.vdn_readout_merge.argtypes = [P, P, P, P, C, P]
+        lib.vdn_sparse_softmax_merge.argtypes = [P, P, P, P, P, P, P, P, C, P]
         lib.vdn_hybrid_attn_fwd_static.argtypes = [P, P, P, P, P, P, P, P, C, P]
         lib.vdn_static_scratch_bytes.restype = ctypes.c_size_t
         lib.vdn_host_staging_bytes.restype = ctypes.c_size_t
@@ -112,11 +114,13 @@ class Shape:
 ANCHOR_LOCAL, ANCHOR_GLOBAL = 0, 1
 OUTPUT_MERGED, OUTPUT_SPLIT = 0, 1
 PREC_BF16, PREC_FP8 = 0, 1
+READOUT_SEPARATE, READOUT_FUSED = 0, 1
 
 
 def make_cfg(s: Shape, *, softmax_scale: float = 0.0, rms_eps: float = -1.0, rms_weight=None,
              debug_flags: int = 0, workspace=None, status=None, export=None,
-             anchor_query_mode: int = ANCHOR_LOCAL, out_linear=None, softmax_precision: int = PREC_BF16) -> VdnCfg:
+             anchor_query_mode: int = ANCHOR_LOCAL, out_linear=None, softmax_precision: int = PREC_BF16,
+             readout_mode: int = READOUT_SEPARATE) -> VdnCfg:
     cfg = VdnCfg()
     cfg.batch, cfg.frames, cfg.tokens_per_frame = s.B, s.F, s.P
     cfg.heads, cfg.head_dim, cfg.text_tokens, cfg.chunk_frames = s.H, s.d, s.T, s.C
@@ -129,6 +133,7 @@ def make_cfg(s: Shape, *, softmax_scale: float = 0.0, rms_eps: float = -1.0, rms
     cfg.output_mode = OUTPUT_SPLIT if out_linear is not None else OUTPUT_MERGED
     cfg.softmax_precision = softmax_precision
     cfg.out_linear = _ptr(out_linear)
+    cfg.readout_mode = readout_mode
     if workspace is not None:
         cfg.workspace = workspace.data_ptr()
         cfg.workspace_bytes = workspace.numel() * workspace.element_size()
@@ -191,13 +196,15 @@ def hybrid_attn_fwd(q, k, v, text_k, text_v, gate_s, gate_l, *, frames: int, chu
                     softmax_scale: float = 0.0, rms_eps: float = -1.0, rms_weight=None, debug_flags: int = 0,
                     workspace=None, status=None, export=None, stream=None,
                     anchor_query_mode: int = ANCHOR_LOCAL, out_linear=None,
-                    softmax_precision: int = PREC_BF16) -> torch.Tensor:
+                    softmax_precision: int = PREC_BF16, readout_mode: int = READOUT_SEPARATE) -> torch.Tensor:
     """The whole hybrid attention call on the current CUDA stream.
 
     q, k, v, gate_s, gate_l: [B, F*P, H, d]; text_k, text_v: [B, T, H, d];
     all contiguous CUDA tensors of one dtype (bf16 or fp32).  With
     ``out_linear`` (a tensor like q) the SPLIT output is written: ``out``
-    gets sigmoid(gate_s) * o_s and ``out_linear`` sigmoid(gate_l) * r."""
+    gets sigmoid(gate_s) * o_s and ``out_linear`` sigmoid(gate_l) * r.
+    ``readout_mode=READOUT_FUSED`` runs the readout and merge in the softmax
+    kernel's epilogue (bf16, head_dim 128, merged output)."""
     s = shape_of(q, text_k, frames, chunk_frames)
     if out is None:
         out = torch.empty_like(q)
@@ -206,7 +213,7 @@ def hybrid_attn_fwd(q, k, v, text_k, text_v, gate_s, gate_l, *, frames: int, chu
     cfg = make_cfg(s, softmax_scale=softmax_scale, rms_eps=rms_eps, rms_weight=rms_weight,
                    debug_flags=debug_flags, workspace=workspace, status=status, export=export,
                    anchor_query_mode=anchor_query_mode, out_linear=out_linear,
-                   softmax_precision=softmax_precision)
+                   softmax_precision=softmax_precision, readout_mode=readout_mode)
     code = library().vdn_hybrid_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(text_k), _ptr(text_v),
                                          gate_s.data_ptr(), gate_l.data_ptr(), out.data_ptr(),
                                          ctypes.byref(cfg), _stream(stream))
@@ -278,7 +285,8 @@ def staging_for(s: Shape, device, split: bool = False) -> torch.Tensor:
 def hybrid_attn_fwd_host(q, k, v, text_k, text_v, gate_s, gate_l, *, frames: int, chunk_frames: int, out=None,
                          softmax_scale: float = 0.0, rms_eps: float = -1.0, rms_weight=None, workspace=None,
                          staging=None, stream=None, anchor_query_mode: int = ANCHOR_LOCAL,
-                         out_linear=None, device="cuda", softmax_precision: int = PREC_BF16) -> torch.Tensor:
+                         out_linear=None, device="cuda", softmax_precision: int = PREC_BF16,
+                         readout_mode: int = READOUT_SEPARATE) -> torch.Tensor:
     """The whole call on HOST tensors (contiguous CPU tensors, ideally pinned),
     copies overlapped with the kernels inside the library.  Returns the host
     ``out``; synchronise ``stream`` (default: the current stream of
@@ -291,7 +299,8 @@ def hybrid_attn_fwd_host(q, k, v, text_k, text_v, gate_s, gate_l, *, frames: int
     if staging is None:
         staging = staging_for(s, device, out_linear is not None)
     cfg = make_cfg(s, softmax_scale=softmax_scale, rms_eps=rms_eps, rms_weight=rms_weight, workspace=workspace,
-                   anchor_query_mode=anchor_query_mode, out_linear=out_linear, softmax_precision=softmax_precision)
+                   anchor_query_mode=anchor_query_mode, out_linear=out_linear, softmax_precision=softmax_precision,
+                   readout_mode=readout_mode)
     code = library().vdn_hybrid_attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(text_k), _ptr(text_v),
                                               gate_s.data_ptr(), gate_l.data_ptr(), out.data_ptr(),
                                               staging.data_ptr(), staging.numel(), ctypes.byref(cfg),
@@ -306,13 +315,14 @@ class Steps:
 
     def __init__(self, q, k, v, text_k, text_v, gate_s, gate_l, out, *, frames, chunk_frames, workspace=None,
                  debug_flags=0, rms_weight=None, export=None, status=None, anchor_query_mode=ANCHOR_LOCAL,
-                 out_linear=None, softmax_precision=PREC_BF16):
+                 out_linear=None, softmax_precision=PREC_BF16, readout_mode=READOUT_SEPARATE):
         self.t = (q, k, v, text_k, text_v, gate_s, gate_l, out)
         self.s = shape_of(q, text_k, frames, chunk_frames)
         self.ws = workspace if workspace is not None else workspace_for(self.s, q.device, softmax_precision)
         self.cfg = make_cfg(self.s, workspace=self.ws, debug_flags=debug_flags, rms_weight=rms_weight,
                             export=export, status=status, anchor_query_mode=anchor_query_mode,
-                            out_linear=out_linear, softmax_precision=softmax_precision)
+                            out_linear=out_linear, softmax_precision=softmax_precision,
+                            readout_mode=readout_mode)
         self.lib = library()
 
     def stage(self, stream=None):
@@ -346,6 +356,21 @@ class Steps:
         q, gs, gl, out = self.t[0], self.t[5], self.t[6], self.t[7]
         _check(self.lib.vdn_readout_merge(q.data_ptr(), gs.data_ptr(), gl.data_ptr(), out.data_ptr(),
                                           ctypes.byref(self.cfg), _stream(stream)), "vdn_readout_merge")
+
+    def softmax_merge(self, stream=None):
+        """The softmax branch with the readout and merge in its epilogue
+        (after state_build and state_scan)."""
+        q, k, v, tk, tv, gs, gl, out = self.t
+        _check(self.lib.vdn_sparse_softmax_merge(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(tk), _ptr(tv),
+                                                 gs.data_ptr(), gl.data_ptr(), out.data_ptr(),
+                                                 ctypes.byref(self.cfg), _stream(stream)),
+               "vdn_sparse_softmax_merge")
+
+    def all_fused(self, stream=None):
+        """The sequence of a call with the fused readout."""
+        self.state_build(stream)
+        self.state_scan(stream)
+        self.softmax_merge(stream)
 
     def all(self, stream=None):
         """The whole call's sequence (the scan inside the softmax kernel)."""

@@ -32,6 +32,14 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The softmax kernel's fused readout epilogue: bf16 tensors of head_dim 128,
+// bf16 softmax operands, the merged output without debug outputs.
+bool fused_readout_supported(const vdn_cfg* cfg) {
+  return cfg->dtype == VDN_BF16 && cfg->head_dim == 128 && cfg->softmax_precision == VDN_PREC_BF16 &&
+         cfg->output_mode == VDN_OUTPUT_MERGED &&
+         !(cfg->debug_flags & (VDN_OUT_SOFTMAX_ONLY | VDN_OUT_LINEAR_ONLY | VDN_OUT_LINEAR_RAW));
+}
+
 vdn_status make_geom(const vdn_cfg* cfg, Geom& g) {
   if (!cfg) return VDN_ERR_INVALID_ARG;
   if (cfg->batch < 1 || cfg->frames < 1 || cfg->tokens_per_frame < 1 || cfg->heads < 1 || cfg->text_tokens < 0 ||
@@ -48,6 +56,8 @@ vdn_status make_geom(const vdn_cfg* cfg, Geom& g) {
   if (cfg->output_mode == VDN_OUTPUT_SPLIT &&
       (cfg->debug_flags & (VDN_OUT_SOFTMAX_ONLY | VDN_OUT_LINEAR_ONLY | VDN_OUT_LINEAR_RAW)))
     return VDN_ERR_INVALID_ARG;
+  if (cfg->readout_mode != VDN_READOUT_SEPARATE && cfg->readout_mode != VDN_READOUT_FUSED) return VDN_ERR_INVALID_ARG;
+  if (cfg->readout_mode == VDN_READOUT_FUSED && !fused_readout_supported(cfg)) return VDN_ERR_UNSUPPORTED;
   if (cfg->frames % cfg->chunk_frames != 0) return VDN_ERR_INVALID_ARG;
   if (cfg->head_dim != 32 && cfg->head_dim != 64 && cfg->head_dim != 128) return VDN_ERR_UNSUPPORTED;
   if (cfg->dtype != VDN_BF16 && cfg->dtype != VDN_FP32) return VDN_ERR_UNSUPPORTED;
@@ -329,7 +339,7 @@ void plan_items(const Geom& g, K3Params& p) {
 // head_dim needs no padding, not under VDN_OUT_SOFTMAX_ONLY), o_s is written
 // as sigmoid(gate_s) * o_s.
 vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s, cudaStream_t st, bool do_scan,
-                               const void* gate_s) {
+                               const void* gate_s, const void* gate_l = nullptr, void* out = nullptr) {
   NvtxRange nvtx("vdn:sparse_softmax");
   Maps m;
   if (!make_maps(m, g, s)) return VDN_ERR_CUDA;
@@ -372,6 +382,14 @@ vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s,
   p.gate_s = (gate_s && tma_readout(g) && !g.fp8 && !(cfg->debug_flags & VDN_OUT_SOFTMAX_ONLY))
                  ? static_cast<const __nv_bfloat16*>(gate_s)
                  : nullptr;
+  if (out) {
+    // fused readout: the kernel writes out itself from the scan's M_c
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.gate_s = static_cast<const __nv_bfloat16*>(gate_s);
+    p.gate_l = static_cast<const __nv_bfloat16*>(gate_l);
+    p.mt = ws(cfg, g.off_mt);
+    p.gamma = cfg->rms_weight;
+  }
   if (do_scan) make_scan_args(cfg, g, p.scan);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -601,6 +619,19 @@ vdn_status vdn_readout_merge(const void* q, const void* gate_s, const void* gate
                             static_cast<cudaStream_t>(stream));
 }
 
+vdn_status vdn_sparse_softmax_merge(const void* q, const void* k, const void* v, const void* text_k,
+                                    const void* text_v, const void* gate_s, const void* gate_l, void* out,
+                                    const vdn_cfg* cfg, void* stream) {
+  Geom g;
+  vdn_status s = make_geom(cfg, g);
+  if (s != VDN_OK) return s;
+  if (!fused_readout_supported(cfg)) return VDN_ERR_UNSUPPORTED;
+  s = check_inputs(cfg, g, {q, k, v, gate_s, gate_l, out}, {text_k, text_v});
+  if (s != VDN_OK) return s;
+  return step_sparse_softmax(cfg, g, kernel_srcs(cfg, g, q, k, v, text_k, text_v), static_cast<cudaStream_t>(stream),
+                             false, gate_s, gate_l, out);
+}
+
 vdn_status vdn_hybrid_attn_fwd(const void* q, const void* k, const void* v, const void* text_k, const void* text_v,
                                const void* gate_s, const void* gate_l, void* out, const vdn_cfg* cfg, void* stream) {
   Geom g;
@@ -615,6 +646,10 @@ vdn_status vdn_hybrid_attn_fwd(const void* q, const void* k, const void* v, cons
   if (poison_ws(cfg, g, st) != cudaSuccess) return VDN_ERR_CUDA;
   if ((s = step_stage(cfg, g, q, k, v, text_k, text_v, st)) != VDN_OK) return s;
   if ((s = step_state_build(cfg, g, src, st)) != VDN_OK) return s;
+  if (cfg->readout_mode == VDN_READOUT_FUSED) {
+    if ((s = step_state_scan(cfg, g, st)) != VDN_OK) return s;
+    return step_sparse_softmax(cfg, g, src, st, false, gate_s, gate_l, out);
+  }
   if ((s = step_sparse_softmax(cfg, g, src, st, true, gate_s)) != VDN_OK) return s;  // the scan runs inside
   return step_readout_merge(cfg, g, src, gate_s, gate_l, out, st);
 }
@@ -688,12 +723,20 @@ vdn_status vdn_hybrid_attn_fwd_host(const void* q, const void* k, const void* v,
     if ((s = step_stage(&c, g, dq, dk, dvv, dtk, dtv, st)) != VDN_OK) return finish(s);
   }
   if ((s = step_state_build(&c, g, src, st)) != VDN_OK) return finish(s);
-  // the softmax branch runs while the gates are still in flight, so here it
-  // leaves o_s ungated and the readout applies both gates
-  if (cudaStreamWaitEvent(st, ev[2], 0) != cudaSuccess) return finish(VDN_ERR_CUDA);
-  if ((s = step_sparse_softmax(&c, g, src, st, true, nullptr)) != VDN_OK) return finish(s);  // the scan runs inside
-  if (cudaStreamWaitEvent(st, ev[3], 0) != cudaSuccess) return finish(VDN_ERR_CUDA);
-  if ((s = step_readout_merge(&c, g, src, dv + h.gs, dv + h.gl, dv + h.out, st)) != VDN_OK) return finish(s);
+  if (c.readout_mode == VDN_READOUT_FUSED) {
+    // the scan while q and the gates land; the fused softmax kernel needs all three
+    if ((s = step_state_scan(&c, g, st)) != VDN_OK) return finish(s);
+    if (cudaStreamWaitEvent(st, ev[3], 0) != cudaSuccess) return finish(VDN_ERR_CUDA);
+    if ((s = step_sparse_softmax(&c, g, src, st, false, dv + h.gs, dv + h.gl, dv + h.out)) != VDN_OK)
+      return finish(s);
+  } else {
+    // the softmax branch runs while the gates are still in flight, so here it
+    // leaves o_s ungated and the readout applies both gates
+    if (cudaStreamWaitEvent(st, ev[2], 0) != cudaSuccess) return finish(VDN_ERR_CUDA);
+    if ((s = step_sparse_softmax(&c, g, src, st, true, nullptr)) != VDN_OK) return finish(s);  // the scan runs inside
+    if (cudaStreamWaitEvent(st, ev[3], 0) != cudaSuccess) return finish(VDN_ERR_CUDA);
+    if ((s = step_readout_merge(&c, g, src, dv + h.gs, dv + h.gl, dv + h.out, st)) != VDN_OK) return finish(s);
+  }
   ce = cudaMemcpyAsync(out, dv + h.out, vid, cudaMemcpyDeviceToHost, st);
   if (ce == cudaSuccess && c.output_mode == VDN_OUTPUT_SPLIT)
     ce = cudaMemcpyAsync(cfg->out_linear, dv + h.out_lin, vid, cudaMemcpyDeviceToHost, st);

@@ -45,10 +45,31 @@
 // S_t(j+1) also covers PV_t(j), so when the softmax of tile t sees S_t(j+1)
 // its O_t is quiescent and may be rescaled (before the first half is handed
 // over).
+//
+// Fused readout (kFused, bf16 and head_dim 128): the linear branch's read and
+// the gated merge run in this kernel's item epilogue instead of a readout
+// kernel of their own (the frame-7 paragraph of 双分支混合注意力机制 combines
+// the linear read with the local branch at the query's position), so o_s is
+// never written and q is read once.  The forward/backward scan has then run
+// before this kernel (its readout operands M_c must be complete).  Per item:
+//  * the producer sends M_c of the item's (batch, chunk, head) through the
+//    K/V ring as one more stage, the hi image in the K slot and the lo image
+//    in the V slot (rows 0..127 of each: the numerator columns);
+//  * after handing over the last P of the item, softmax warpgroup t applies
+//    phi to its query row in place in Q_t (its S MMAs are complete) and forms
+//    the denominator phi(q) . z on the CUDA cores (z = row 128 of the images);
+//  * the MMA thread issues num_t = phi(Q_t) M_hi + phi(Q_t) M_lo into S_t's
+//    TMEM columns (behind the item's last P.V, which reads P_t from them),
+//    then releases the stage and Q;
+//  * the epilogue reads num_t and O_t: o_l = num / den (0 for an empty state
+//    or a GLOBAL anchor segment), r = o_l / sqrt(mean(o_l^2) + eps) * gamma,
+//    out = sigmoid(g_s) O / l + sigmoid(g_l) r; then S_t's columns are free
+//    for the next item's first S_t (kRDone).
 #include <type_traits>
 
 #include "k3_common.cuh"
 #include "kernels.h"
+#include "phi.cuh"
 #include "scan.cuh"
 #include "sm100.cuh"
 
@@ -68,6 +89,17 @@ struct K3Layout {
   static constexpr int kBar = kV + kStages * kTile;
   static constexpr int kBytes = kBar + 256 + 1024;  // + barriers + alignment slack
 };
+
+// Barriers of the fused readout, after the common ones.  kPhiFull + t:
+// phi(Q_t) is in shared memory (128 arrivals); kRFull + t: num_t is in TMEM;
+// kRDone + t: the epilogue has read num_t (128 arrivals).
+enum { kPhiFull = kNumBars, kRFull = kNumBars + 2, kRDone = kNumBars + 4, kNumBarsAll = kNumBars + 6 };
+
+// Readout operand image of one (batch, chunk, head) at head_dim 128 (scan.cuh):
+// hi then lo, each two K halves of 144 rows x 128 bytes; rows 0..127 hold the
+// numerator columns, row 128 holds z.
+constexpr int kMtHalf = 144 * 128;
+constexpr int kMtImage = 2 * kMtHalf;
 
 constexpr int kThreads = 384;  // warp 0 loads, warp 1 MMA, warps 2-3 scan, warps 4-11 softmax
 constexpr uint32_t kLaunchRegs = 168;  // per thread at launch (65536 / 384, in steps of 8)
@@ -113,9 +145,133 @@ __device__ __forceinline__ void scan_dynamic(const K3Params& p, uint32_t lane) {
   }
 }
 
+// The fused readout and merge of query tile t of an item (kFused), run by the
+// tile's softmax warpgroup after it handed over the item's last P: phi(Q_t)
+// in place and den, the wait for O_t and num_t, the RMSNorm and the merge.
+// Returns false when a wait ran out.
+template <int D>
+__device__ __forceinline__ bool fused_readout_tile(const K3Params& p, int item, int t, int row, uint32_t lane_base,
+                                                uint32_t tmem, uint8_t* sQ, uint64_t* bars, uint32_t o_cnt,
+                                                float l_run, CtaAbort ab) {
+  using L = K3Layout<D>;
+  const Geom& g = p.g;
+  const Item it = decode_item(item, p);
+  const bool no_read = it.c == kAllFrames || state_tokens(it.c, g) == 0;
+  const uint8_t* img =
+      p.mt + (((size_t)it.b * g.Nc + (it.c == kAllFrames ? 0 : it.c)) * g.H + it.h) * (size_t)kMtImage * 2;
+  const int nrows = min(kBlockM, it.nrows - t * kBlockM);  // valid rows of this tile
+  const size_t row_el = (((size_t)it.b * g.N + (size_t)(it.row0 + t * kBlockM + row)) * g.H + it.h) * D;
+  const uint4* gsp = reinterpret_cast<const uint4*>(p.gate_s + row_el);
+  const uint4* glp = reinterpret_cast<const uint4*>(p.gate_l + row_el);
+  // phi(q) in place over this thread's row of Q_t (K-major, 128-byte
+  // swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)) and
+  // den = phi(q) . (z_hi + z_lo), with the bf16 phi(q) the MMA reads
+  uint8_t* qrow = sQ + t * L::kTile + row * 128;
+  uint64_t den2 = f32x2_pack(0.f, 0.f);
+#pragma unroll 1
+  for (int bx = 0; bx < 2; ++bx) {
+    const uint4* zh = reinterpret_cast<const uint4*>(img + bx * kMtHalf + 128 * 128);
+    const uint4* zl = reinterpret_cast<const uint4*>(img + kMtImage + bx * kMtHalf + 128 * 128);
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+      uint4* pq = reinterpret_cast<uint4*>(qrow + bx * 16384 + ((ch ^ (row & 7)) << 4));
+      const uint4 w = *pq;
+      const uint4 f = make_uint4(phi_bf16x2(w.x), phi_bf16x2(w.y), phi_bf16x2(w.z), phi_bf16x2(w.w));
+      *pq = f;
+      const uint4 a = __ldg(zh + ch), b = __ldg(zl + ch);
+      const uint32_t fw[4] = {f.x, f.y, f.z, f.w}, aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        den2 = f32x2_fma(f32x2_pack(bf16_lo(fw[e]), bf16_hi(fw[e])),
+                         f32x2_add(f32x2_pack(bf16_lo(aw[e]), bf16_hi(aw[e])),
+                                   f32x2_pack(bf16_lo(bw[e]), bf16_hi(bw[e]))),
+                         den2);
+    }
+  }
+  fence_proxy_async_smem();
+  mbar_arrive(&bars[kPhiFull + t]);
+  bool got = mbar_wait(&bars[kOFull + t], o_cnt & 1, ab);
+  got = got && mbar_wait(&bars[kRFull + t], o_cnt & 1, ab);  // one num_t per O_t
+  if (__any_sync(0xffffffffu, !got)) return false;
+  tc_fence_after();
+  float d0, d1;
+  f32x2_unpack(den2, d0, d1);
+  const float inv_den = no_read ? 0.f : 1.0f / (d0 + d1);
+  const uint32_t n_addr = tmem_addr(tmem, lane_base, t * 128);
+  const uint32_t o_addr = tmem_addr(tmem, lane_base, 256 + t * D);
+  // the row's sum of squares of num (o_l = num / den)
+  uint64_t ss2 = f32x2_pack(0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < D / 32; ++i) {
+    uint32_t v[32];
+    tmem_ld32(n_addr + 32 * i, v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint64_t x = f32x2_pack(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+      ss2 = f32x2_fma(x, x, ss2);
+    }
+  }
+  float s0, s1;
+  f32x2_unpack(ss2, s0, s1);
+  const float scale = inv_den * rsqrtf((s0 + s1) * inv_den * inv_den / (float)g.d + g.eps);  // r = num * scale
+  const uint64_t scale2 = f32x2_pack(scale, scale);
+  const float inv_l = 1.0f / l_run;
+  const uint64_t inv_l2 = f32x2_pack(inv_l, inv_l);
+  const float* gam = p.gamma ? p.gamma + (size_t)it.h * D : nullptr;
+#pragma unroll 1
+  for (int i = 0; i < D / 32; ++i) {
+    uint32_t nm[32], o[32];
+    tmem_ld32(n_addr + 32 * i, nm);
+    tmem_ld32(o_addr + 32 * i, o);
+    tmem_wait_ld();
+    if (i + 1 == D / 32) {
+      tc_fence_before();
+      mbar_arrive(&bars[kRDone + t]);  // S_t's columns may take the next item's S_t
+    }
+    if (row < nrows) {
+      // the gates of these 32 columns (in L2 since the item's start): loaded
+      // only once num and O are in registers, so that no gate registers are
+      // held across the TMEM reads (holding them, or the next group's,
+      // spilled registers of the KV loop and cost more than the load waits)
+      uint4 cs[4], cl[4];
+#pragma unroll
+      for (int v4 = 0; v4 < 4; ++v4) {
+        cs[v4] = __ldg(gsp + 4 * i + v4);
+        cl[v4] = __ldg(glp + 4 * i + v4);
+      }
+      uint4* d4 = reinterpret_cast<uint4*>(p.out + row_el + 32 * i);
+#pragma unroll
+      for (int v4 = 0; v4 < 4; ++v4) {
+        const uint32_t sw[4] = {cs[v4].x, cs[v4].y, cs[v4].z, cs[v4].w};
+        const uint32_t lw[4] = {cl[v4].x, cl[v4].y, cl[v4].z, cl[v4].w};
+        uint32_t ow[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int k = 8 * v4 + 2 * e;
+          // sigmoid(g_s) o_s + sigmoid(g_l) r
+          const uint64_t st2 = f32x2_mul(sigmoid2_tanh(f32x2_pack(bf16_lo(sw[e]), bf16_hi(sw[e]))),
+                                         f32x2_mul(f32x2_pack(__uint_as_float(o[k]), __uint_as_float(o[k + 1])),
+                                                   inv_l2));
+          uint64_t rr2 = f32x2_mul(f32x2_pack(__uint_as_float(nm[k]), __uint_as_float(nm[k + 1])), scale2);
+          if (gam) {
+            const float2 g2 = __ldg(reinterpret_cast<const float2*>(gam + 32 * i + k));
+            rr2 = f32x2_mul(rr2, f32x2_pack(g2.x, g2.y));
+          }
+          float y0, y1;
+          f32x2_unpack(f32x2_fma(sigmoid2_tanh(f32x2_pack(bf16_lo(lw[e]), bf16_hi(lw[e]))), rr2, st2), y0, y1);
+          ow[e] = pack_bf16x2(y0, y1);
+        }
+        d4[v4] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+      }
+    }
+  }
+  return true;
+}
+
 }  // namespace
 
-template <int D>
+template <int D, bool kFused>
 __global__ void __launch_bounds__(kThreads, 1)
     k3_sparse_softmax(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_tk,
@@ -124,8 +280,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + kNumBars * 8);
-  int* abort_flag = reinterpret_cast<int*>(smem + L::kBar + kNumBars * 8 + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + kNumBarsAll * 8);
+  int* abort_flag = reinterpret_cast<int*>(smem + L::kBar + kNumBarsAll * 8 + 4);
+  static_assert(kNumBarsAll * 8 + 8 <= 256, "barrier region");
+  static_assert(!kFused || D == 128, "the fused readout is built for head_dim 128");
 
   const Geom& g = p.g;
   const uint32_t warp = warp_id();
@@ -147,6 +305,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[kOFull + t], 1);
     }
     mbar_init(&bars[kDone], 1);
+    if (kFused) {
+      for (int t = 0; t < 2; ++t) {
+        mbar_init(&bars[kPhiFull + t], kBlockM);
+        mbar_init(&bars[kRFull + t], 1);
+        mbar_init(&bars[kRDone + t], kBlockM);
+      }
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -207,6 +372,25 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_2d(sV + st * L::kTile + bx * 16384, mv, &bars[kVFull + st], it.h * D + bx * 64, base + off);
           }
         }
+        if (kFused && ok) {
+          // the item's readout operand as one more stage: M_hi rows 0..127 in
+          // the K slot, M_lo rows 0..127 in the V slot (a GLOBAL anchor
+          // segment reads nothing through the states; it takes chunk 0's
+          // operand and the epilogue zeroes its read)
+          const int st = kv_cnt % L::kStages;
+          const uint32_t ph = (kv_cnt / L::kStages) & 1;
+          const int mc = it.c == kAllFrames ? 0 : it.c;
+          const uint8_t* img = p.mt + (((size_t)it.b * g.Nc + mc) * g.H + it.h) * (size_t)kMtImage * 2;
+          ++kv_cnt;
+          if (!mbar_wait(&bars[kKEmpty + st], ph ^ 1, ab)) { ok = false; break; }
+          mbar_expect_tx(&bars[kKFull + st], L::kTile);
+          for (int bx = 0; bx < 2; ++bx)
+            bulk_load(sK + st * L::kTile + bx * 16384, img + bx * kMtHalf, 16384, &bars[kKFull + st]);
+          if (!mbar_wait(&bars[kVEmpty + st], ph ^ 1, ab)) { ok = false; break; }
+          mbar_expect_tx(&bars[kVFull + st], L::kTile);
+          for (int bx = 0; bx < 2; ++bx)
+            bulk_load(sV + st * L::kTile + bx * 16384, img + kMtImage + bx * kMtHalf, 16384, &bars[kVFull + st]);
+        }
       }
       if (!ok) {
         // Let loads already in flight land before the CTA's shared memory goes away.
@@ -226,7 +410,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t q_desc0 = smem_desc(smem_u32(sQ), 16, 1024, kLayoutSw128);
       const uint64_t k_desc0 = smem_desc(smem_u32(sK), 16, 1024, kLayoutSw128);
       const uint64_t v_desc0 = smem_desc(smem_u32(sV), 16384, 1024, kLayoutSw128);
+      const uint64_t m_lo_desc0 = smem_desc(smem_u32(sV), 16, 1024, kLayoutSw128);  // fused readout: M_lo, K-major
       uint32_t kv_cnt = 0, item_cnt = 0, p_cnt[2] = {0, 0};
+      // fused readout: phi(Q_t) hand-overs seen, kRDone phases waited, and
+      // whether S_t's columns still hold a num_t the epilogue may be reading
+      uint32_t phi_cnt[2] = {0, 0}, rd_cnt[2] = {0, 0};
+      bool rd_pend[2] = {false, false};
       bool ok = true;
 
       auto issue_qk = [&](int t, int st) {
@@ -251,6 +440,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
 
+      // num_t = phi(Q_t) (M_hi + M_lo) over the numerator columns, into S_t's columns
+      auto issue_readout = [&](int t, int st) {
+        const uint32_t d_tmem = tmem + t * 128;
+        const uint64_t qd = q_desc0 + (uint64_t)((t * L::kTile) >> 4);
+        const uint64_t hd = k_desc0 + (uint64_t)((st * L::kTile) >> 4);
+        const uint64_t ld = m_lo_desc0 + (uint64_t)((st * L::kTile) >> 4);
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            mma_ss(d_tmem, qd + off, (hl ? ld : hd) + off, idesc_qk, (hl | kk) ? 1u : 0u);
+          }
+      };
+
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++item_cnt) {
         const Item it = decode_item(item, p);
         const int nkv = seg_kv_tiles(it.c, g);
@@ -260,9 +464,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&bars[kKFull + st], (kv_cnt / L::kStages) & 1, ab)) { ok = false; break; }
           tc_fence_after();
           for (int t = 0; t < it.ntiles; ++t) {
+            if (kFused && rd_pend[t]) {
+              // S_t's columns hold the previous item's num_t until its epilogue has read it
+              if (!mbar_wait(&bars[kRDone + t], rd_cnt[t] & 1, ab)) { ok = false; break; }
+              ++rd_cnt[t];
+              rd_pend[t] = false;
+              tc_fence_after();
+            }
             issue_qk(t, st);
             mma_commit(&bars[kSFull + t]);
           }
+          if (!ok) break;
           mma_commit(&bars[kKEmpty + st]);
         }
         for (int j = 0; j < nkv; ++j, ++kv_cnt) {
@@ -294,6 +506,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (has_next) mma_commit(&bars[kKEmpty + nst]);
         }
         if (!ok) break;
+        if (kFused) {
+          // the readout stage: M_hi in the K slot, M_lo in the V slot
+          const int st = kv_cnt % L::kStages;
+          const uint32_t ph = (kv_cnt / L::kStages) & 1;
+          ++kv_cnt;
+          if (!mbar_wait(&bars[kKFull + st], ph, ab) || !mbar_wait(&bars[kVFull + st], ph, ab)) {
+            ok = false;
+            break;
+          }
+          for (int t = 0; t < it.ntiles; ++t) {
+            if (!mbar_wait(&bars[kPhiFull + t], phi_cnt[t] & 1, ab)) { ok = false; break; }
+            ++phi_cnt[t];
+            tc_fence_after();
+            issue_readout(t, st);
+            mma_commit(&bars[kRFull + t]);
+            rd_pend[t] = true;
+          }
+          if (!ok) break;
+          mma_commit(&bars[kKEmpty + st]);
+          mma_commit(&bars[kVEmpty + st]);
+        }
         mma_commit(&bars[kQEmpty]);
       }
       // All MMAs issued by this thread complete before TMEM is released.
@@ -330,6 +563,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               p.gate_s + (((size_t)it.b * g.N + (size_t)(it.row0 + t * kBlockM + row)) * g.H + it.h) * D;
 #pragma unroll
           for (int i = 0; i < D / 64; ++i) prefetch_l2(gr + 64 * i);
+          if (kFused) {
+            const __nv_bfloat16* gl = p.gate_l + (gr - p.gate_s);
+#pragma unroll
+            for (int i = 0; i < D / 64; ++i) prefetch_l2(gl + 64 * i);
+          }
         }
       }
       if (t >= ntiles) continue;
@@ -428,6 +666,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_run = l_run * alpha + ((c0 + c1) + (c2 + c3));
       }
       if (!ok) break;
+      if constexpr (kFused) {
+        // ---------------------------------------------------------- fused readout and merge
+        const bool good = fused_readout_tile<D>(p, item, t, row, lane_base, tmem, sQ, bars, o_cnt, l_run, ab);
+        ++o_cnt;
+        if (!good) { ok = false; break; }
+        continue;
+      }
       // ---------------------------------------------------------- epilogue: o_s = O / l
       // (times sigmoid(g_s) when the gate is given: the softmax branch's term
       // of the gated merge; the gate logits were brought into L2 at the start
@@ -490,17 +735,23 @@ size_t k3_smem_bytes(int Dp) {
   return need < 118 * 1024 ? 118 * 1024 : need;
 }
 
-template <int D>
+template <int D, bool kFused>
 static cudaError_t launch_k3(const Maps& m, const K3Params& p, int grid, cudaStream_t st) {
   const size_t smem = k3_smem_bytes(D);
-  cudaError_t e = cudaFuncSetAttribute(k3_sparse_softmax<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e =
+      cudaFuncSetAttribute(k3_sparse_softmax<D, kFused>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k3_sparse_softmax<D><<<grid, kThreads, smem, st>>>(m.q, m.k, m.v, m.tk, m.tv, p);
+  k3_sparse_softmax<D, kFused><<<grid, kThreads, smem, st>>>(m.q, m.k, m.v, m.tk, m.tv, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_sparse_softmax(const Maps& m, const K3Params& p, int grid, cudaStream_t st) {
-  return p.g.Dp == 128 ? launch_k3<128>(m, p, grid, st) : launch_k3<64>(m, p, grid, st);
+  if (p.out) {
+    // fused readout: bf16, head_dim 128, scan already run, gates and out given
+    if (p.g.Dp != 128 || p.g.d != 128 || p.do_scan || !p.gate_s || !p.gate_l || !p.mt) return cudaErrorInvalidValue;
+    return launch_k3<128, true>(m, p, grid, st);
+  }
+  return p.g.Dp == 128 ? launch_k3<128, false>(m, p, grid, st) : launch_k3<64, false>(m, p, grid, st);
 }
 
 }  // namespace vdn

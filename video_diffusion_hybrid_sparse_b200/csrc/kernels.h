@@ -44,6 +44,12 @@ struct K3Params {
   int do_scan;             // the kernel also runs the forward/backward scan (scan below)
   unsigned long long* scan_counter;  // next scan unit to take (workspace; zeroed by the state build)
   ScanArgs scan;
+  // Fused readout (out != null; bf16, head_dim 128, do_scan 0): the kernel
+  // writes the merged output itself from M_c, which the scan has written.
+  __nv_bfloat16* out;      // [B, N, H, 128] bf16
+  const __nv_bfloat16* gate_l;  // [B, N, H, 128]
+  const uint8_t* mt;       // readout operand images per (b, chunk, head) (scan.cuh)
+  const float* gamma;      // [H, 128] fp32 or null (ones)
 };
 
 struct K1Params {
