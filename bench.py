@@ -441,7 +441,7 @@ def bench_line(args, w, world, wk, per_kernel, ms, e2e_ms, h2d, d2h, launches_pe
         "call_roofline": {"roofline_ms": roof_s * 1e3, "frac": roof_s * 1e3 / ms},
         "kernels": kern,
         "e2e": {"value": flops_call * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
-                "calls_in_flight": 2,
+                "calls_in_flight": 2, "readout": "separate",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
@@ -505,11 +505,14 @@ def run_ours(args, w, world, rank, local):
     d2h = host_out.numel() * host_out.element_size()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n_e2e = max(4, args.steps // 4)
-    # Two calls in flight, as a server streaming requests would run them: call
-    # i on stream i % 2 with its own staging buffer, workspace and host output,
-    # so the copy-out of one call overlaps the copy-in of the next (the two
-    # PCIe directions); the library's copy stream still takes the copies-in
-    # one call after the other.
+    # The host calls use the separate readout whatever --readout says: there
+    # the softmax kernel runs while the gates are still being copied in,
+    # which the fused kernel (it reads the gates) cannot (36.9 against 35.4
+    # ms per call at 768p).  Two calls in flight, as a server streaming
+    # requests would run them: call i on stream i % 2 with its own staging
+    # buffer, workspace and host output, so the copy-out of one call overlaps
+    # the copy-in of the next (the two PCIe directions); the library's copy
+    # stream still takes the copies-in one call after the other.
     streams = [stream, torch.cuda.Stream()]
     stagings = [vb.new_staging(steps.s, dev["q"].device) for _ in range(2)]
     wss = [steps.ws, vb.new_workspace(steps.s, dev["q"].device, prec)]
@@ -524,7 +527,8 @@ def run_ours(args, w, world, rank, local):
         k = i % 2
         vb.hybrid_attn_fwd_host(host["q"], host["k"], host["v"], host["text_k"], host["text_v"], host["gate_s"],
                                 host["gate_l"], frames=w.F, chunk_frames=w.C, out=host_outs[k], workspace=wss[k],
-                                staging=stagings[k], stream=streams[k], softmax_precision=prec, readout_mode=mode)
+                                staging=stagings[k], stream=streams[k], softmax_precision=prec,
+                                readout_mode=vb.READOUT_SEPARATE)
     joined = torch.cuda.Event()
     joined.record(streams[1])
     stream.wait_event(joined)
