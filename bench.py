@@ -42,14 +42,12 @@ METRIC = "hybrid-attn ms/call & TFLOP/s at 768p-shaped latent, 1×B200, % of roo
 SPEC_TFLOPS, SPEC_GBS = 2250.0, 8000.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # Steps timed separately (CUDA events between them), with the Steps method
-# that runs each.  Separate readout (the default): the forward/backward scan
-# runs inside the softmax kernel (its otherwise idle warps), the readout and
-# merge in a kernel of their own.  Fused readout: the scan is a kernel of its
-# own and the softmax kernel's epilogue does the readout and merge.
+# that runs each.  The forward/backward scan runs inside the softmax kernel
+# (its otherwise idle warps) on both paths; the readout and merge run in a
+# kernel of their own (separate) or in the softmax kernel's epilogue (fused).
 KERNELS = [("stage", "stage"), ("state_build", "state_build"), ("sparse_softmax", "softmax_and_scan"),
            ("readout_merge", "readout_merge")]
-KERNELS_FUSED = [("stage", "stage"), ("state_build", "state_build"), ("state_scan", "state_scan"),
-                 ("sparse_softmax", "softmax_merge")]
+KERNELS_FUSED = [("stage", "stage"), ("state_build", "state_build"), ("sparse_softmax", "softmax_merge")]
 
 
 # ---------------------------------------------------------------- algorithmic work
@@ -406,7 +404,7 @@ def bench_line(args, w, world, wk, per_kernel, ms, e2e_ms, h2d, d2h, launches_pe
     k3_key = "sparse_softmax_fused" if fused else "sparse_softmax"
     traffic = recorded_traffic(k3_key, w.name)
     kern = {}
-    hbm_steps = (("state_build", wk["k1_bytes"], "hbm"), ("state_scan", wk["k2_bytes"], "hbm")) if fused else \
+    hbm_steps = (("state_build", wk["k1_bytes"], "hbm"),) if fused else \
         (("state_build", wk["k1_bytes"], "hbm"), ("readout_merge", wk["k4_bytes"], "hbm"))
     for n, amount, bound in hbm_steps + (("sparse_softmax", wk["softmax_flops"], "tensor"),):
         t = per_kernel[n] * 1e-3
@@ -421,8 +419,7 @@ def bench_line(args, w, world, wk, per_kernel, ms, e2e_ms, h2d, d2h, launches_pe
     if fused:
         kern["sparse_softmax"]["includes"] = "readout, RMSNorm and gated merge (fused epilogue)"
         kern["sparse_softmax"]["bytes"] = wk["k3_bytes"]
-    else:
-        kern["state_scan"] = {"ms": None, "in": "sparse_softmax (warps 2-3)", "bytes": wk["k2_bytes"]}
+    kern["state_scan"] = {"ms": None, "in": "sparse_softmax (warps 2-3)", "bytes": wk["k2_bytes"]}
     roof_s = wk["softmax_flops"] / (tc_peak * 1e12) + wk["linear_bytes"] / (hbm * 1e9)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,

@@ -43,8 +43,7 @@
  *     VDN_READOUT_FUSED: the readout, the RMSNorm and the merge run in the
  *     softmax kernel's epilogue (the frame-7 paragraph combines the linear read
  *     with the local branch at the query's position): o_s stays in TMEM in
- *     fp32, q is read once, and the forward/backward scan runs as a kernel of
- *     its own before the softmax kernel.  Needs bf16 tensors, head_dim 128,
+ *     fp32 and q is read once.  Needs bf16 tensors, head_dim 128,
  *     the BF16 softmax precision and VDN_OUTPUT_MERGED without the VDN_OUT_*
  *     debug outputs (VDN_ERR_UNSUPPORTED otherwise).
  *
@@ -188,8 +187,8 @@ VDN_API vdn_status vdn_membership_device(const vdn_cfg* cfg, uint8_t* table_dev,
 /* Whole call: staging (fp32 or head_dim 32 only), state build, sparse
  * softmax with the forward/backward scan (and, for bf16 with head_dim 64 or
  * 128, the softmax branch's gate) in the same kernel, readout + merge, all on
- * stream; under VDN_READOUT_FUSED: state build, scan, then the softmax kernel
- * with the readout and merge in its epilogue.  out: [B, N, H, d] in dtype (and cfg->out_linear under
+ * stream; under VDN_READOUT_FUSED: state build, then the softmax kernel with
+ * the scan inside and the readout and merge in its epilogue.  out: [B, N, H, d] in dtype (and cfg->out_linear under
  * VDN_OUTPUT_SPLIT). */
 VDN_API vdn_status vdn_hybrid_attn_fwd(const void* q, const void* k, const void* v,
                                const void* text_k, const void* text_v,
@@ -246,12 +245,14 @@ VDN_API vdn_status vdn_softmax_and_scan(const void* q, const void* k, const void
 /* phi(Q) M_c readout, RMSNorm, gates and merge into out. */
 VDN_API vdn_status vdn_readout_merge(const void* q, const void* gate_s, const void* gate_l,
                              void* out, const vdn_cfg* cfg, void* stream);
-/* The steps of a VDN_READOUT_FUSED call: vdn_state_build -> vdn_state_scan ->
- * vdn_sparse_softmax_merge, which runs the softmax branch and, in the same
- * kernel's epilogue, the readout, RMSNorm, gates and merge into out (the scan's
- * readout operands M_c must be in the workspace).  Requirements of
- * VDN_READOUT_FUSED apply whatever cfg->readout_mode says (VDN_ERR_UNSUPPORTED
- * otherwise); VDN_ERR_ALIGNMENT for a misaligned pointer. */
+/* The steps of a VDN_READOUT_FUSED call: vdn_state_build ->
+ * vdn_sparse_softmax_merge, which runs the softmax branch, the
+ * forward/backward scan (in otherwise idle warps, as vdn_softmax_and_scan) and,
+ * in the kernel's item epilogue, the readout, RMSNorm, gates and merge into
+ * out; it must follow vdn_state_build on the same workspace (stream order).
+ * Requirements of VDN_READOUT_FUSED apply whatever cfg->readout_mode says
+ * (VDN_ERR_UNSUPPORTED otherwise); VDN_ERR_ALIGNMENT for a misaligned
+ * pointer; VDN_ERR_INVALID_ARG for VDN_EXPORT_STATES without export buffers. */
 VDN_API vdn_status vdn_sparse_softmax_merge(const void* q, const void* k, const void* v,
                                             const void* text_k, const void* text_v,
                                             const void* gate_s, const void* gate_l, void* out,

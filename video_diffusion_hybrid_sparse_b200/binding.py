@@ -358,8 +358,8 @@ class Steps:
                                           ctypes.byref(self.cfg), _stream(stream)), "vdn_readout_merge")
 
     def softmax_merge(self, stream=None):
-        """The softmax branch with the readout and merge in its epilogue
-        (after state_build and state_scan)."""
+        """The softmax branch with the scan inside and the readout and merge
+        in its epilogue (after state_build)."""
         q, k, v, tk, tv, gs, gl, out = self.t
         _check(self.lib.vdn_sparse_softmax_merge(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(tk), _ptr(tv),
                                                  gs.data_ptr(), gl.data_ptr(), out.data_ptr(),
@@ -369,7 +369,6 @@ class Steps:
     def all_fused(self, stream=None):
         """The sequence of a call with the fused readout."""
         self.state_build(stream)
-        self.state_scan(stream)
         self.softmax_merge(stream)
 
     def all(self, stream=None):

@@ -115,6 +115,7 @@ vdn_status make_geom(const vdn_cfg* cfg, Geom& g) {
   g.off_parts = off; off = align_up(off + (size_t)g.n_part_slots * state_bytes, 1024);
   g.off_segst = off; off = align_up(off + (size_t)g.B * g.H * g.n_state_segs * state_bytes, 1024);
   g.off_mt = off; off = align_up(off + (size_t)g.B * g.Nc * g.H * 2 * g.mt_rows * g.Dp * 2, 1024);
+  g.off_done = off; off = align_up(off + (size_t)g.B * g.H * 4, 1024);  // scan units done per (batch, head)
   g.fp8 = cfg->softmax_precision == VDN_PREC_FP8;
   if (g.fp8) {
     g.pitch_v8 = (long long)align_up((size_t)g.N, 16);
@@ -266,6 +267,11 @@ unsigned long long* scan_counter_ptr(const vdn_cfg* cfg, const Geom& g) {
   return reinterpret_cast<unsigned long long*>(ws(cfg, g.off_status) + 128);
 }
 
+// Scan units completed per (batch, head), counted by the softmax kernel's
+// scan and zeroed by the state build (the fused readout waits for its
+// (batch, head) to be complete before it reads M_c).
+unsigned* scan_done_ptr(const vdn_cfg* cfg, const Geom& g) { return reinterpret_cast<unsigned*>(ws(cfg, g.off_done)); }
+
 // Flag at byte 136 of the status slot, written by the softmax kernel: 1 when
 // o_s in the workspace holds sigmoid(g_s) * o_s.
 int* os_gated_ptr(const vdn_cfg* cfg, const Geom& g) { return reinterpret_cast<int*>(ws(cfg, g.off_status) + 136); }
@@ -286,6 +292,7 @@ vdn_status step_state_build(const vdn_cfg* cfg, const Geom& g, const Srcs& s, cu
   p.record = record_ptr(cfg, g);
   p.inject_timeout = (cfg->debug_flags & VDN_INJECT_TIMEOUT) != 0;
   p.scan_counter = scan_counter_ptr(cfg, g);
+  p.scan_done = scan_done_ptr(cfg, g);
   return cuda_status(launch_state_build(m, p, st));
 }
 
@@ -337,7 +344,8 @@ void plan_items(const Geom& g, K3Params& p) {
 // The softmax branch; with do_scan, the kernel also runs the forward/backward
 // scan of the state partials in the workspace; with gate_s (bf16 tensors whose
 // head_dim needs no padding, not under VDN_OUT_SOFTMAX_ONLY), o_s is written
-// as sigmoid(gate_s) * o_s.
+// as sigmoid(gate_s) * o_s.  With out (the fused readout): the kernel writes
+// the merged output itself, from gate_s, gate_l and the readout operands.
 vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s, cudaStream_t st, bool do_scan,
                                const void* gate_s, const void* gate_l = nullptr, void* out = nullptr) {
   NvtxRange nvtx("vdn:sparse_softmax");
@@ -389,6 +397,7 @@ vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s,
     p.gate_l = static_cast<const __nv_bfloat16*>(gate_l);
     p.mt = ws(cfg, g.off_mt);
     p.gamma = cfg->rms_weight;
+    p.scan_done = do_scan ? scan_done_ptr(cfg, g) : nullptr;
   }
   if (do_scan) make_scan_args(cfg, g, p.scan);
   int dev = 0, sms = 148;
@@ -628,8 +637,9 @@ vdn_status vdn_sparse_softmax_merge(const void* q, const void* k, const void* v,
   if (!fused_readout_supported(cfg)) return VDN_ERR_UNSUPPORTED;
   s = check_inputs(cfg, g, {q, k, v, gate_s, gate_l, out}, {text_k, text_v});
   if (s != VDN_OK) return s;
+  if ((cfg->debug_flags & VDN_EXPORT_STATES) && (!cfg->export_fwd || !cfg->export_bwd)) return VDN_ERR_INVALID_ARG;
   return step_sparse_softmax(cfg, g, kernel_srcs(cfg, g, q, k, v, text_k, text_v), static_cast<cudaStream_t>(stream),
-                             false, gate_s, gate_l, out);
+                             true, gate_s, gate_l, out);
 }
 
 vdn_status vdn_hybrid_attn_fwd(const void* q, const void* k, const void* v, const void* text_k, const void* text_v,
@@ -646,10 +656,8 @@ vdn_status vdn_hybrid_attn_fwd(const void* q, const void* k, const void* v, cons
   if (poison_ws(cfg, g, st) != cudaSuccess) return VDN_ERR_CUDA;
   if ((s = step_stage(cfg, g, q, k, v, text_k, text_v, st)) != VDN_OK) return s;
   if ((s = step_state_build(cfg, g, src, st)) != VDN_OK) return s;
-  if (cfg->readout_mode == VDN_READOUT_FUSED) {
-    if ((s = step_state_scan(cfg, g, st)) != VDN_OK) return s;
-    return step_sparse_softmax(cfg, g, src, st, false, gate_s, gate_l, out);
-  }
+  if (cfg->readout_mode == VDN_READOUT_FUSED)  // the scan runs inside as well
+    return step_sparse_softmax(cfg, g, src, st, true, gate_s, gate_l, out);
   if ((s = step_sparse_softmax(cfg, g, src, st, true, gate_s)) != VDN_OK) return s;  // the scan runs inside
   return step_readout_merge(cfg, g, src, gate_s, gate_l, out, st);
 }
@@ -724,10 +732,9 @@ vdn_status vdn_hybrid_attn_fwd_host(const void* q, const void* k, const void* v,
   }
   if ((s = step_state_build(&c, g, src, st)) != VDN_OK) return finish(s);
   if (c.readout_mode == VDN_READOUT_FUSED) {
-    // the scan while q and the gates land; the fused softmax kernel needs all three
-    if ((s = step_state_scan(&c, g, st)) != VDN_OK) return finish(s);
+    // the fused softmax kernel (which runs the scan as well) reads q and both gates
     if (cudaStreamWaitEvent(st, ev[3], 0) != cudaSuccess) return finish(VDN_ERR_CUDA);
-    if ((s = step_sparse_softmax(&c, g, src, st, false, dv + h.gs, dv + h.gl, dv + h.out)) != VDN_OK)
+    if ((s = step_sparse_softmax(&c, g, src, st, true, dv + h.gs, dv + h.gl, dv + h.out)) != VDN_OK)
       return finish(s);
   } else {
     // the softmax branch runs while the gates are still in flight, so here it

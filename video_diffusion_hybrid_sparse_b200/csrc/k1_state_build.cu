@@ -113,6 +113,8 @@ __global__ void __launch_bounds__(kK1Threads, 1)
   const uint32_t warp = warp_id(), lane = lane_id();
 
   if (threadIdx.x == 0 && blockIdx.x == 0 && p.scan_counter) *p.scan_counter = 0ull;
+  if (blockIdx.x == 0 && p.scan_done)
+    for (int i = threadIdx.x; i < p.g.B * p.g.H; i += blockDim.x) p.scan_done[i] = 0u;
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&bars[kFull + s], 1);

@@ -50,8 +50,10 @@
 // the gated merge run in this kernel's item epilogue instead of a readout
 // kernel of their own (the frame-7 paragraph of 双分支混合注意力机制 combines
 // the linear read with the local branch at the query's position), so o_s is
-// never written and q is read once.  The forward/backward scan has then run
-// before this kernel (its readout operands M_c must be complete).  Per item:
+// never written and q is read once.  The forward/backward scan runs in warps
+// 2-3 as on the other path and counts its completed units per (batch, head);
+// an item's readout waits (bounded) until its (batch, head) is complete, which
+// it is long before the first item ends.  Per item:
 //  * the producer sends M_c of the item's (batch, chunk, head) through the
 //    K/V ring as one more stage, the hi image in the K slot and the lo image
 //    in the V slot (rows 0..127 of each: the numerator columns);
@@ -141,7 +143,14 @@ __device__ __forceinline__ void scan_dynamic(const K3Params& p, uint32_t lane) {
     if (lane == 0) base = (long long)atomicAdd(p.scan_counter, 32ull);
     base = __shfl_sync(0xffffffffu, base, 0);
     if (base >= units) break;
-    if (base + lane < units) scan_unit(p.scan, base + lane);
+    if (base + lane < units) {
+      scan_unit(p.scan, base + lane);
+      if (p.scan_done) {
+        // release: this unit's M_c writes before the count that says so
+        __threadfence();
+        atomicAdd(p.scan_done + (base + lane) / scan_units_per_bh(p.g), 1u);
+      }
+    }
   }
 }
 
@@ -163,6 +172,9 @@ __device__ __forceinline__ bool fused_readout_tile(const K3Params& p, int item, 
   const size_t row_el = (((size_t)it.b * g.N + (size_t)(it.row0 + t * kBlockM + row)) * g.H + it.h) * D;
   const uint4* gsp = reinterpret_cast<const uint4*>(p.gate_s + row_el);
   const uint4* glp = reinterpret_cast<const uint4*>(p.gate_l + row_el);
+  // z of M_c (read below) comes from this kernel's own scan under do_scan
+  const bool z_ready = !p.do_scan || counter_wait(p.scan_done + it.b * g.H + it.h, (unsigned)scan_units_per_bh(g), ab);
+  if (__any_sync(0xffffffffu, !z_ready)) return false;
   // phi(q) in place over this thread's row of Q_t (K-major, 128-byte
   // swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)) and
   // den = phi(q) . (z_hi + z_lo), with the bf16 phi(q) the MMA reads
@@ -178,7 +190,7 @@ __device__ __forceinline__ bool fused_readout_tile(const K3Params& p, int item, 
       const uint4 w = *pq;
       const uint4 f = make_uint4(phi_bf16x2(w.x), phi_bf16x2(w.y), phi_bf16x2(w.z), phi_bf16x2(w.w));
       *pq = f;
-      const uint4 a = __ldg(zh + ch), b = __ldg(zl + ch);
+      const uint4 a = __ldcg(zh + ch), b = __ldcg(zl + ch);  // written in this kernel under do_scan: not __ldg
       const uint32_t fw[4] = {f.x, f.y, f.z, f.w}, aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e)
@@ -382,6 +394,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int mc = it.c == kAllFrames ? 0 : it.c;
           const uint8_t* img = p.mt + (((size_t)it.b * g.Nc + mc) * g.H + it.h) * (size_t)kMtImage * 2;
           ++kv_cnt;
+          if (p.do_scan) {
+            // M_c of this (batch, head) comes from the kernel's own scan
+            if (!counter_wait(p.scan_done + it.b * g.H + it.h, (unsigned)scan_units_per_bh(g), ab)) {
+              ok = false;
+              break;
+            }
+            fence_proxy_async_global();
+          }
           if (!mbar_wait(&bars[kKEmpty + st], ph ^ 1, ab)) { ok = false; break; }
           mbar_expect_tx(&bars[kKFull + st], L::kTile);
           for (int bx = 0; bx < 2; ++bx)
@@ -747,8 +767,10 @@ static cudaError_t launch_k3(const Maps& m, const K3Params& p, int grid, cudaStr
 
 cudaError_t launch_sparse_softmax(const Maps& m, const K3Params& p, int grid, cudaStream_t st) {
   if (p.out) {
-    // fused readout: bf16, head_dim 128, scan already run, gates and out given
-    if (p.g.Dp != 128 || p.g.d != 128 || p.do_scan || !p.gate_s || !p.gate_l || !p.mt) return cudaErrorInvalidValue;
+    // fused readout: bf16, head_dim 128, gates and out given; its own scan
+    // needs the per-(batch, head) counters
+    if (p.g.Dp != 128 || p.g.d != 128 || !p.gate_s || !p.gate_l || !p.mt || (p.do_scan && !p.scan_done))
+      return cudaErrorInvalidValue;
     return launch_k3<128, true>(m, p, grid, st);
   }
   return p.g.Dp == 128 ? launch_k3<128, false>(m, p, grid, st) : launch_k3<64, false>(m, p, grid, st);

@@ -44,12 +44,16 @@ struct K3Params {
   int do_scan;             // the kernel also runs the forward/backward scan (scan below)
   unsigned long long* scan_counter;  // next scan unit to take (workspace; zeroed by the state build)
   ScanArgs scan;
-  // Fused readout (out != null; bf16, head_dim 128, do_scan 0): the kernel
-  // writes the merged output itself from M_c, which the scan has written.
+  // Fused readout (out != null; bf16, head_dim 128): the kernel writes the
+  // merged output itself from M_c.  With do_scan, M_c comes from this
+  // kernel's own scan: the scan counts the units it completed per (batch,
+  // head) in scan_done, and an item reads M_c of its (batch, head) once all
+  // of them are in; without, the scan ran before the kernel.
   __nv_bfloat16* out;      // [B, N, H, 128] bf16
   const __nv_bfloat16* gate_l;  // [B, N, H, 128]
   const uint8_t* mt;       // readout operand images per (b, chunk, head) (scan.cuh)
   const float* gamma;      // [H, 128] fp32 or null (ones)
+  unsigned* scan_done;     // [B * H] (workspace; zeroed by the state build)
 };
 
 struct K1Params {
@@ -60,6 +64,7 @@ struct K1Params {
   int* record;             // timeout record (workspace), may be null
   int inject_timeout;      // test only: CTA 0 waits for a phase nothing completes (short limit)
   unsigned long long* scan_counter;  // zeroed by CTA 0 for the scan of the softmax kernel that follows
+  unsigned* scan_done;     // [B * H] zeroed by CTA 0 likewise
 };
 
 struct K4Params {

@@ -48,7 +48,7 @@ struct Geom {
   float scale;              // softmax scale
   float eps;                // RMSNorm epsilon
   // workspace layout (byte offsets; each 1024-aligned)
-  size_t off_status, off_os, off_q, off_k, off_v, off_tk, off_tv, off_parts, off_segst, off_mt, total;
+  size_t off_status, off_os, off_q, off_k, off_v, off_tk, off_tv, off_parts, off_segst, off_mt, off_done, total;
   int fp8;                  // softmax branch with e4m3 operands
   long long pitch_v8, pitch_t8;  // row pitches (bytes) of the transposed e4m3 v and text_v
   size_t off_q8, off_k8, off_vt8, off_tk8, off_tvt8, off_amax;

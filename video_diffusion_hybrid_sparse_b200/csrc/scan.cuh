@@ -47,6 +47,9 @@ __host__ __device__ __forceinline__ long long scan_units(const Geom& g) {
   return (long long)g.B * g.H * (g.Dp + 1) * (g.Dp / 4);
 }
 
+// Units of one (batch, head): unit u belongs to (batch, head) u / this.
+__host__ __device__ __forceinline__ int scan_units_per_bh(const Geom& g) { return (g.Dp + 1) * (g.Dp / 4); }
+
 __device__ __forceinline__ void scan_unit(const ScanArgs& sa, long long unit) {
   const Geom& g = sa.g;
   const StatePlan& sp = sa.sp;

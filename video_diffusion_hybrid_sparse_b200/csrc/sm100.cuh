@@ -308,6 +308,33 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// Bounded wait until the gpu-scope counter *counter has reached `target`
+// (an acquire load, so that what the counting threads wrote before their
+// release is visible after it); false, with the timeout recorded (barrier
+// offset 0, parity 2: a counter wait), after kWaitNs of global time or when
+// the CTA gave up.
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ bool counter_wait(const unsigned* counter, unsigned target, const CtaAbort& ab) {
+  if (ld_acquire_u32(counter) >= target) return true;
+  const long long g0 = global_ns();
+  while (true) {
+    __nanosleep(256);
+    if (ld_acquire_u32(counter) >= target) return true;
+    if (aborted(ab)) return false;
+    const long long g1 = global_ns();
+    if (g1 - g0 > kWaitNs) {
+      record_timeout(ab, ab.flag, 2u, g1 - g0);
+      raise_abort(ab);
+      return false;
+    }
+  }
+}
+
 // Short bounded wait (kWaitNs / 4) used only while draining on the abort path.
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   const long long t0 = global_ns();
@@ -353,6 +380,13 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 // (TMA, tensor core operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Global memory written through the generic proxy (plain stores, made visible
+// by a release/acquire pair) and then read through the async proxy (a bulk
+// copy): the reading thread fences between its acquire and the copy.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05: TMEM
