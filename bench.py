@@ -77,12 +77,12 @@ def work(w, fp8: bool = False, fused: bool = False):
     gated = w.dtype == "bf16" and w.d in (64, 128) and not fp8
     k4 = (4 if gated else 5) * w.B * w.N * w.H * w.d * e + n_chunks * state
     k3_bytes = ((3 + (1 if gated else 0)) * w.B * w.N + 2 * w.B * w.T) * w.H * w.d * e + w.B * w.N * w.H * w.d * 2
-    # fused: q, k, v, text, g_s and g_l read, M_c read once per item pair of
-    # tiles (counted once per (batch, chunk, head)), out written
-    k3f_bytes = ((5 * w.B * w.N + 2 * w.B * w.T) * w.H * w.d + w.B * w.N * w.H * w.d) * e + n_chunks * state
+    # fused: q, k, v, text, g_s and g_l read, M_c read once per (batch,
+    # chunk, head), out written, and the scan that runs inside
+    k3f_bytes = ((5 * w.B * w.N + 2 * w.B * w.T) * w.H * w.d + w.B * w.N * w.H * w.d) * e + n_chunks * state + k2
     if fused:
         return dict(softmax_flops=softmax_flops, linear_flops=linear_flops, k1_bytes=k1, k2_bytes=k2, k4_bytes=0,
-                    k3_bytes=k3f_bytes, linear_bytes=k1 + k2 + (k3f_bytes - k3_bytes))
+                    k3_bytes=k3f_bytes, linear_bytes=k1 + (k3f_bytes - k3_bytes))
     return dict(softmax_flops=softmax_flops, linear_flops=linear_flops, k1_bytes=k1, k2_bytes=k2, k4_bytes=k4,
                 k3_bytes=k3_bytes, linear_bytes=k1 + k2 + k4)
 
@@ -514,6 +514,12 @@ def run_ours(args, w, world, rank, local):
     stagings = [vb.new_staging(steps.s, dev["q"].device) for _ in range(2)]
     wss = [steps.ws, vb.new_workspace(steps.s, dev["q"].device, prec)]
     host_outs = [host_out, torch.empty(out.shape, dtype=out.dtype, pin_memory=True)]
+    # one untimed host call first: its kernels (the separate readout's, which
+    # the fused device-resident timing above did not launch) are loaded then
+    vb.hybrid_attn_fwd_host(host["q"], host["k"], host["v"], host["text_k"], host["text_v"], host["gate_s"],
+                            host["gate_l"], frames=w.F, chunk_frames=w.C, out=host_outs[0], workspace=wss[0],
+                            staging=stagings[0], stream=streams[0], softmax_precision=prec,
+                            readout_mode=vb.READOUT_SEPARATE)
     barrier(world)
     torch.cuda.synchronize()
     e0.record(stream)

@@ -39,13 +39,14 @@ def test_768p_work_figures():
 
 def test_fused_work_figures():
     """With the readout fused into the softmax kernel there is no readout
-    kernel: the softmax kernel reads q, k, v, text, both gates and M_c and
-    writes out (five video tensors read, one written)."""
+    kernel: the softmax kernel reads q, k, v, text, both gates and M_c,
+    writes out (five video tensors read, one written) and runs the scan."""
     w = BY_NAME["768p_bf16"]
     sep, fus = bench.work(w), bench.work(w, fused=True)
     assert fus["k4_bytes"] == 0 and fus["softmax_flops"] == sep["softmax_flops"]
     video = w.N * w.H * w.d * 2
-    assert fus["k3_bytes"] == 6 * video + 2 * w.T * w.H * w.d * 2 + 15 * w.H * w.d * (w.d + 1) * 4
+    assert fus["k3_bytes"] == (6 * video + 2 * w.T * w.H * w.d * 2 + 15 * w.H * w.d * (w.d + 1) * 4
+                               + sep["k2_bytes"])
 
 
 @pytest.mark.parametrize("name", sorted({n for n, _ in bench.KERNELS + bench.KERNELS_FUSED} - {"stage"}
