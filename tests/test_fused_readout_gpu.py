@@ -129,7 +129,8 @@ def test_fused_exported_states_equal_separate():
     assert torch.equal(ex[0], ex[2]) and torch.equal(ex[1], ex[3])
 
 
-@pytest.mark.parametrize("name,heads", [("768p_bf16", [0, 9, 23]), ("chunk5_bf16", [0, 15])])
+@pytest.mark.parametrize("name,heads", [("768p_bf16", [0, 9, 23]), ("chunk5_bf16", [0, 15]),
+                                        ("768p_long_bf16", [0, 23])])
 def test_fused_workload_sampled_rows(name, heads):
     w = BY_NAME[name]
     inputs = make_inputs(w)
