@@ -504,8 +504,7 @@ def run_ours(args, w, world, rank, local):
     n_e2e = max(4, args.steps // 4)
     # The host calls use the separate readout whatever --readout says: there
     # the softmax kernel runs while the gates are still being copied in,
-    # which the fused kernel (it reads the gates) cannot (36.9 against 35.4
-    # ms per call at 768p).  Two calls in flight, as a server streaming
+    # which the fused kernel (it reads the gates) cannot.  Two calls in flight, as a server streaming
     # requests would run them: call i on stream i % 2 with its own staging
     # buffer, workspace and host output, so the copy-out of one call overlaps
     # the copy-in of the next (the two PCIe directions); the library's copy
@@ -514,8 +513,8 @@ def run_ours(args, w, world, rank, local):
     stagings = [vb.new_staging(steps.s, dev["q"].device) for _ in range(2)]
     wss = [steps.ws, vb.new_workspace(steps.s, dev["q"].device, prec)]
     host_outs = [host_out, torch.empty(out.shape, dtype=out.dtype, pin_memory=True)]
-    # one untimed host call first: its kernels (the separate readout's, which
-    # the fused device-resident timing above did not launch) are loaded then
+    # one untimed host call first (under --readout fused, the separate
+    # readout's kernels are loaded then)
     vb.hybrid_attn_fwd_host(host["q"], host["k"], host["v"], host["text_k"], host["text_v"], host["gate_s"],
                             host["gate_l"], frames=w.F, chunk_frames=w.C, out=host_outs[0], workspace=wss[0],
                             staging=stagings[0], stream=streams[0], softmax_precision=prec,
@@ -558,9 +557,9 @@ def main():
     ap.add_argument("--workload", default="768p_bf16", choices=sorted(BY_NAME))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--readout", default="fused", choices=["fused", "separate"],
-                    help="readout and merge in the softmax kernel's epilogue (bf16, head_dim 128; the faster "
-                         "path, falls back to separate elsewhere), or in a kernel of their own")
+    ap.add_argument("--readout", default="separate", choices=["separate", "fused"],
+                    help="readout and merge in a kernel of their own, or in the softmax kernel's epilogue "
+                         "(bf16, head_dim 128; separate elsewhere)")
     ap.add_argument("--precision", default="bf16", choices=["bf16", "fp8"],
                     help="operand precision of the softmax branch (bf16 is the headline)")
     args = ap.parse_args()
