@@ -8,7 +8,9 @@
 //    one (batch, head, query segment), a segment being the rows of one chunk
 //    (under the GLOBAL anchor reading the rows of frames 0 and F-1 are
 //    segments of their own whose key set is every frame); items are handed
-//    out statically, (batch, head)-major (k3_common.cuh says why);
+//    out statically in blocks ordered (batch, head, segment, pair), so the
+//    CTAs running at once share one head's keys and values in L2
+//    (plan_items in api.cu chooses the blocks);
 //  * only the KV tiles of the item's key set are enumerated: at most three
 //    merged video token ranges plus the text range, 128 keys per tile; the
 //    last tile of a range is masked past the range end;
