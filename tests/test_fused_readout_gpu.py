@@ -34,6 +34,11 @@ CASES = [
     Workload("many_items", 1, 15, 300, 16, 128, 64, 1, "bf16", "rms", 31),
     # one frame: both anchors are frame 0
     Workload("one_frame_d128", 1, 1, 150, 2, 128, 20, 1, "bf16", "normal", 32),
+    # the most chunks the scan keeps on chip (96): 96 readout operands per
+    # head, every item a single tile with 4 valid rows
+    Workload("max_chunks_d128", 1, 96, 4, 1, 128, 3, 1, "bf16", "normal", 33),
+    # one token per frame, one text token
+    Workload("tiny_tokens_d128", 1, 7, 1, 2, 128, 1, 1, "bf16", "normal", 34),
 ]
 
 
