@@ -386,14 +386,19 @@ def k3_roles(items, stages=2, halves=2, fused=False):
     fused readout also num), O0/O1.  fused: the readout operand M_c travels
     as one more K/V stage, the softmax warps write phi(Q_t) over Q_t, the MMA
     thread writes num_t over S_t's columns, the epilogue reads it and
-    releases the columns (RDone)."""
+    releases the columns (RDone); the scan (warps 2-3) writes M_c in global
+    memory (Mg) and completes its count (ScanDone, a counter in the kernel,
+    a barrier of one arrival here), which the producer waits for before it
+    copies M_c and the softmax warps before they read z."""
     loads, kv = [], 0
     for n_item, (nt, nkv) in enumerate(items):
         if n_item > 0:
             loads.append(wait("QEmpty", n_item - 1))
         loads.append(tma("QFull", *[(f"Q{t}", ("Q", n_item)) for t in range(nt)]))
-        for _ in range(nkv + (1 if fused else 0)):
+        for i in range(nkv + (1 if fused else 0)):
             st, r = kv % stages, kv // stages
+            if i == nkv:  # the readout stage: M_c copied from global memory
+                loads += [wait("ScanDone", 0), beg(reads=[("Mg", "scanned")]), end("Mg")]
             loads += [wait(f"KEmpty{st}", r - 1), tma(f"KFull{st}", (f"K{st}", kv)), wait(f"VEmpty{st}", r - 1),
                       tma(f"VFull{st}", (f"V{st}", kv))]
             kv += 1
@@ -459,6 +464,8 @@ def k3_roles(items, stages=2, halves=2, fused=False):
     mma_ += [commit("Done"), wait("Done", 0)]
 
     roles = {"loads": loads, "mma": mma_}
+    if fused:
+        roles["scan"] = [beg(writes=[("Mg", "scanned")]), end("Mg"), arrive("ScanDone")]
     for t in range(2):
         sm, s_cnt, o_cnt = [], 0, 0
         for n_item, (nt, nkv) in enumerate(items):
@@ -475,7 +482,8 @@ def k3_roles(items, stages=2, halves=2, fused=False):
                     sm += [beg(writes=[(f"SPb{t}", ("P", s_cnt))]), end(f"SPb{t}"), arrive(f"PFull2{t}")]
                 s_cnt += 1
             if fused:
-                sm += [beg(writes=[(f"Q{t}", ("phi", n_item))]), end(f"Q{t}"), arrive(f"PhiFull{t}"),
+                sm += [wait("ScanDone", 0), beg(reads=[("Mg", "scanned")]), end("Mg"),  # z
+                       beg(writes=[(f"Q{t}", ("phi", n_item))]), end(f"Q{t}"), arrive(f"PhiFull{t}"),
                        wait(f"OFull{t}", o_cnt), wait(f"RFull{t}", o_cnt),
                        beg(reads=[(f"O{t}", ("O", n_item, nkv - 1))] + [(f"SP{h}{t}", ("num", n_item))
                                                                         for h in regions]),
@@ -683,6 +691,12 @@ PLANTED = {
     # fused readout: the epilogue reads num before the readout MMAs completed
     "fused_epilogue_skips_num": lambda: _drop(k3_roles([(1, 2)], fused=True), "softmax0",
                                               lambda op: op.kind == "wait" and op.bar == "RFull0"),
+    # fused readout: the producer copies M_c before the scan has completed it
+    "fused_loader_skips_scan_count": lambda: _drop(k3_roles([(1, 1), (1, 1)], fused=True), "loads",
+                                                   lambda op: op.kind == "wait" and op.bar == "ScanDone"),
+    # fused readout: the softmax warps read z before the scan has completed it
+    "fused_epilogue_skips_scan_count": lambda: _drop(k3_roles([(1, 1)], fused=True), "softmax0",
+                                                     lambda op: op.kind == "wait" and op.bar == "ScanDone"),
     # fused readout: the softmax warps write phi over Q before the item's last S landed
     "fused_phi_before_last_s": lambda: _move_before(
         k3_roles([(1, 2)], fused=True), "softmax0", lambda op: op.kind == "beg" and op.writes
