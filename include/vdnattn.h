@@ -130,10 +130,15 @@ enum {
                                sleeps 50 microseconds whenever it moves to another readout operand
                                (batch, chunk, head), letting the other warps run as far ahead as the
                                protocol allows.  Outputs are unchanged. */
-  VDN_POISON_WS = 64          /* vdn_hybrid_attn_fwd, _host and _static first fill the workspace past its
+  VDN_POISON_WS = 64,         /* vdn_hybrid_attn_fwd, _host and _static first fill the workspace past its
                                256-byte status slot with 0xFF bytes (NaN in bf16 and fp32), so that a
                                read of scratch the call has not written would show in the output.
                                Outputs are unchanged. */
+  VDN_INJECT_TIMEOUT_SCAN = 128 /* test of the failure path only: under VDN_READOUT_FUSED, the producer of
+                               CTA 0 of the softmax kernel waits, with a 10-ms limit, for one scan unit
+                               more than its (batch, head) has; it gives up, the CTA's other warps
+                               follow, the kernel writes VDN_ERR_TIMEOUT to status_word and returns.
+                               The call's outputs are then undefined; the context stays usable. */
 };
 
 typedef struct {

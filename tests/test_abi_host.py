@@ -72,9 +72,9 @@ def test_validate_rejects_unknown_dtype_and_flags():
     cfg = vb.make_cfg(shape())
     cfg.dtype = 7
     assert lib.vdn_validate(ctypes.byref(cfg)) == 2
-    cfg = vb.make_cfg(shape(), debug_flags=128)
+    cfg = vb.make_cfg(shape(), debug_flags=256)
     assert lib.vdn_validate(ctypes.byref(cfg)) == 1
-    for flag in (vb.INJECT_TIMEOUT, vb.STALL_READOUT_MMA, vb.POISON_WS):
+    for flag in (vb.INJECT_TIMEOUT, vb.STALL_READOUT_MMA, vb.POISON_WS, vb.INJECT_TIMEOUT_SCAN):
         cfg = vb.make_cfg(shape(), debug_flags=flag)
         assert lib.vdn_validate(ctypes.byref(cfg)) == 0
     cfg = vb.make_cfg(shape())
@@ -140,6 +140,10 @@ def test_readout_mode_validation():
     unsupported.append(split)
     for cfg in unsupported:
         assert lib.vdn_validate(ctypes.byref(cfg)) == 2
+    # the injected wait of the fused readout's scan count is a known debug flag
+    assert lib.vdn_validate(ctypes.byref(vb.make_cfg(ok, readout_mode=vb.READOUT_FUSED,
+                                                      debug_flags=vb.INJECT_TIMEOUT_SCAN))) == 0
+    assert lib.vdn_validate(ctypes.byref(vb.make_cfg(ok, debug_flags=256))) == 1
     # the fused step itself checks the requirements whatever the mode says
     cfg = vb.make_cfg(vb.Shape(1, 15, 256, 2, 64, 64, 1))
     assert lib.vdn_sparse_softmax_merge(*([None] * 8), ctypes.byref(cfg), None) == 2

@@ -166,3 +166,32 @@ def test_fused_rejects_unsupported_configurations():
     dev = to_dev(make_inputs(w))
     with pytest.raises(vb.VdnError, match="unsupported"):
         fused(w, dev)
+
+
+def test_injected_scan_count_timeout_reports_status_and_context_survives():
+    """The fused readout's wait for the in-kernel scan's count
+    (VDN_INJECT_TIMEOUT_SCAN: CTA 0's producer asks for one unit more than its
+    (batch, head) has, 10-ms limit) ends with VDN_ERR_TIMEOUT in the status
+    word instead of a hang or a fault; the timeout record names that wait
+    (softmax kernel, block 0, warp 0, barrier offset 0 and parity 2: a counter
+    wait), and the next call is correct."""
+    import time
+    w = CASES[4]
+    inputs = make_inputs(w)
+    dev = to_dev(inputs)
+    ws = vb.workspace_for(vb.shape_of(dev["q"], dev["text_k"], w.F, w.C), dev["q"].device)
+    vb.clear_timeout_record(ws)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.time()
+    fused(w, dev, debug_flags=vb.INJECT_TIMEOUT_SCAN, status=status, workspace=ws)
+    assert time.time() - t0 < 30
+    assert int(status.item()) == 6
+    rec = vb.timeout_record(ws)
+    assert rec["timeouts"] >= 1 and rec["kernel"] == 3 and rec["block"] == 0 and rec["warp"] == 0, rec
+    assert rec["bar_off"] == 0 and rec["parity"] == 2, rec
+    assert 10_000_000 <= rec["ns"] < 1_000_000_000, rec
+    vb.clear_timeout_record(ws)
+    status.zero_()
+    out = fused(w, dev, status=status, workspace=ws)
+    assert int(status.item()) == 0
+    assert_close(out.float().cpu().numpy(), oracle_full(w, inputs)["out"], f"{w.name} after the injected timeout")

@@ -19,7 +19,7 @@ _lib = None
 
 VDN_BF16, VDN_FP32 = 0, 1
 OUT_SOFTMAX_ONLY, OUT_LINEAR_ONLY, OUT_LINEAR_RAW, EXPORT_STATES, INJECT_TIMEOUT = 1, 2, 4, 8, 16
-STALL_READOUT_MMA, POISON_WS = 32, 64
+STALL_READOUT_MMA, POISON_WS, INJECT_TIMEOUT_SCAN = 32, 64, 128
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "pointer not aligned",
           4: "workspace missing or too small", 5: "CUDA error", 6: "device wait timed out"}
 

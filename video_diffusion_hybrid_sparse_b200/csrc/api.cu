@@ -63,6 +63,7 @@ vdn_status make_geom(const vdn_cfg* cfg, Geom& g) {
   if (cfg->dtype != VDN_BF16 && cfg->dtype != VDN_FP32) return VDN_ERR_UNSUPPORTED;
   if (cfg->debug_flags &
       ~(VDN_OUT_SOFTMAX_ONLY | VDN_OUT_LINEAR_ONLY | VDN_OUT_LINEAR_RAW | VDN_EXPORT_STATES | VDN_INJECT_TIMEOUT |
+        VDN_INJECT_TIMEOUT_SCAN |
         VDN_STALL_READOUT_MMA | VDN_POISON_WS))
     return VDN_ERR_INVALID_ARG;
   const int Nc = cfg->frames / cfg->chunk_frames;
@@ -398,6 +399,7 @@ vdn_status step_sparse_softmax(const vdn_cfg* cfg, const Geom& g, const Srcs& s,
     p.mt = ws(cfg, g.off_mt);
     p.gamma = cfg->rms_weight;
     p.scan_done = do_scan ? scan_done_ptr(cfg, g) : nullptr;
+    p.inject_scan_wait = do_scan && (cfg->debug_flags & VDN_INJECT_TIMEOUT_SCAN) ? 1 : 0;
   }
   if (do_scan) make_scan_args(cfg, g, p.scan);
   int dev = 0, sms = 148;

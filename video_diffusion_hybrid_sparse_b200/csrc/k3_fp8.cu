@@ -114,11 +114,12 @@ __global__ void __launch_bounds__(384, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t kv_cnt = 0, item_cnt = 0;
+      uint32_t kv_cnt = 0, item_cnt = 0, q_loads = 0;  // q_loads: Q loads issued (the last is drained on an abort)
       bool ok = true;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++item_cnt) {
         const Item it = decode_item(item, p);
         if (item_cnt > 0 && !mbar_wait(&bars[kQEmpty], (item_cnt - 1) & 1, ab)) { ok = false; break; }
+        ++q_loads;
         mbar_expect_tx(&bars[kQFull], it.ntiles * L::kTile);
         for (int t = 0; t < it.ntiles; ++t)
           tma_load_2d(sQ + t * L::kTile, &tm_q, &bars[kQFull], it.h * D, it.b * (int)g.N + it.row0 + t * kBlockM);
@@ -150,7 +151,7 @@ __global__ void __launch_bounds__(384, 1)
           mbar_drain(&bars[kKFull + i % L::kStages], (i / L::kStages) & 1);
           mbar_drain(&bars[kVFull + i % L::kStages], (i / L::kStages) & 1);
         }
-        if (item_cnt > 0) mbar_drain(&bars[kQFull], (item_cnt - 1) & 1);
+        if (q_loads > 0) mbar_drain(&bars[kQFull], (q_loads - 1) & 1);
       }
     }
   } else if (warp == 1) {

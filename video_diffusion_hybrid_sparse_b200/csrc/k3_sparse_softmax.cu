@@ -355,11 +355,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && blockIdx.x == 0 && p.os_gated) *p.os_gated = p.gate_s != nullptr;  // for the readout
     if (lane == 0) {
-      uint32_t kv_cnt = 0, item_cnt = 0;
+      uint32_t kv_cnt = 0, item_cnt = 0, q_loads = 0;  // q_loads: Q loads issued (the last is drained on an abort)
       bool ok = true;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++item_cnt) {
         const Item it = decode_item(item, p);
         if (item_cnt > 0 && !mbar_wait(&bars[kQEmpty], (item_cnt - 1) & 1, ab)) { ok = false; break; }
+        ++q_loads;
         mbar_expect_tx(&bars[kQFull], it.ntiles * L::kTile);
         for (int t = 0; t < it.ntiles; ++t)
           for (int bx = 0; bx < D / 64; ++bx)
@@ -397,8 +398,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint8_t* img = p.mt + (((size_t)it.b * g.Nc + mc) * g.H + it.h) * (size_t)kMtImage * 2;
           ++kv_cnt;
           if (p.do_scan) {
-            // M_c of this (batch, head) comes from the kernel's own scan
-            if (!counter_wait(p.scan_done + it.b * g.H + it.h, (unsigned)scan_units_per_bh(g), ab)) {
+            // M_c of this (batch, head) comes from the kernel's own scan (a
+            // test of the failure path asks CTA 0 for one unit more, 10 ms)
+            const bool inject = p.inject_scan_wait && blockIdx.x == 0;
+            if (!counter_wait(p.scan_done + it.b * g.H + it.h, (unsigned)scan_units_per_bh(g) + (inject ? 1u : 0u),
+                              ab, inject ? 10000000ll : kWaitNs)) {
               ok = false;
               break;
             }
@@ -420,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_drain(&bars[kKFull + i % L::kStages], (i / L::kStages) & 1);
           mbar_drain(&bars[kVFull + i % L::kStages], (i / L::kStages) & 1);
         }
-        if (item_cnt > 0) mbar_drain(&bars[kQFull], (item_cnt - 1) & 1);
+        if (q_loads > 0) mbar_drain(&bars[kQFull], (q_loads - 1) & 1);
       }
     }
   } else if (warp == 1) {

@@ -54,6 +54,7 @@ struct K3Params {
   const uint8_t* mt;       // readout operand images per (b, chunk, head) (scan.cuh)
   const float* gamma;      // [H, 128] fp32 or null (ones)
   unsigned* scan_done;     // [B * H] (workspace; zeroed by the state build)
+  int inject_scan_wait;    // test only: CTA 0's producer waits for one unit more (short limit)
 };
 
 struct K1Params {

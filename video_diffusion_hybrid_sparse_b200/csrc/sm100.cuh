@@ -311,7 +311,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
 // Bounded wait until the gpu-scope counter *counter has reached `target`
 // (an acquire load, so that what the counting threads wrote before their
 // release is visible after it); false, with the timeout recorded (barrier
-// offset 0, parity 2: a counter wait), after kWaitNs of global time or when
+// offset 0, parity 2: a counter wait), after limit_ns of global time or when
 // the CTA gave up.
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
   unsigned v;
@@ -319,7 +319,8 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
   return v;
 }
 
-__device__ __forceinline__ bool counter_wait(const unsigned* counter, unsigned target, const CtaAbort& ab) {
+__device__ __forceinline__ bool counter_wait(const unsigned* counter, unsigned target, const CtaAbort& ab,
+                                             long long limit_ns = kWaitNs) {
   if (ld_acquire_u32(counter) >= target) return true;
   const long long g0 = global_ns();
   while (true) {
@@ -327,7 +328,7 @@ __device__ __forceinline__ bool counter_wait(const unsigned* counter, unsigned t
     if (ld_acquire_u32(counter) >= target) return true;
     if (aborted(ab)) return false;
     const long long g1 = global_ns();
-    if (g1 - g0 > kWaitNs) {
+    if (g1 - g0 > limit_ns) {
       record_timeout(ab, ab.flag, 2u, g1 - g0);
       raise_abort(ab);
       return false;
