@@ -463,7 +463,8 @@ def run_ours(args, w, world, rank, local):
     stream = torch.cuda.current_stream()
     wk = work(w, fp8, fused)
     staged = w.dtype == "fp32" or w.d == 32
-    launches_per_step = 3 + (5 if staged else 0) + (4 if fp8 and w.T > 0 else 3 if fp8 else 0)
+    # state build, softmax (+ scan), readout; the fused readout has no readout launch
+    launches_per_step = (2 if fused else 3) + (5 if staged else 0) + (4 if fp8 and w.T > 0 else 3 if fp8 else 0)
     seq = KERNELS_FUSED if fused else KERNELS
 
     def one_call():
